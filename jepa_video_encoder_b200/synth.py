@@ -1,0 +1,327 @@
+"""Seeded synthetic inputs: model configurations, tensor tables and pixel clips.
+
+This module holds no step of the encoder's arithmetic.  It only *makes inputs*:
+
+* the five workload shapes of the JEPA model cards and benchmark pages
+  (ViT-Ti/14 LeWM image encoder, LeVJEPA ViT-L/16 block-causal video encoder,
+  V-JEPA 2 ViT-L/16 with its SSv2 attentive-pooler head, the same LeVJEPA
+  encoder with q4_0 matrices, and the 64-frame V-JEPA 2 long clip), plus small
+  shapes for tests;
+* a tensor table of seeded N(0, 0.02) weights named as in the "Quantization"
+  docs page, section "The rule" (``enc.blk.N.attn_qkv.weight`` ...), stored as
+  f32, f16, or in the ggml block formats q8_0 / q4_0 that the LeVJEPA and V-JEPA 2
+  model cards ship ("Files" tables);
+* seeded uint8 frames put through a per-channel mean/std normalisation, the way
+  the "jepa.cpp — measured benchmarks" page makes its synthetic input
+  (section "jepa.cpp — measured benchmarks", first paragraph).
+
+The block *quantiser* lives here because it only produces blocks; both the
+oracle and the CUDA path consume the identical bytes and dequantise them with
+their own code.  Random numbers come from numpy's PCG64 (``default_rng``).
+"""
+from __future__ import annotations
+
+import dataclasses
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional
+
+import numpy as np
+
+# dtype ids follow ggml's general.file_type / tensor type numbering
+# ("Quantization" page, section "The rule": 0 f32, 1 f16, 2 q4_0, 8 q8_0 ...)
+DT_F32, DT_F16, DT_Q4_0, DT_Q8_0 = 0, 1, 2, 8
+DTYPE_NAMES = {DT_F32: "f32", DT_F16: "f16", DT_Q4_0: "q4_0", DT_Q8_0: "q8_0"}
+DTYPE_IDS = {v: k for k, v in DTYPE_NAMES.items()}
+
+QK = 32                 # elements per q8_0 / q4_0 block
+Q8_0_BLOCK_BYTES = 34   # fp16 scale + 32 x int8
+Q4_0_BLOCK_BYTES = 18   # fp16 scale + 16 bytes of nibbles
+
+POOL_NONE, POOL_MEAN, POOL_CLS, POOL_ATTENTIVE = 0, 1, 2, 3
+POOL_IDS = {"none": POOL_NONE, "mean": POOL_MEAN, "cls": POOL_CLS, "attentive": POOL_ATTENTIVE}
+MASK_BIDIR, MASK_BLOCK_CAUSAL = 0, 1
+MASK_IDS = {"bidir": MASK_BIDIR, "block_causal": MASK_BLOCK_CAUSAL}
+
+IMAGENET_MEAN = (0.485, 0.456, 0.406)
+IMAGENET_STD = (0.229, 0.224, 0.225)
+
+
+@dataclass(frozen=True)
+class EncoderConfig:
+    """Shape of one JEPA ViT encoder (plus optional attentive head) workload."""
+    name: str
+    dim: int
+    depth: int
+    heads: int
+    mlp: int
+    patch: int
+    tubelet: int
+    img_h: int
+    img_w: int
+    frames: int
+    has_cls: bool
+    mask: str                 # "bidir" | "block_causal"
+    weights: str              # "f32" | "f16" | "q8_0" | "q4_0"
+    batch: int
+    pool: str                 # "none" | "mean" | "cls" | "attentive"
+    seed: int = 0
+    head_sa_blocks: int = 0
+    n_classes: int = 0
+    ln_eps: float = 1e-6
+    pix_mean: tuple = IMAGENET_MEAN
+    pix_std: tuple = IMAGENET_STD
+    random_ln_affine: bool = False   # tests: exercise gamma/beta instead of 1/0
+
+    # -- derived shapes ---------------------------------------------------
+    @property
+    def head_dim(self) -> int:
+        return self.dim // self.heads
+
+    @property
+    def patches_per_slot(self) -> int:        # P_f
+        return (self.img_h // self.patch) * (self.img_w // self.patch)
+
+    @property
+    def slots(self) -> int:                   # T' = T / tubelet
+        return self.frames // self.tubelet
+
+    @property
+    def n_patches(self) -> int:               # N_p
+        return self.slots * self.patches_per_slot
+
+    @property
+    def n_tokens(self) -> int:                # N
+        return self.n_patches + (1 if self.has_cls else 0)
+
+    @property
+    def patch_k(self) -> int:                 # 3 * kt * p * p
+        return 3 * self.tubelet * self.patch * self.patch
+
+    @property
+    def has_head(self) -> bool:
+        return self.n_classes > 0
+
+    def with_(self, **kw) -> "EncoderConfig":
+        return dataclasses.replace(self, **kw)
+
+
+# ---------------------------------------------------------------------------
+# The five workloads (model cards: LeWorldModel Push-T, LeVJEPA ViT-L/16,
+# V-JEPA 2 ViT-L/16 SSv2 classifier; benchmarks page: 64-frame long clip).
+# ---------------------------------------------------------------------------
+LEWM_VIT_TI = EncoderConfig(
+    name="lewm_vit_ti14_224_b1", dim=192, depth=12, heads=3, mlp=768, patch=14,
+    tubelet=1, img_h=224, img_w=224, frames=1, has_cls=True, mask="bidir",
+    weights="f32", batch=1, pool="cls", seed=0, pix_mean=(0.5, 0.5, 0.5),
+    pix_std=(0.5, 0.5, 0.5))
+LEVJEPA_VIT_L = EncoderConfig(
+    name="levjepa_vit_l16_16f224_b4", dim=1024, depth=24, heads=16, mlp=4096,
+    patch=16, tubelet=1, img_h=224, img_w=224, frames=16, has_cls=True,
+    mask="block_causal", weights="f16", batch=4, pool="cls", seed=1)
+VJEPA2_SSV2 = EncoderConfig(
+    name="vjepa2_vit_l16_16f256_ssv2_q8_b8", dim=1024, depth=24, heads=16,
+    mlp=4096, patch=16, tubelet=2, img_h=256, img_w=256, frames=16,
+    has_cls=False, mask="bidir", weights="q8_0", batch=8, pool="attentive",
+    seed=2, head_sa_blocks=3, n_classes=174)
+LEVJEPA_VIT_L_Q4 = LEVJEPA_VIT_L.with_(
+    name="levjepa_vit_l16_16f224_q4_b8", weights="q4_0", batch=8, pool="mean",
+    seed=3)
+VJEPA2_LONG = EncoderConfig(
+    name="vjepa2_vit_l16_64f256_b2", dim=1024, depth=24, heads=16, mlp=4096,
+    patch=16, tubelet=2, img_h=256, img_w=256, frames=64, has_cls=False,
+    mask="bidir", weights="f16", batch=2, pool="none", seed=4)
+
+WORKLOADS: Dict[str, EncoderConfig] = {
+    c.name: c for c in (LEWM_VIT_TI, LEVJEPA_VIT_L, VJEPA2_SSV2,
+                        LEVJEPA_VIT_L_Q4, VJEPA2_LONG)}
+
+
+def small_config(base: EncoderConfig, **kw) -> EncoderConfig:
+    """A shrunk copy of a workload that the oracle runs in seconds."""
+    d = dict(dim=256, depth=2, heads=4, mlp=1024, img_h=64, img_w=64,
+             frames=min(base.frames, 4), batch=2, random_ln_affine=True)
+    if base.tubelet == 2:
+        d["frames"] = 4
+    d.update(kw)
+    return base.with_(name=base.name + "_small", **d)
+
+
+# ---------------------------------------------------------------------------
+# Tensor table
+# ---------------------------------------------------------------------------
+@dataclass
+class Tensor:
+    """One entry of the tensor table: PyTorch-order shape ([out, in] for a
+    matrix), a ggml dtype id and the raw bytes as a contiguous numpy array
+    (float32 / float16 values, or uint8 block bytes for q8_0 / q4_0)."""
+    name: str
+    dtype: int
+    shape: tuple
+    data: np.ndarray
+
+    @property
+    def nbytes(self) -> int:
+        return int(self.data.nbytes)
+
+
+# Matrices the "Quantization" page (section "The rule") re-types.
+_RETYPED_SUFFIXES = ("attn_qkv.weight", "attn_out.weight", "ffn_up.weight",
+                     "ffn_down.weight", "head.xattn.q.weight",
+                     "head.xattn.k.weight", "head.xattn.v.weight",
+                     "head.xattn.out.weight", "head.cls.weight")
+
+
+def is_retyped(name: str) -> bool:
+    return name.endswith(_RETYPED_SUFFIXES)
+
+
+def _block_names(prefix: str, D: int, M: int) -> List[tuple]:
+    return [
+        (prefix + "ln1.weight", (D,), "ln_g"), (prefix + "ln1.bias", (D,), "ln_b"),
+        (prefix + "attn_qkv.weight", (3 * D, D), "w"),
+        (prefix + "attn_qkv.bias", (3 * D,), "b"),
+        (prefix + "attn_out.weight", (D, D), "w"), (prefix + "attn_out.bias", (D,), "b"),
+        (prefix + "ln2.weight", (D,), "ln_g"), (prefix + "ln2.bias", (D,), "ln_b"),
+        (prefix + "ffn_up.weight", (M, D), "w"), (prefix + "ffn_up.bias", (M,), "b"),
+        (prefix + "ffn_down.weight", (D, M), "w"), (prefix + "ffn_down.bias", (D,), "b"),
+    ]
+
+
+def tensor_specs(cfg: EncoderConfig, with_pos: bool = True) -> List[tuple]:
+    """(name, shape, kind) in table order."""
+    D, M, kt, p = cfg.dim, cfg.mlp, cfg.tubelet, cfg.patch
+    s = [("enc.patch_embed.weight", (D, 3, kt, p, p), "w"),
+         ("enc.patch_embed.bias", (D,), "b")]
+    if with_pos:
+        s.append(("enc.pos_embed", (cfg.n_tokens, D), "w"))
+    if cfg.has_cls:
+        s.append(("enc.cls_token", (D,), "w"))
+    for i in range(cfg.depth):
+        s += _block_names(f"enc.blk.{i}.", D, M)
+    s += [("enc.norm.weight", (D,), "ln_g"), ("enc.norm.bias", (D,), "ln_b")]
+    if cfg.has_head:
+        for i in range(cfg.head_sa_blocks):
+            s += _block_names(f"head.blk.{i}.", D, M)
+        s += [("head.query", (D,), "w"),
+              ("head.ln_kv.weight", (D,), "ln_g"), ("head.ln_kv.bias", (D,), "ln_b")]
+        for t in ("q", "k", "v", "out"):
+            s += [(f"head.xattn.{t}.weight", (D, D), "w"), (f"head.xattn.{t}.bias", (D,), "b")]
+        s += [("head.xattn.ln2.weight", (D,), "ln_g"), ("head.xattn.ln2.bias", (D,), "ln_b"),
+              ("head.xattn.ffn_up.weight", (M, D), "w"), ("head.xattn.ffn_up.bias", (M,), "b"),
+              ("head.xattn.ffn_down.weight", (D, M), "w"), ("head.xattn.ffn_down.bias", (D,), "b"),
+              ("head.cls.weight", (cfg.n_classes, D), "w"),
+              ("head.cls.bias", (cfg.n_classes,), "b")]
+    return s
+
+
+def quantize_q8_0(x: np.ndarray) -> np.ndarray:
+    """Rows of float values -> q8_0 blocks (uint8 [..., K/32 * 34]).
+
+    Per 32-element block: amax = max|x|, d = amax/127, q = round-half-away(x/d)
+    clamped to [-127, 127], d stored as IEEE binary16 (round to nearest even),
+    then 32 int8.  An all-zero block gets d = 0, q = 0."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    lead, K = x.shape[:-1], x.shape[-1]
+    assert K % QK == 0, "q8_0 needs the row length to be a multiple of 32"
+    b = x.reshape(-1, QK)
+    amax = np.abs(b).max(axis=1)
+    d = (amax / np.float32(127.0)).astype(np.float32)
+    inv = np.where(d > 0, np.float32(1.0) / np.where(d > 0, d, 1), 0).astype(np.float32)
+    v = b * inv[:, None]
+    q = np.trunc(v + np.copysign(np.float32(0.5), v))
+    q = np.clip(q, -127, 127).astype(np.int8)
+    out = np.empty((b.shape[0], Q8_0_BLOCK_BYTES), np.uint8)
+    out[:, 0:2] = d.astype(np.float16).view(np.uint8).reshape(-1, 2)
+    out[:, 2:] = q.view(np.uint8)
+    return out.reshape(*lead, (K // QK) * Q8_0_BLOCK_BYTES)
+
+
+def quantize_q4_0(x: np.ndarray) -> np.ndarray:
+    """Rows of float values -> q4_0 blocks (uint8 [..., K/32 * 18]).
+
+    Per block: m = the element of largest magnitude (first on ties), d = m/-8,
+    q = min(15, floor(x/d + 8.5)), value (q-8)*d; d stored as binary16.  Byte j
+    of the 16 nibble bytes holds element j in its low and element j+16 in its
+    high nibble (ggml's q4_0 packing)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    lead, K = x.shape[:-1], x.shape[-1]
+    assert K % QK == 0, "q4_0 needs the row length to be a multiple of 32"
+    b = x.reshape(-1, QK)
+    idx = np.argmax(np.abs(b), axis=1)
+    m = b[np.arange(b.shape[0]), idx]
+    d = (m / np.float32(-8.0)).astype(np.float32)
+    inv = np.where(d != 0, np.float32(1.0) / np.where(d != 0, d, 1), 0).astype(np.float32)
+    q = np.floor(b * inv[:, None] + np.float32(8.5))
+    q = np.clip(q, 0, 15).astype(np.uint8)
+    out = np.empty((b.shape[0], Q4_0_BLOCK_BYTES), np.uint8)
+    out[:, 0:2] = d.astype(np.float16).view(np.uint8).reshape(-1, 2)
+    out[:, 2:] = q[:, :16] | (q[:, 16:] << 4)
+    return out.reshape(*lead, (K // QK) * Q4_0_BLOCK_BYTES)
+
+
+def _store(name: str, shape: tuple, vals: np.ndarray, wdt: str) -> Tensor:
+    if wdt in ("q8_0", "q4_0") and is_retyped(name) and shape[-1] % QK == 0:
+        q = quantize_q8_0(vals) if wdt == "q8_0" else quantize_q4_0(vals)
+        return Tensor(name, DTYPE_IDS[wdt], shape, np.ascontiguousarray(q))
+    if wdt == "f32":
+        return Tensor(name, DT_F32, shape, np.ascontiguousarray(vals, np.float32))
+    return Tensor(name, DT_F16, shape, np.ascontiguousarray(vals.astype(np.float16)))
+
+
+def make_tensor_table(cfg: EncoderConfig, seed: Optional[int] = None,
+                      std: float = 0.02) -> List[Tensor]:
+    """Seeded tensor table: weights, biases, pos_embed, cls, query ~ N(0, std);
+    LayerNorm gamma = 1, beta = 0 (or, with ``random_ln_affine``, gamma ~
+    1 + N(0, 0.1) and beta ~ N(0, 0.02)).  Tensors are drawn in table order
+    from one PCG64 stream."""
+    rng = np.random.default_rng(cfg.seed if seed is None else seed)
+    table = []
+    for name, shape, kind in tensor_specs(cfg):
+        if kind == "ln_g":
+            v = (np.float32(1.0) + np.float32(0.1) * rng.standard_normal(shape, dtype=np.float32)
+                 if cfg.random_ln_affine else np.ones(shape, np.float32))
+        elif kind == "ln_b":
+            v = (np.float32(std) * rng.standard_normal(shape, dtype=np.float32)
+                 if cfg.random_ln_affine else np.zeros(shape, np.float32))
+        else:
+            v = np.float32(std) * rng.standard_normal(shape, dtype=np.float32)
+        table.append(_store(name, shape, v, cfg.weights))
+    return table
+
+
+def table_dict(table: List[Tensor]) -> Dict[str, Tensor]:
+    return {t.name: t for t in table}
+
+
+def make_pixels(cfg: EncoderConfig, batch: Optional[int] = None,
+                seed: Optional[int] = None) -> np.ndarray:
+    """Seeded uint8 frames [B, T, 3, H, W] normalised per channel:
+    (x/255 - mean[c]) / std[c], as float32."""
+    B = cfg.batch if batch is None else batch
+    rng = np.random.default_rng((cfg.seed if seed is None else seed) + 1000)
+    u8 = rng.integers(0, 256, size=(B, cfg.frames, 3, cfg.img_h, cfg.img_w), dtype=np.uint8)
+    mean = np.asarray(cfg.pix_mean, np.float32).reshape(1, 1, 3, 1, 1)
+    sd = np.asarray(cfg.pix_std, np.float32).reshape(1, 1, 3, 1, 1)
+    return np.ascontiguousarray((u8.astype(np.float32) / np.float32(255.0) - mean) / sd)
+
+
+def param_count(cfg: EncoderConfig, with_pos: bool = False) -> int:
+    """Number of parameters of the encoder (and head) tensors."""
+    return int(sum(int(np.prod(s)) for _, s, _ in tensor_specs(cfg, with_pos=with_pos)))
+
+
+def table_bytes(cfg: EncoderConfig, wdt: str, with_pos: bool = False,
+                rest: str = "f32") -> int:
+    """Bytes of the tensor data with the re-typed matrices stored as ``wdt``
+    and every other tensor as ``rest``."""
+    per = {"f32": 4, "f16": 2}
+    total = 0
+    for name, shape, _ in tensor_specs(cfg, with_pos=with_pos):
+        n = int(np.prod(shape))
+        if wdt in ("q8_0", "q4_0") and is_retyped(name):
+            total += n // QK * (Q8_0_BLOCK_BYTES if wdt == "q8_0" else Q4_0_BLOCK_BYTES)
+        elif wdt in per and is_retyped(name):
+            total += n * per[wdt]
+        else:
+            total += n * per[rest]
+    return total

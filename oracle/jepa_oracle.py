@@ -1,0 +1,338 @@
+"""Oracle: a plain, slow, float64 CPU forward of the JEPA ViT encoder.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports this module;
+only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may call it.  It shares no code with
+the CUDA path: it reads the same seeded tensor table and pixels and nothing
+else.
+
+Every step is the textbook definition written out in numpy float64 (library
+matmul as the only primitive), in the order the pages describe the model:
+
+* tubelet patch-embed: a conv with stride = kernel, i.e. unfold + matmul
+  (model cards "LeVJEPA ViT-L/16" and "V-JEPA 2 ViT-L/16 SSv2 classifier":
+  patch 16, tubelet 1 / 2; benchmarks page, "What the milliseconds are": the
+  engine unfolds patches before the graph);
+* an additive positional table and a CLS row where the model has one
+  ("LeVJEPA" card, intro; "Quantization" page, "The rule": enc.pos_embed,
+  enc.cls_token);
+* pre-LN blocks ln1 -> attn_qkv -> attention -> attn_out -> +res, ln2 ->
+  ffn_up -> GELU -> ffn_down -> +res ("Quantization" page, "The rule": the
+  tensor set of a block);
+* the block-causal mask of LeVJEPA: bidirectional inside a frame, causal
+  across frames, CLS a read-only sink ("LeVJEPA" card, intro);
+* the final ``norm`` before last_hidden_state ("Quantization" page, "Reading
+  the numbers");
+* pooling mean / cls / none ("LeVJEPA" card, "Run it": --pool) and the
+  attentive-pool classifier: 3 self-attention blocks over the tokens, one
+  cross-attention query, MLP, linear ("jepa.cpp — measured benchmarks",
+  "Attentive-pool head");
+* q8_0 / q4_0 dequantisation: value = q*d and (q-8)*d per 32-element block
+  with one fp16 scale ("Quantization" page, "File sizes": 8.5 / 4.5 bits per
+  weight).
+
+Readings where the pages are silent (LayerNorm eps, exact-erf GELU, 1/sqrt(d_h)
+scale, qkv column order, mean pooling over patch tokens only, the head's
+cross-attention out-projection) are listed in the design notes and are passed
+in through the config.
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Iterable, Optional, Sequence
+
+import numpy as np
+from scipy.special import erf as _erf
+
+# ggml dtype ids (the tensor table's own numbering)
+DT_F32, DT_F16, DT_Q4_0, DT_Q8_0 = 0, 1, 2, 8
+
+
+# ---------------------------------------------------------------------------
+# Weight decoding
+# ---------------------------------------------------------------------------
+def _f16_bits_to_f64(lo: np.ndarray, hi: np.ndarray) -> np.ndarray:
+    """IEEE binary16 (little-endian byte pair) -> float64, decoded from the
+    bit fields: sign, 5-bit exponent (bias 15), 10-bit fraction."""
+    bits = lo.astype(np.uint32) | (hi.astype(np.uint32) << 8)
+    sign = np.where(bits >> 15, -1.0, 1.0)
+    e = ((bits >> 10) & 0x1F).astype(np.int64)
+    f = (bits & 0x3FF).astype(np.float64)
+    normal = sign * np.ldexp(1.0 + f / 1024.0, e - 15)
+    sub = sign * np.ldexp(f / 1024.0, -14)
+    out = np.where(e == 0, sub, normal)
+    out = np.where(e == 31, np.where(f == 0, sign * np.inf, np.nan), out)
+    return out
+
+
+def dequant_q8_0(blocks: np.ndarray, n: int) -> np.ndarray:
+    """q8_0: each 34-byte block = fp16 scale d, then 32 signed bytes q;
+    element value q*d."""
+    b = np.asarray(blocks, np.uint8).reshape(-1, 34)
+    d = _f16_bits_to_f64(b[:, 0], b[:, 1])
+    q = b[:, 2:].view(np.int8).astype(np.float64)
+    out = (q * d[:, None]).reshape(-1)
+    assert out.size == n
+    return out
+
+
+def dequant_q4_0(blocks: np.ndarray, n: int) -> np.ndarray:
+    """q4_0: each 18-byte block = fp16 scale d, then 16 bytes; byte j carries
+    element j (low nibble) and element j+16 (high nibble); value (q-8)*d."""
+    b = np.asarray(blocks, np.uint8).reshape(-1, 18)
+    d = _f16_bits_to_f64(b[:, 0], b[:, 1])
+    nib = b[:, 2:]
+    q = np.empty((b.shape[0], 32), np.float64)
+    q[:, :16] = (nib & 0x0F).astype(np.float64)
+    q[:, 16:] = (nib >> 4).astype(np.float64)
+    out = ((q - 8.0) * d[:, None]).reshape(-1)
+    assert out.size == n
+    return out
+
+
+def tensor_f64(t) -> np.ndarray:
+    """A tensor-table entry -> float64 values in its PyTorch-order shape."""
+    shape = tuple(t.shape)
+    n = int(np.prod(shape))
+    if t.dtype == DT_F32:
+        return np.asarray(t.data, np.float32).astype(np.float64).reshape(shape)
+    if t.dtype == DT_F16:
+        raw = np.ascontiguousarray(t.data).view(np.uint8).reshape(-1, 2)
+        return _f16_bits_to_f64(raw[:, 0], raw[:, 1]).reshape(shape)
+    if t.dtype == DT_Q8_0:
+        return dequant_q8_0(t.data, n).reshape(shape)
+    if t.dtype == DT_Q4_0:
+        return dequant_q4_0(t.data, n).reshape(shape)
+    raise ValueError(f"unknown dtype {t.dtype} for {t.name}")
+
+
+def weights_f64(table) -> Dict[str, np.ndarray]:
+    return {t.name: tensor_f64(t) for t in table}
+
+
+# ---------------------------------------------------------------------------
+# Building blocks (each the plain definition)
+# ---------------------------------------------------------------------------
+def patchify(pixels: np.ndarray, patch: int, tubelet: int) -> np.ndarray:
+    """[B, T, 3, H, W] -> [B, N_p, 3*kt*p*p].  Token order: time slot t',
+    then patch row, then patch column.  Vector order (c, dt, kh, kw), the
+    row-major flattening of a conv weight [D, 3, kt, p, p]."""
+    B, T, C, H, W = pixels.shape
+    kt, p = tubelet, patch
+    x = np.asarray(pixels, np.float64).reshape(B, T // kt, kt, C, H // p, p, W // p, p)
+    # axes: b, t', dt, c, hp, kh, wp, kw  ->  b, t', hp, wp, c, dt, kh, kw
+    x = x.transpose(0, 1, 4, 6, 3, 2, 5, 7)
+    return x.reshape(B, (T // kt) * (H // p) * (W // p), C * kt * p * p)
+
+
+def patch_embed(pixels, w_pe, b_pe, patch, tubelet) -> np.ndarray:
+    """Conv3d with stride = kernel = (kt, p, p) written as unfold + matmul."""
+    cols = patchify(pixels, patch, tubelet)
+    D = w_pe.shape[0]
+    return cols @ w_pe.reshape(D, -1).T + b_pe
+
+
+def layer_norm(x: np.ndarray, gamma, beta, eps: float) -> np.ndarray:
+    """(x - mean) / sqrt(var + eps) * gamma + beta over the last axis, with
+    the biased variance."""
+    x = np.asarray(x, np.float64)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * gamma + beta
+
+
+def gelu(x: np.ndarray) -> np.ndarray:
+    """Exact GELU: x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2))."""
+    return 0.5 * x * (1.0 + _erf(x / math.sqrt(2.0)))
+
+
+def linear(x, w, b) -> np.ndarray:
+    """y = x W^T + b with W in PyTorch [out, in] order."""
+    y = np.asarray(x, np.float64) @ w.T
+    return y + b if b is not None else y
+
+
+def allowed_keys(n_patches: int, patches_per_slot: int, has_cls: bool,
+                 mask: str) -> np.ndarray:
+    """Boolean [N, N]: may query i read key j?
+
+    bidir: every pair.  block_causal (LeVJEPA): a patch of time slot s reads
+    the patches of slots <= s (bidirectional inside a slot, causal across
+    slots); the CLS row, when present, reads every token including itself and
+    no patch reads CLS (the read-only sink)."""
+    c = 1 if has_cls else 0
+    N = n_patches + c
+    if mask == "bidir":
+        return np.ones((N, N), bool)
+    if mask != "block_causal":
+        raise ValueError(mask)
+    slot = np.arange(n_patches) // patches_per_slot
+    allow = np.zeros((N, N), bool)
+    allow[c:, c:] = slot[None, :] <= slot[:, None]
+    if has_cls:
+        allow[0, :] = True
+    return allow
+
+
+def attention(q, k, v, allow: Optional[np.ndarray]) -> np.ndarray:
+    """softmax(q k^T / sqrt(d) + mask) v for q [.., Nq, d], k/v [.., Nk, d];
+    ``allow`` [Nq, Nk] boolean (None = every pair).  The row max is
+    subtracted before exp (exact in the softmax's definition)."""
+    d = q.shape[-1]
+    s = (q @ np.swapaxes(k, -1, -2)) / math.sqrt(d)
+    if allow is not None:
+        s = np.where(allow, s, -np.inf)
+    s = s - s.max(axis=-1, keepdims=True)
+    e = np.exp(s)
+    p = e / e.sum(axis=-1, keepdims=True)
+    return p @ v
+
+
+def split_heads(x, heads):
+    """[B, N, h*d] -> [B, h, N, d]  (head hd owns columns hd*d .. hd*d+d-1)."""
+    B, N, C = x.shape
+    return x.reshape(B, N, heads, C // heads).transpose(0, 2, 1, 3)
+
+
+def merge_heads(x):
+    B, h, N, d = x.shape
+    return x.transpose(0, 2, 1, 3).reshape(B, N, h * d)
+
+
+def block(x, W: Dict[str, np.ndarray], prefix: str, heads: int, eps: float,
+          allow: Optional[np.ndarray]) -> np.ndarray:
+    """One pre-LN transformer block.  attn_qkv's output columns are
+    [q | k | v], each head-major (head hd at hd*d_h ...)."""
+    D = x.shape[-1]
+    y = layer_norm(x, W[prefix + "ln1.weight"], W[prefix + "ln1.bias"], eps)
+    qkv = linear(y, W[prefix + "attn_qkv.weight"], W[prefix + "attn_qkv.bias"])
+    q, k, v = (split_heads(qkv[..., i * D:(i + 1) * D], heads) for i in range(3))
+    o = merge_heads(attention(q, k, v, allow))
+    x = x + linear(o, W[prefix + "attn_out.weight"], W[prefix + "attn_out.bias"])
+    y = layer_norm(x, W[prefix + "ln2.weight"], W[prefix + "ln2.bias"], eps)
+    h = gelu(linear(y, W[prefix + "ffn_up.weight"], W[prefix + "ffn_up.bias"]))
+    return x + linear(h, W[prefix + "ffn_down.weight"], W[prefix + "ffn_down.bias"])
+
+
+def embed(cfg, W, pixels) -> np.ndarray:
+    """Patch-embed, prepend CLS (when the model has one), add pos_embed."""
+    x = patch_embed(pixels, W["enc.patch_embed.weight"], W["enc.patch_embed.bias"],
+                    cfg.patch, cfg.tubelet)
+    if cfg.has_cls:
+        cls = np.broadcast_to(W["enc.cls_token"], (x.shape[0], 1, x.shape[-1]))
+        x = np.concatenate([cls, x], axis=1)
+    return x + W["enc.pos_embed"][None]
+
+
+def encoder_allow(cfg) -> Optional[np.ndarray]:
+    if cfg.mask == "bidir":
+        return None
+    return allowed_keys(cfg.n_patches, cfg.patches_per_slot, cfg.has_cls, cfg.mask)
+
+
+def encoder(cfg, W, pixels, layers: Optional[int] = None,
+            return_residuals: bool = False):
+    """Full encoder: embed, ``depth`` blocks, final LayerNorm ->
+    last_hidden_state [B, N, D]."""
+    allow = encoder_allow(cfg)
+    x = embed(cfg, W, pixels)
+    res = [x]
+    for i in range(cfg.depth if layers is None else layers):
+        x = block(x, W, f"enc.blk.{i}.", cfg.heads, cfg.ln_eps, allow)
+        res.append(x)
+    y = layer_norm(x, W["enc.norm.weight"], W["enc.norm.bias"], cfg.ln_eps)
+    return (y, res) if return_residuals else y
+
+
+def pool(cfg, y: np.ndarray, mode: str) -> np.ndarray:
+    """cls: the CLS row; mean: mean over the patch tokens (CLS excluded);
+    none: the full token map."""
+    if mode == "none":
+        return y
+    if mode == "cls":
+        if not cfg.has_cls:
+            raise ValueError("cls pooling needs a CLS token")
+        return y[:, 0]
+    if mode == "mean":
+        return y[:, 1 if cfg.has_cls else 0:].mean(axis=1)
+    raise ValueError(mode)
+
+
+def attentive_head(cfg, W, tokens: np.ndarray) -> np.ndarray:
+    """Attentive-pool classifier: ``head_sa_blocks`` pre-LN self-attention
+    blocks over the tokens, then one cross-attention block whose single query
+    is the learned ``head.query`` (not normalised): q = W_q query + b_q;
+    k, v = W_{k,v} LN_kv(tokens) + b; z = query + W_out attn + b_out;
+    z += MLP(LN2(z)); logits = W_cls z + b_cls."""
+    x = tokens
+    for i in range(cfg.head_sa_blocks):
+        x = block(x, W, f"head.blk.{i}.", cfg.heads, cfg.ln_eps, None)
+    B, N, D = x.shape
+    kv_in = layer_norm(x, W["head.ln_kv.weight"], W["head.ln_kv.bias"], cfg.ln_eps)
+    qv = linear(W["head.query"][None, None, :], W["head.xattn.q.weight"], W["head.xattn.q.bias"])
+    qv = np.broadcast_to(qv, (B, 1, D))
+    k = linear(kv_in, W["head.xattn.k.weight"], W["head.xattn.k.bias"])
+    v = linear(kv_in, W["head.xattn.v.weight"], W["head.xattn.v.bias"])
+    o = merge_heads(attention(split_heads(qv, cfg.heads), split_heads(k, cfg.heads),
+                              split_heads(v, cfg.heads), None))
+    z = W["head.query"][None, None, :] + linear(o, W["head.xattn.out.weight"],
+                                                W["head.xattn.out.bias"])
+    h = layer_norm(z, W["head.xattn.ln2.weight"], W["head.xattn.ln2.bias"], cfg.ln_eps)
+    h = gelu(linear(h, W["head.xattn.ffn_up.weight"], W["head.xattn.ffn_up.bias"]))
+    z = z + linear(h, W["head.xattn.ffn_down.weight"], W["head.xattn.ffn_down.bias"])
+    return linear(z[:, 0], W["head.cls.weight"], W["head.cls.bias"])
+
+
+def forward(cfg, W, pixels, pool_mode: Optional[str] = None) -> np.ndarray:
+    """Encoder + output selected by ``pool_mode`` (default: the config's)."""
+    mode = cfg.pool if pool_mode is None else pool_mode
+    y = encoder(cfg, W, pixels)
+    if mode == "attentive":
+        return attentive_head(cfg, W, y)
+    return pool(cfg, y, mode)
+
+
+# ---------------------------------------------------------------------------
+# Sampled rows of one block: the block's output for chosen query rows of one
+# clip, given that clip's block input.  Same definitions, evaluated only where
+# needed (K and V still come from every row).
+# ---------------------------------------------------------------------------
+def block_rows(x_clip: np.ndarray, W, prefix: str, heads: int, eps: float,
+               allow: Optional[np.ndarray], rows: Sequence[int]) -> np.ndarray:
+    rows = np.asarray(rows)
+    N, D = x_clip.shape
+    y = layer_norm(x_clip, W[prefix + "ln1.weight"], W[prefix + "ln1.bias"], eps)
+    wqkv, bqkv = W[prefix + "attn_qkv.weight"], W[prefix + "attn_qkv.bias"]
+    q = linear(y[rows], wqkv[:D], bqkv[:D])
+    k = linear(y, wqkv[D:2 * D], bqkv[D:2 * D])
+    v = linear(y, wqkv[2 * D:], bqkv[2 * D:])
+    qh, kh, vh = (split_heads(t[None], heads)[0] for t in (q, k, v))
+    o = merge_heads(attention(qh, kh, vh, None if allow is None else allow[rows])[None])[0]
+    xr = x_clip[rows] + linear(o, W[prefix + "attn_out.weight"], W[prefix + "attn_out.bias"])
+    y2 = layer_norm(xr, W[prefix + "ln2.weight"], W[prefix + "ln2.bias"], eps)
+    h = gelu(linear(y2, W[prefix + "ffn_up.weight"], W[prefix + "ffn_up.bias"]))
+    return xr + linear(h, W[prefix + "ffn_down.weight"], W[prefix + "ffn_down.bias"])
+
+
+# ---------------------------------------------------------------------------
+# Comparison metrics ("Quantization" page, "How the accuracy was measured")
+# ---------------------------------------------------------------------------
+def token_cosines(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    a = np.asarray(a, np.float64).reshape(-1, a.shape[-1])
+    b = np.asarray(b, np.float64).reshape(-1, b.shape[-1])
+    num = (a * b).sum(-1)
+    den = np.sqrt((a * a).sum(-1) * (b * b).sum(-1))
+    return np.where(den > 0, num / np.where(den > 0, den, 1), 1.0)
+
+
+def rel_max(a, b) -> float:
+    """max|a-b| / max|b| with b the reference."""
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.abs(a - b).max() / max(np.abs(b).max(), 1e-300))
+
+
+def rel_fro(a, b) -> float:
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
