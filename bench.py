@@ -1,0 +1,369 @@
+"""Benchmark of the JEPA ViT encoder forward on B200.
+
+One step = one forward of one batch of the workload through jepa_b200_encode
+(patch-embed, all blocks, final norm, pooling), inputs resident in HBM.
+Default workload: LeVJEPA ViT-L/16, 16 frames 224^2 (3137 tokens with the CLS
+sink), block-causal mask, f16 weights, batch 4, CLS output.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+Prints one JSON line (rank 0).  Multi-GPU runs are replicas (one process per
+GPU via torchrun; each GPU encodes its own batch; no data-path collective).
+The reference arm times the float64 CPU oracle on the host cores on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import glob
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from jepa_video_encoder_b200 import synth  # noqa: E402
+
+METRIC = "ViT-L/16 encoder tokens/s & clips/s on 1 B200; % of dense f16/bf16 TC peak"
+DEFAULT_WORKLOAD = synth.LEVJEPA_VIT_L.name
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def _flops(cfg) -> dict:
+    """Algorithmic FLOPs per clip by kernel class (attention counts only the
+    allowed query/key pairs of the mask)."""
+    import numpy as np
+    N, D, M, L = cfg.n_tokens, cfg.dim, cfg.mlp, cfg.depth
+    if cfg.mask == "block_causal":
+        pf, c = cfg.patches_per_slot, (1 if cfg.has_cls else 0)
+        slots = np.arange(cfg.n_patches) // pf
+        pairs = int(((slots + 1) * pf).sum()) + (N if c else 0)
+    else:
+        pairs = N * N
+    f = {
+        "patch_embed": 2.0 * cfg.n_patches * cfg.patch_k * D,
+        "gemm_qkv": 2.0 * N * D * 3 * D * L,
+        "attention": 4.0 * pairs * D * L,
+        "gemm_out": 2.0 * N * D * D * L,
+        "gemm_up": 2.0 * N * D * M * L,
+        "gemm_down": 2.0 * N * M * D * L,
+    }
+    if cfg.has_head:
+        f["head"] = cfg.head_sa_blocks * (24.0 * N * D * D + 4.0 * N * N * D) + 4.0 * N * D * D
+    return f
+
+
+def _clock_sampler_start(path):
+    q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    try:
+        f = open(path, "w")
+        return subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200"],
+                                stdout=f, stderr=subprocess.DEVNULL), f
+    except Exception:
+        return None, None
+
+
+def _clock_sampler_stop(proc, fh, path, gpu_index):
+    if proc is None:
+        return None
+    proc.terminate()
+    try:
+        proc.wait(timeout=5)
+    except Exception:
+        proc.kill()
+    fh.close()
+    sm, mx, reasons = [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in open(path):
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9 or parts[0] != str(gpu_index):
+            continue
+        try:
+            sm.append(float(parts[1]))
+            mx.append(float(parts[2]))
+        except ValueError:
+            continue
+        for n, v in zip(names, parts[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    if not sm:
+        return None
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+            "samples": len(sm)}
+
+
+def _src_hash():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "jepa_video_encoder_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(kernel_class, cfg_name):
+    """DRAM bytes per launch of a kernel class from the committed ncu summary
+    (profiles/traffic.txt), valid only for the kernel sources it was taken on."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    src = _src_hash()
+    for line in open(p):
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel_class and parts[1] == cfg_name \
+                and parts[2] == src:
+            return float(parts[3])
+    return None
+
+
+def cpu_oracle_sample(cfg, target_s: float = 12.0):
+    """Time the float64 oracle on a bounded sample of one clip: patch-embed
+    and as many blocks as fit in ~target_s, extrapolated to the full depth."""
+    import numpy as np
+    from oracle import jepa_oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    table = synth.table_dict(synth.make_tensor_table(cfg))
+    pix = synth.make_pixels(cfg, batch=1).astype(np.float64)
+    names = [n for n in table if not n.startswith("enc.blk.") and not n.startswith("head.")]
+    W = {n: orc.tensor_f64(table[n]) for n in names}
+    t0 = time.perf_counter()
+    x = orc.embed(cfg, W, pix)
+    t_embed = time.perf_counter() - t0
+    allow = orc.encoder_allow(cfg)
+    blocks, t_blocks = 0, 0.0
+    while blocks < cfg.depth and t_blocks < target_s:
+        pre = f"enc.blk.{blocks}."
+        for n in table:
+            if n.startswith(pre):
+                W[n] = orc.tensor_f64(table[n])
+        t1 = time.perf_counter()
+        x = orc.block(x, W, pre, cfg.heads, cfg.ln_eps, allow)
+        t_blocks += time.perf_counter() - t1
+        blocks += 1
+    t2 = time.perf_counter()
+    orc.layer_norm(x, W["enc.norm.weight"], W["enc.norm.bias"], cfg.ln_eps)
+    t_norm = time.perf_counter() - t2
+    t_clip = t_embed + cfg.depth * (t_blocks / blocks) + t_norm
+    return {"value": cfg.n_tokens / t_clip, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "clips_per_s": 1.0 / t_clip,
+            "sample": f"1 clip: patch-embed + {blocks} of {cfg.depth} blocks + final norm in float64 numpy, "
+                      f"block time extrapolated to {cfg.depth} blocks ({t_embed + t_blocks + t_norm:.1f} s of CPU work)"}
+
+
+def run_reference(args, cfg, rank, world):
+    if rank != 0:
+        return 0
+    steps = []
+    sample = None
+    for _ in range(max(1, args.steps)):
+        sample = cpu_oracle_sample(cfg, target_s=max(2.0, 60.0 / max(1, args.steps)))
+        steps.append(sample["value"])
+    v = statistics.median(steps)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * cfg.n_tokens * cfg.batch / v,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "batch": cfg.batch, "tokens_per_clip": cfg.n_tokens},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": sample["cores"], "kind": "oracle",
+                             "sample": sample["sample"]},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, cfg, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import jepa_video_encoder_b200 as jb
+    from jepa_video_encoder_b200 import build as jbuild
+
+    if rank == 0 or not os.path.exists(jbuild.LIB):
+        jbuild.build()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    table = synth.make_tensor_table(cfg)
+    pix_np = synth.make_pixels(cfg)
+    model = jb.Model(cfg, table, device=local_rank)
+    pixels = torch.from_numpy(pix_np).to(dev)
+    out = torch.empty(model.out_shape(cfg.batch, cfg.pool), dtype=torch.float32, device=dev)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MiB > L2
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        model.encode(pixels, pool=cfg.pool, out=out, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if model.sync_status(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    # ---- timed region: K steps, each between CUDA events, L2 flushed between steps
+    clock_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv") if os.path.isdir(
+        os.path.join(ROOT, "gpurun_out")) else f"/tmp/jepa_clocks_rank{rank}.csv"
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    proc, fh = _clock_sampler_start(clock_path)
+    time.sleep(0.3)
+    launches = 0
+    for k in range(args.steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        step()
+        ev[k][1].record(stream)
+        launches += model.last_launch_count()
+    torch.cuda.synchronize(dev)
+    clocks = _clock_sampler_stop(proc, fh, clock_path, local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    if model.sync_status(stream) != 0:
+        raise RuntimeError("device error in the timed region")
+    ms_steps = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(ms_steps)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens = world * cfg.batch * cfg.n_tokens * args.steps
+    value = tokens / (total_ms / 1000.0)
+
+    # ---- per-kernel timing pass (event pairs around every launch)
+    model.set_profiling(True)
+    prof = {k: [0.0, 0] for k in jb._abi.KERNEL_CLASSES}
+    for k in range(args.steps):
+        flush.zero_()
+        step()
+        for kc, (ms, n) in model.profile_read().items():
+            prof[kc][0] += ms
+            prof[kc][1] += n
+    model.set_profiling(False)
+
+    # ---- end to end through the public API from pinned host memory
+    pix_host = torch.from_numpy(pix_np).pin_memory()
+    out_host = torch.empty(tuple(out.shape), dtype=torch.float32).pin_memory()
+    for _ in range(2):
+        model.encode_host(pix_host, pool=cfg.pool, out=out_host, stream=stream)
+    e2e_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        model.encode_host(pix_host, pool=cfg.pool, out=out_host, stream=stream)
+        b.record(stream)
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    te = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+    e2e_value = tokens / (float(te.item()) / 1000.0)
+
+    if rank != 0:
+        model.close()
+        return 0
+
+    peaks, peak_src = _peaks()
+    fl = _flops(cfg)
+    B = cfg.batch
+    total_flop = B * sum(fl.values())
+    tflops = total_flop / (ms_per_step / 1000.0) / 1e12
+    # dominant kernel class by measured time
+    per_class = {k: v for k, v in prof.items() if v[1] > 0}
+    dom = max(per_class, key=lambda k: per_class[k][0])
+    dom_ms, dom_n = per_class[dom]
+    avg_ms = dom_ms / dom_n
+    if dom in fl:
+        per_launch = B * fl[dom] / (cfg.depth if dom.startswith("gemm") or dom == "attention" else 1)
+        achieved = per_launch / (avg_ms / 1000.0) / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": _traffic(dom, cfg.name),
+                "flop_per_launch": per_launch, "avg_launch_ms": avg_ms,
+                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)"}
+    else:
+        roof = {"bound": "hbm", "kernel": dom, "achieved": None, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "frac": None, "traffic": None}
+    kernels = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
+               for k, v in per_class.items()}
+    for k in kernels:
+        if k in fl and kernels[k]["ms_per_step"] > 0:
+            kernels[k]["tflops"] = B * fl[k] / (kernels[k]["ms_per_step"] / 1000.0) / 1e12
+
+    cpu = cpu_oracle_sample(cfg) if (world == 1 and not args.no_cpu) else None
+    peak_dense = float(peaks.get("bf16_tflops"))
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": cfg.name, "batch_per_gpu": B, "global_batch": B * world,
+                   "tokens_per_clip": cfg.n_tokens, "weights": cfg.weights, "mask": cfg.mask, "pool": cfg.pool,
+                   "parallelism": f"replicas x{world}", "l2": "flushed between steps (256 MiB write)"},
+        "clips_per_s": world * B * args.steps / (total_ms / 1000.0),
+        "tflops": tflops, "tc_peak_frac": tflops / peak_dense,
+        "tc_peak": {"value": peak_dense, "source": f"{peak_src} bf16 burst"},
+        "roofline": roof,
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": int(pix_host.numel() * 4), "d2h_bytes_per_step": int(out_host.numel() * 4)},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "when": datetime.datetime.utcnow().isoformat() + "Z",
+    }
+    print(json.dumps(line), flush=True)
+    model.close()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
+    args = ap.parse_args()
+    cfg = synth.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, cfg, rank, world)
+    if world > 1:
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        return run_ours(args, cfg, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,535 @@
+// tcgen05 GEMM for the encoder's dense layers: out = epilogue(A W^T + bias).
+//
+// The pre-LN block of the JEPA encoders ("Quantization" page, section "The
+// rule": attn_qkv, attn_out, ffn_up, ffn_down per block) spends its time in
+// four GEMMs whose A operand is the token matrix [B*N, D] (or [B*N, 4D]) and
+// whose B operand is a weight matrix [N_out, K] in PyTorch [out, in] order.
+// The same kernel, with a gathering A loader, is the tubelet patch-embed (a
+// conv with stride = kernel, i.e. an implicit GEMM over unfolded pixels).
+//
+// Design (one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer: A tile [128 x 64] and, for f16 weights, the
+//               B tile [BN x 64] per stage, 128-byte swizzled, into a ring
+//               of shared-memory stages;
+//   warp 1      MMA issuer: tcgen05.mma kind::f16 M=128 N=BN K=16, f32
+//               accumulators in TMEM, two accumulator buffers so the
+//               epilogue of tile i overlaps the main loop of tile i+1;
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator rows, bias, then
+//               f16 store / GELU / f32 residual add / QKV head scatter /
+//               patch-embed + pos_embed;
+//   warps 6-9   (quantised weights or patch-embed only) converters: unpack
+//               q8_0 (q*d) or q4_0 ((q-8)*d) blocks, or gather pixels, into
+//               the swizzled operand tile in shared memory.
+#include <cudaTypedefs.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "internal.h"
+
+namespace jb {
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = BN == 256 ? 4 : (BN == 192 ? 5 : 6);
+  static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;
+};
+
+__device__ __forceinline__ float gelu_erf(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
+
+// Epilogue for 32 consecutive output columns col0..col0+31 of one row.
+__device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int col0, const uint32_t (&r)[32]) {
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  if (p.bias) {
+    const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 b = __ldg(b4 + j);
+      v[4 * j] += b.x;
+      v[4 * j + 1] += b.y;
+      v[4 * j + 2] += b.z;
+      v[4 * j + 3] += b.w;
+    }
+  }
+  switch (p.epi) {
+    case EPI_GELU_F16:
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+      // fall through
+    case EPI_F16: {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(p.out) + static_cast<size_t>(row) * p.ldo + col0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        dst[j] = make_uint4(pack_half2(v[8 * j], v[8 * j + 1]), pack_half2(v[8 * j + 2], v[8 * j + 3]),
+                            pack_half2(v[8 * j + 4], v[8 * j + 5]), pack_half2(v[8 * j + 6], v[8 * j + 7]));
+    } break;
+    case EPI_RESID_F32: {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + static_cast<size_t>(row) * p.ldo + col0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float4 o = dst[j];
+        o.x += v[4 * j];
+        o.y += v[4 * j + 1];
+        o.z += v[4 * j + 2];
+        o.w += v[4 * j + 3];
+        dst[j] = o;
+      }
+    } break;
+    case EPI_F32: {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + static_cast<size_t>(row) * p.ldo + col0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } break;
+    case EPI_QKV: {
+      const int D = p.qkv.dim;
+      const int part = col0 / D + p.qkv.first_part;
+      const int within = col0 % D;
+      const int hd = within >> 6, d0 = within & 63;
+      const int b = row / p.qkv.ntok, t = row % p.qkv.ntok;
+      const size_t bh = static_cast<size_t>(b) * p.qkv.heads + hd;
+      if (part < 2) {
+        __half* base = part == 0 ? p.qkv.q : p.qkv.k;
+        if (base) {
+          uint4* dst = reinterpret_cast<uint4*>(base + (bh * p.qkv.ntok + t) * 64 + d0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(pack_half2(v[8 * j], v[8 * j + 1]), pack_half2(v[8 * j + 2], v[8 * j + 3]),
+                                pack_half2(v[8 * j + 4], v[8 * j + 5]), pack_half2(v[8 * j + 6], v[8 * j + 7]));
+        }
+      } else if (p.qkv.vt) {
+        __half* base = p.qkv.vt + (bh * 64 + d0) * static_cast<size_t>(p.qkv.npad) + t;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) base[static_cast<size_t>(j) * p.qkv.npad] = __float2half_rn(v[j]);
+      }
+    } break;
+    case EPI_PATCH: {
+      const int b = row / p.patch.n_patches, i = row % p.patch.n_patches;
+      const int tok = i + p.patch.has_cls;
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) +
+                                              (static_cast<size_t>(b) * p.patch.ntok + tok) * p.ldo + col0);
+      const float4* pos = reinterpret_cast<const float4*>(p.patch.pos + static_cast<size_t>(tok) * p.ldo + col0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float4 q = __ldg(pos + j);
+        dst[j] = make_float4(v[4 * j] + q.x, v[4 * j + 1] + q.y, v[4 * j + 2] + q.z, v[4 * j + 3] + q.w);
+      }
+    } break;
+    default:
+      break;
+  }
+}
+
+// Unpack a [BN x 64] slice of a q8_0 / q4_0 weight matrix into the swizzled
+// f16 B tile.  Each thread converts 8 consecutive K elements of one row per
+// step: value = q * d (q8_0) or (q - 8) * d (q4_0), rounded once to f16.
+template <int BMODE, int BN>
+__device__ __forceinline__ void fill_b_quant(uint8_t* sB, const GemmParams& p, int n0, int kb, int ct) {
+  const int K = p.K;
+  const uint32_t sbase = smem_u32(sB);
+#pragma unroll 4
+  for (int idx = ct; idx < BN * 8; idx += 128) {
+    const int r = idx >> 3, u = idx & 7;
+    const int n = n0 + r;
+    const int k = kb * 64 + u * 8;
+    const float d = __half2float(p.bscale[static_cast<size_t>(n) * (K >> 5) + (k >> 5)]);
+    uint32_t w[4];
+    if (BMODE == B_Q8) {
+      const uint2 q = __ldg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(p.bq) +
+                                                           static_cast<size_t>(n) * K + k));
+      const uint32_t qq[2] = {q.x, q.y};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t word = qq[e >> 1];
+        const int sh = (e & 1) * 16;
+        const float a = static_cast<float>(static_cast<int8_t>((word >> sh) & 0xFF));
+        const float b = static_cast<float>(static_cast<int8_t>((word >> (sh + 8)) & 0xFF));
+        w[e] = pack_half2(a * d, b * d);
+      }
+    } else {
+      const int j0 = k & 31;
+      const uint2 q = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(p.bq) +
+                                                           static_cast<size_t>(n) * (K >> 1) + (k >> 5) * 16 +
+                                                           (j0 & 15)));
+      const int nsh = j0 >= 16 ? 4 : 0;
+      const uint32_t qq[2] = {q.x, q.y};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t word = qq[e >> 1];
+        const int sh = (e & 1) * 16;
+        const float a = static_cast<float>(static_cast<int>((word >> (sh + nsh)) & 0xF) - 8);
+        const float b = static_cast<float>(static_cast<int>((word >> (sh + 8 + nsh)) & 0xF) - 8);
+        w[e] = pack_half2(a * d, b * d);
+      }
+    }
+    st_shared_v4(sbase + sw128_offset(r, u * 8), w[0], w[1], w[2], w[3]);
+  }
+}
+
+// Gather a [128 x 64] slice of the unfolded patch matrix: row m = patch
+// (clip b, slot t', patch row, patch col); column k = (c, dt, kh, kw) in the
+// row-major order of a conv weight [D, 3, kt, p, p].  Columns >= 3*kt*p*p
+// and rows >= M are zero.
+__device__ __forceinline__ void fill_a_patch(uint8_t* sA, const GemmParams& p, int m0, int kb, int ct) {
+  const PatchSrc& s = p.patch;
+  const int wp = s.W / s.patch;
+  const int ppf = (s.H / s.patch) * wp;
+  const int pp = s.patch * s.patch;
+  const int ktpp = s.tubelet * pp;
+  const uint32_t sbase = smem_u32(sA);
+  for (int idx = ct; idx < 128 * 8; idx += 128) {
+    const int r = idx >> 3, u = idx & 7;
+    const int m = m0 + r;
+    float f[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = 0.0f;
+    if (m < p.M) {
+      const int b = m / s.n_patches, i = m % s.n_patches;
+      const int tp = i / ppf, rem = i % ppf;
+      const int hp = rem / wp, wq = rem % wp;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int k = kb * 64 + u * 8 + e;
+        if (k < s.k_real) {
+          const int c = k / ktpp, rk = k % ktpp;
+          const int dt = rk / pp, rk2 = rk % pp;
+          const int kh = rk2 / s.patch, kw = rk2 % s.patch;
+          const size_t plane = (static_cast<size_t>(b) * s.T + tp * s.tubelet + dt) * 3 + c;
+          f[e] = __ldg(s.pixels + (plane * s.H + hp * s.patch + kh) * s.W + wq * s.patch + kw);
+        }
+      }
+    }
+    st_shared_v4(sbase + sw128_offset(r, u * 8), pack_half2(f[0], f[1]), pack_half2(f[2], f[3]),
+                 pack_half2(f[4], f[5]), pack_half2(f[6], f[7]));
+  }
+}
+
+template <int BN, int BMODE, bool GATHER>
+__global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 320 : 192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmParams p) {
+  using C = GemmCfg<BN>;
+  constexpr bool CONV = (BMODE != B_F16) || GATHER;
+  constexpr int S = C::STAGES;
+  extern __shared__ uint8_t dsmem[];
+  __shared__ uint64_t full_bar[S], conv_bar[S], empty_bar[S], tfull_bar[2], tempty_bar[2], drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  const uint32_t raw = smem_u32(dsmem);
+  uint8_t* smem = dsmem + ((1024u - (raw & 1023u)) & 1023u);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&conv_bar[s], 128);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 128);
+    }
+    mbar_init(&drain_bar, 1);
+    abort_sh = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    if (!GATHER) tma_prefetch_desc(&tmA);
+    if (BMODE == B_F16) tma_prefetch_desc(&tmB);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_sh;
+
+  WaitCtl w;
+  w.abort = reinterpret_cast<volatile int*>(&abort_sh);
+  w.err = p.err;
+  w.timeout_ns = p.timeout_ns;
+  w.where = (KID_GEMM << 8) | static_cast<unsigned>(warp);
+  const int num_tiles = p.m_tiles * p.n_tiles;
+  const int kblocks = p.K / 64;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_par = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int mb = t % p.m_tiles, nb = t / p.m_tiles;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, w)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sA = smem + stage * C::STAGE_BYTES;
+          uint8_t* sB = sA + C::A_BYTES;
+          constexpr uint32_t tx = (GATHER ? 0u : (uint32_t)C::A_BYTES) + (BMODE == B_F16 ? (uint32_t)C::B_BYTES : 0u);
+          mbar_expect_tx(&full_bar[stage], tx);
+          if (!GATHER) tma_load_2d(sA, &tmA, &full_bar[stage], kb * 64, mb * 128);
+          if (BMODE == B_F16) tma_load_2d(sB, &tmB, &full_bar[stage], kb * 64, nb * BN);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {  // let the copies already issued land before the CTA exits
+        for (int s = 0; s < S; ++s)
+          if ((armed >> s) & 1u) mbar_wait_drain(&full_bar[s], (armed_par >> s) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(128, BN);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, aphase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(&tempty_bar[acc], aphase ^ 1, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dtm = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, w)) {
+            ok = false;
+            break;
+          }
+          if (CONV && !mbar_wait(&conv_bar[stage], phase, w)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint64_t ad = sdesc_kmajor_sw128(a0);
+          const uint64_t bd = sdesc_kmajor_sw128(a0 + C::A_BYTES);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma_f16_ss(dtm, ad + static_cast<uint64_t>(2 * k), bd + static_cast<uint64_t>(2 * k), idesc,
+                          (kb | k) != 0 ? 1u : 0u);
+          tc_commit(&empty_bar[stage]);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tfull_bar[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          aphase ^= 1;
+        }
+      }
+      // every MMA issued above completes before TMEM is released
+      tc_commit(&drain_bar);
+      mbar_wait_drain(&drain_bar, 0);
+    }
+  } else if (warp < 6) {
+    const int quad = warp & 3;
+    int acc = 0;
+    uint32_t aphase = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      bool ok = mbar_wait(&tfull_bar[acc], aphase, w);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int mb = t % p.m_tiles, nb = t / p.m_tiles;
+      const int row = mb * 128 + quad * 32 + lane;
+      const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tb + static_cast<uint32_t>(c * 32), r);
+        if (row < p.M) epilogue_chunk(p, row, nb * BN + c * 32, r);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty_bar[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        aphase ^= 1;
+      }
+    }
+  } else if (CONV) {
+    const int ct = threadIdx.x - 192;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      const int mb = t % p.m_tiles, nb = t / p.m_tiles;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        bool okw = mbar_wait(&empty_bar[stage], phase ^ 1, w);
+        okw = __all_sync(0xffffffffu, okw);
+        if (!okw) {
+          ok = false;
+          break;
+        }
+        uint8_t* sA = smem + stage * C::STAGE_BYTES;
+        uint8_t* sB = sA + C::A_BYTES;
+        if (GATHER)
+          fill_a_patch(sA, p, mb * 128, kb, ct);
+        else
+          fill_b_quant<BMODE, BN>(sB, p, nb * BN, kb, ct);
+        fence_proxy_async_smem();
+        mbar_arrive(&conv_bar[stage]);
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host --
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+bool make_tmap_f16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                   const uint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[3], s[2];
+  cuuint32_t b[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank, const_cast<void*>(base), d, s, b, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  static int cache[64] = {0};
+  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (n <= 0) n = 148;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& W, const float* bias, int epi,
+                 void* out, int ldo, const QkvDst* qkv, const PatchSrc* patch) {
+  if (!op || !out || M < 1 || K < 64 || K % 64 != 0 || W.K != K || W.N < 1 || !W.data) return JEPA_B200_ERR_SHAPE;
+  if (!patch && !A) return JEPA_B200_ERR_ARG;
+  const int N = W.N;
+  const int bn = N % 256 == 0 ? 256 : (N % 192 == 0 ? 192 : (N % 128 == 0 ? 128 : 0));
+  if (!bn) return JEPA_B200_ERR_SHAPE;
+  if (patch && W.bmode != B_F16) return JEPA_B200_ERR_UNSUPPORTED;
+  if (W.bmode != B_F16 && !W.scales) return JEPA_B200_ERR_ARG;
+  if ((epi == EPI_F16 || epi == EPI_GELU_F16 || epi == EPI_RESID_F32 || epi == EPI_F32) && ldo < N)
+    return JEPA_B200_ERR_SHAPE;
+  memset(op, 0, sizeof(*op));
+  op->bn = bn;
+  op->bmode = W.bmode;
+  op->gather = patch ? 1 : 0;
+  GemmParams& p = op->p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.m_tiles = (M + 127) / 128;
+  p.n_tiles = N / bn;
+  p.bias = bias;
+  p.epi = epi;
+  p.out = out;
+  p.ldo = ldo;
+  if (qkv) p.qkv = *qkv;
+  if (patch) p.patch = *patch;
+  p.bq = W.bmode != B_F16 ? W.data : nullptr;
+  p.bscale = W.scales;
+  if (!patch) {
+    const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+    const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
+    const uint32_t box[2] = {64, 128};
+    if (!make_tmap_f16(&op->tmA, A, 2, dims, str, box)) return JEPA_B200_ERR_CUDA;
+  }
+  if (W.bmode == B_F16) {
+    const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
+    const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
+    const uint32_t box[2] = {64, static_cast<uint32_t>(bn)};
+    if (!make_tmap_f16(&op->tmB, W.data, 2, dims, str, box)) return JEPA_B200_ERR_CUDA;
+  }
+  op->grid = std::min(p.m_tiles * p.n_tiles, num_sms());
+  op->smem = bn == 256 ? GemmCfg<256>::SMEM : (bn == 192 ? GemmCfg<192>::SMEM : GemmCfg<128>::SMEM);
+  return JEPA_B200_OK;
+}
+
+template <int BN, int BMODE, bool GATHER>
+static int launch_impl(const GemmOp& op, cudaStream_t st) {
+  auto kern = gemm_tc_kernel<BN, BMODE, GATHER>;
+  static unsigned long long attr_done = 0;  // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !((attr_done >> dev) & 1ull)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<BN>::SMEM) != cudaSuccess)
+      return JEPA_B200_ERR_CUDA;
+    attr_done |= 1ull << dev;
+  }
+  constexpr int threads = (BMODE != B_F16 || GATHER) ? 320 : 192;
+  kern<<<op.grid, threads, GemmCfg<BN>::SMEM, st>>>(op.tmA, op.tmB, op.p);
+  return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+}
+
+int gemm_launch(const GemmOp& op_in, cudaStream_t st, DevErr* err, unsigned long long timeout_ns) {
+  GemmOp op = op_in;
+  op.p.err = err;
+  op.p.timeout_ns = timeout_ns;
+  if (op.gather) {
+    switch (op.bn) {
+      case 256: return launch_impl<256, B_F16, true>(op, st);
+      case 192: return launch_impl<192, B_F16, true>(op, st);
+      default: return launch_impl<128, B_F16, true>(op, st);
+    }
+  }
+#define JB_GEMM_CASE(BNV)                                      \
+  case BNV:                                                    \
+    switch (op.bmode) {                                        \
+      case B_Q8: return launch_impl<BNV, B_Q8, false>(op, st); \
+      case B_Q4: return launch_impl<BNV, B_Q4, false>(op, st); \
+      default: return launch_impl<BNV, B_F16, false>(op, st);  \
+    }
+  switch (op.bn) {
+    JB_GEMM_CASE(256)
+    JB_GEMM_CASE(192)
+    JB_GEMM_CASE(128)
+    default:
+      return JEPA_B200_ERR_SHAPE;
+  }
+#undef JB_GEMM_CASE
+}
+
+}  // namespace jb

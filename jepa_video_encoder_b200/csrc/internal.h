@@ -1,0 +1,114 @@
+// Host-side declarations shared by the translation units of libjepa_b200.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/jepa_b200.h"
+#include "common.cuh"
+
+namespace jb {
+
+enum Epi { EPI_F16 = 0, EPI_GELU_F16 = 1, EPI_RESID_F32 = 2, EPI_F32 = 3, EPI_QKV = 4, EPI_PATCH = 5 };
+enum BMode { B_F16 = 0, B_Q8 = 1, B_Q4 = 2 };
+
+constexpr unsigned long long kDefaultTimeoutNs = 4000000000ull;
+
+// A weight matrix [N, K] on the device in the GEMM's layout.
+struct DevMatrix {
+  int bmode = B_F16;  // B_F16 | B_Q8 | B_Q4
+  int N = 0, K = 0;   // K: row length as stored (f16: padded to 64 with zeros)
+  void* data = nullptr;       // f16 [N, K] | int8 [N, K] | nibble bytes [N, K/2]
+  __half* scales = nullptr;   // fp16 [N, K/32] for quantised matrices
+};
+
+// Destination of the QKV scatter epilogue.
+struct QkvDst {
+  __half* q = nullptr;
+  __half* k = nullptr;
+  __half* vt = nullptr;
+  int ntok = 0, heads = 0, npad = 0, first_part = 0, dim = 0;
+};
+
+// Source geometry of the implicit-GEMM patch-embed.
+struct PatchSrc {
+  const float* pixels = nullptr;
+  int T = 0, H = 0, W = 0, patch = 0, tubelet = 0;
+  int n_patches = 0;   // per clip
+  int k_real = 0;      // 3 * kt * p * p
+  const float* pos = nullptr;  // [ntok, D]
+  int ntok = 0, has_cls = 0;
+};
+
+struct GemmParams {
+  int M, N, K;
+  int m_tiles, n_tiles;
+  const float* bias;
+  int epi;
+  void* out;
+  int ldo;
+  QkvDst qkv;
+  PatchSrc patch;
+  const void* bq;           // quantised weights
+  const __half* bscale;
+  DevErr* err;
+  unsigned long long timeout_ns;
+};
+
+// Everything one GEMM launch needs, built once and replayed.
+struct GemmOp {
+  CUtensorMap tmA;
+  CUtensorMap tmB;
+  GemmParams p;
+  int bn = 0, bmode = 0, gather = 0, grid = 0, smem = 0;
+};
+
+// Build a GEMM op.  A: f16 [M, K] (ignored when patch != nullptr: the patch
+// pixels are gathered instead).  Returns a jepa_b200_status.
+int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& W, const float* bias, int epi,
+                 void* out, int ldo, const QkvDst* qkv, const PatchSrc* patch);
+int gemm_launch(const GemmOp& op, cudaStream_t st, DevErr* err, unsigned long long timeout_ns);
+
+struct AttnParams {
+  int N, heads, n_q_tiles, mask, has_cls, ppf;
+  float scale_log2;
+  __half* out;
+  int ldo;
+  DevErr* err;
+  unsigned long long timeout_ns;
+};
+
+struct AttnOp {
+  CUtensorMap tmQ, tmK, tmV;
+  AttnParams p;
+  int B = 0, smem = 0;
+};
+
+int attn_prepare(AttnOp* op, const __half* q, const __half* k, const __half* vt, int B, int heads, int ntok,
+                 int npad, int mask, int has_cls, int ppf, __half* out);
+int attn_launch(const AttnOp& op, cudaStream_t st, DevErr* err, unsigned long long timeout_ns);
+
+// LayerNorm: rows of D f32 -> f16 or f32; input row r*in_stride.
+int launch_layernorm(const float* x, int rows, int D, long long in_stride, const float* g, const float* b,
+                     float eps, void* out, bool out_f16, cudaStream_t st);
+// Write the CLS rows x[b*ntok + 0] = cls + pos[0].
+int launch_cls_rows(float* x, int B, int ntok, int D, const float* cls, const float* pos, cudaStream_t st);
+int launch_mean_pool(const float* y, int B, int ntok, int D, int first, float* partial, float* out,
+                     cudaStream_t st);
+int mean_pool_partial_floats(int B, int D);
+int launch_repack(int bmode, const uint8_t* blocks, int N, int K, void* qs, __half* scales, cudaStream_t st);
+int launch_gemv(const float* x, int M, int K, const DevMatrix& W, const float* bias, int epi, const float* resid,
+                long long resid_stride, float* y, cudaStream_t st);
+int launch_xattn_1q(const float* q, const __half* k, const __half* vt, int B, int heads, int ntok, int npad,
+                    float* out, cudaStream_t st);
+
+// Driver entry point for tensor maps (resolved once through the runtime).
+bool make_tmap_f16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                   const uint32_t* box);
+
+int num_sms();
+
+}  // namespace jb

@@ -1,0 +1,900 @@
+// Host runtime of the JEPA ViT encoder forward: weight loading from a tensor
+// table, the device workspace, and the fixed kernel sequence of one forward
+// pass (the C ABI calls of include/jepa_b200.h).
+//
+// Sequence of jepa_b200_encode (B clips, R = B * N token rows):
+//   patch-embed (implicit GEMM + pos_embed) and the CLS rows       -> X f32 [R, D]
+//   per block:  LN1 -> Y f16; QKV GEMM -> Q, K, V^T (head-major)
+//               attention -> O f16 [R, D]; out GEMM: X += O Wo^T + bo
+//               LN2 -> Y; up GEMM + GELU -> H f16 [R, 4D]; down GEMM: X += H Wd^T + bd
+//   final LN -> full map / CLS rows / mean over patch tokens / attentive head.
+// The block structure is the pre-LN block of the "Quantization" page ("The
+// rule": ln1, attn_qkv, attn_out, ln2, ffn_up, ffn_down); the head follows
+// "jepa.cpp -- measured benchmarks", "Attentive-pool head".
+#include <string.h>
+
+#include <cmath>
+#include <string>
+#include <unordered_map>
+#include <vector>
+
+#include "internal.h"
+
+using namespace jb;
+
+namespace {
+
+struct LayerW {
+  float *ln1_g = nullptr, *ln1_b = nullptr, *ln2_g = nullptr, *ln2_b = nullptr;
+  DevMatrix qkv, out, up, down;
+  float *b_qkv = nullptr, *b_out = nullptr, *b_up = nullptr, *b_down = nullptr;
+};
+
+struct BlockOps {
+  GemmOp qkv, out, up, down;
+};
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    cudaGetDevice(&prev);
+    if (prev != dev) cudaSetDevice(dev);
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (prev >= 0 && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+}  // namespace
+
+struct jepa_b200_model {
+  jepa_b200_config cfg{};
+  int device = 0;
+  int N = 0, Np = 0, ppf = 0, Kpe = 0, Kpe_pad = 0, npad = 0;
+  DevMatrix pe;
+  float *b_pe = nullptr, *pos = nullptr, *cls = nullptr;
+  std::vector<LayerW> enc, head;
+  float *norm_g = nullptr, *norm_b = nullptr;
+  bool has_head = false;
+  float *query = nullptr, *lnkv_g = nullptr, *lnkv_b = nullptr, *ln2x_g = nullptr, *ln2x_b = nullptr;
+  DevMatrix xq, xkv, xout, xup, xdown, hcls;
+  float *b_xq = nullptr, *b_xkv = nullptr, *b_xout = nullptr, *b_xup = nullptr, *b_xdown = nullptr,
+        *b_cls = nullptr;
+  std::vector<void*> allocs;
+  size_t weight_bytes = 0;
+
+  // workspace for the largest B seen
+  int ws_B = 0;
+  float* X = nullptr;
+  __half *Y = nullptr, *Q = nullptr, *Kb = nullptr, *Vt = nullptr, *O = nullptr, *H = nullptr;
+  float *Yf = nullptr, *partial = nullptr;
+  float *hq = nullptr, *hattn = nullptr, *hz = nullptr, *hzn = nullptr, *hu = nullptr;
+  std::vector<void*> ws_allocs;
+  std::vector<BlockOps> enc_ops, head_ops;
+  GemmOp pe_op, kv_op;
+  AttnOp attn_enc, attn_head;
+
+  float* stage_pix = nullptr;
+  size_t stage_pix_bytes = 0;
+  float* stage_out = nullptr;
+  size_t stage_out_bytes = 0;
+
+  DevErr* err = nullptr;
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+  bool have_timing = false;
+  unsigned long long timeout_ns = kDefaultTimeoutNs;
+  int launches = 0;
+
+  // per-kernel timing (jepa_b200_set_profiling)
+  bool prof = false;
+  std::vector<cudaEvent_t> prof_events;
+  size_t prof_used = 0;
+  struct ProfRec {
+    int cls;
+    size_t e0, e1;
+  };
+  std::vector<ProfRec> prof_recs;
+};
+
+namespace {
+
+typedef std::unordered_map<std::string, const jepa_b200_tensor*> TableMap;
+
+bool is_retyped(const std::string& n) {
+  static const char* suffixes[] = {"attn_qkv.weight",     "attn_out.weight",     "ffn_up.weight",
+                                   "ffn_down.weight",     "head.xattn.q.weight", "head.xattn.k.weight",
+                                   "head.xattn.v.weight", "head.xattn.out.weight", "head.cls.weight"};
+  for (const char* s : suffixes) {
+    const size_t L = strlen(s);
+    if (n.size() >= L && n.compare(n.size() - L, L, s) == 0) return true;
+  }
+  return false;
+}
+
+int64_t numel(const jepa_b200_tensor* t) {
+  int64_t n = 1;
+  for (int i = 0; i < t->ndim; ++i) n *= t->shape[i];
+  return n;
+}
+
+size_t expected_bytes(const jepa_b200_tensor* t) {
+  const int64_t n = numel(t);
+  switch (t->dtype) {
+    case JEPA_B200_F32: return static_cast<size_t>(n) * 4;
+    case JEPA_B200_F16: return static_cast<size_t>(n) * 2;
+    case JEPA_B200_Q8_0: return static_cast<size_t>(n / 32) * 34;
+    case JEPA_B200_Q4_0: return static_cast<size_t>(n / 32) * 18;
+    default: return 0;
+  }
+}
+
+struct Loader {
+  jepa_b200_model* m;
+  TableMap tab;
+  int status = JEPA_B200_OK;
+
+  bool dry = false;  // validate only: no device calls, no conversions
+
+  void* dalloc(size_t bytes) {
+    void* p = nullptr;
+    if (status != JEPA_B200_OK) return nullptr;
+    if (dry) return reinterpret_cast<void*>(static_cast<uintptr_t>(256));
+    if (cudaMalloc(&p, bytes) != cudaSuccess) {
+      status = JEPA_B200_ERR_CUDA;
+      return nullptr;
+    }
+    m->allocs.push_back(p);
+    m->weight_bytes += bytes;
+    return p;
+  }
+  bool upload(void* dst, const void* src, size_t bytes) {
+    if (status != JEPA_B200_OK) return false;
+    if (dry) return true;
+    if (cudaMemcpy(dst, src, bytes, cudaMemcpyHostToDevice) != cudaSuccess) {
+      status = JEPA_B200_ERR_CUDA;
+      return false;
+    }
+    return true;
+  }
+  const jepa_b200_tensor* get(const std::string& name, std::initializer_list<int64_t> shape) {
+    if (status != JEPA_B200_OK) return nullptr;
+    auto it = tab.find(name);
+    if (it == tab.end()) {
+      status = JEPA_B200_ERR_MISSING_TENSOR;
+      return nullptr;
+    }
+    const jepa_b200_tensor* t = it->second;
+    if (t->ndim != static_cast<int>(shape.size())) {
+      status = JEPA_B200_ERR_SHAPE;
+      return nullptr;
+    }
+    int i = 0;
+    for (int64_t s : shape) {
+      if (t->shape[i++] != s) {
+        status = JEPA_B200_ERR_SHAPE;
+        return nullptr;
+      }
+    }
+    const bool quant = t->dtype == JEPA_B200_Q8_0 || t->dtype == JEPA_B200_Q4_0;
+    if (t->dtype != JEPA_B200_F32 && t->dtype != JEPA_B200_F16 && !quant) {
+      status = JEPA_B200_ERR_DTYPE;
+      return nullptr;
+    }
+    if (quant && !is_retyped(name)) {
+      status = JEPA_B200_ERR_DTYPE;
+      return nullptr;
+    }
+    if (!t->data || t->nbytes != expected_bytes(t)) {
+      status = t->data ? JEPA_B200_ERR_SHAPE : JEPA_B200_ERR_ARG;
+      return nullptr;
+    }
+    return t;
+  }
+  // host values of an f32 / f16 tensor as float
+  std::vector<float> host_floats(const jepa_b200_tensor* t) {
+    const int64_t n = numel(t);
+    if (dry) return std::vector<float>(static_cast<size_t>(n));
+    std::vector<float> v(static_cast<size_t>(n));
+    if (t->dtype == JEPA_B200_F32) {
+      memcpy(v.data(), t->data, static_cast<size_t>(n) * 4);
+    } else {
+      const __half* h = static_cast<const __half*>(t->data);
+      for (int64_t i = 0; i < n; ++i) v[static_cast<size_t>(i)] = __half2float(h[i]);
+    }
+    return v;
+  }
+  float* vec(const std::string& name, int64_t len) {
+    const jepa_b200_tensor* t = get(name, {len});
+    if (!t) return nullptr;
+    if (t->dtype != JEPA_B200_F32 && t->dtype != JEPA_B200_F16) {
+      status = JEPA_B200_ERR_DTYPE;
+      return nullptr;
+    }
+    std::vector<float> v = host_floats(t);
+    float* d = static_cast<float*>(dalloc(v.size() * 4));
+    if (d) upload(d, v.data(), v.size() * 4);
+    return d;
+  }
+  float* table2d(const std::string& name, int64_t rows, int64_t cols) {
+    const jepa_b200_tensor* t = get(name, {rows, cols});
+    if (!t) return nullptr;
+    if (t->dtype != JEPA_B200_F32 && t->dtype != JEPA_B200_F16) {
+      status = JEPA_B200_ERR_DTYPE;
+      return nullptr;
+    }
+    std::vector<float> v = host_floats(t);
+    float* d = static_cast<float*>(dalloc(v.size() * 4));
+    if (d) upload(d, v.data(), v.size() * 4);
+    return d;
+  }
+  // Matrix [N, K] from one or more tensors stacked along N (all one dtype).
+  DevMatrix matrix(const std::vector<const jepa_b200_tensor*>& parts, int64_t K, int64_t Kpad) {
+    DevMatrix M;
+    if (status != JEPA_B200_OK) return M;
+    int64_t N = 0;
+    const int dt = parts[0]->dtype;
+    for (auto* t : parts) {
+      if (t->dtype != dt) {
+        status = JEPA_B200_ERR_DTYPE;
+        return M;
+      }
+      N += numel(t) / K;
+    }
+    M.N = static_cast<int>(N);
+    M.K = static_cast<int>(Kpad);
+    const bool quant = dt == JEPA_B200_Q8_0 || dt == JEPA_B200_Q4_0;
+    if (quant && (K % 64 != 0 || Kpad != K)) {
+      status = JEPA_B200_ERR_SHAPE;
+      return M;
+    }
+    if (dry) {
+      M.bmode = dt == JEPA_B200_Q8_0 ? B_Q8 : (dt == JEPA_B200_Q4_0 ? B_Q4 : B_F16);
+      M.data = dalloc(1);
+      M.scales = quant ? static_cast<__half*>(dalloc(1)) : nullptr;
+      return M;
+    }
+    if (dt == JEPA_B200_F32 || dt == JEPA_B200_F16) {
+      std::vector<__half> h(static_cast<size_t>(N * Kpad), __float2half_rn(0.0f));
+      int64_t row = 0;
+      for (auto* t : parts) {
+        std::vector<float> v = host_floats(t);
+        const int64_t rows = numel(t) / K;
+        for (int64_t r = 0; r < rows; ++r)
+          for (int64_t k = 0; k < K; ++k)
+            h[static_cast<size_t>((row + r) * Kpad + k)] = __float2half_rn(v[static_cast<size_t>(r * K + k)]);
+        row += rows;
+      }
+      M.bmode = B_F16;
+      M.data = dalloc(h.size() * 2);
+      if (M.data) upload(M.data, h.data(), h.size() * 2);
+      return M;
+    }
+    // quantised: split the blocks into quants and fp16 scales (byte moves)
+    const bool q8 = dt == JEPA_B200_Q8_0;
+    const int bsz = q8 ? 34 : 18, qb = q8 ? 32 : 16;
+    const int64_t nblk = N * (K / 32);
+    std::vector<uint8_t> qs(static_cast<size_t>(nblk * qb));
+    std::vector<uint16_t> sc(static_cast<size_t>(nblk));
+    int64_t bi = 0;
+    for (auto* t : parts) {
+      const uint8_t* src = static_cast<const uint8_t*>(t->data);
+      const int64_t nb = numel(t) / 32;
+      for (int64_t i = 0; i < nb; ++i, ++bi) {
+        const uint8_t* b = src + i * bsz;
+        sc[static_cast<size_t>(bi)] = static_cast<uint16_t>(b[0] | (b[1] << 8));
+        memcpy(&qs[static_cast<size_t>(bi * qb)], b + 2, qb);
+      }
+    }
+    M.bmode = q8 ? B_Q8 : B_Q4;
+    M.data = dalloc(qs.size());
+    M.scales = static_cast<__half*>(dalloc(sc.size() * 2));
+    if (M.data) upload(M.data, qs.data(), qs.size());
+    if (M.scales) upload(M.scales, sc.data(), sc.size() * 2);
+    return M;
+  }
+  DevMatrix mat(const std::string& name, int64_t N, int64_t K) {
+    const jepa_b200_tensor* t = get(name, {N, K});
+    if (!t) return DevMatrix();
+    return matrix({t}, K, K);
+  }
+  void block(LayerW& L, const std::string& p, int64_t D, int64_t Mh) {
+    L.ln1_g = vec(p + "ln1.weight", D);
+    L.ln1_b = vec(p + "ln1.bias", D);
+    L.qkv = mat(p + "attn_qkv.weight", 3 * D, D);
+    L.b_qkv = vec(p + "attn_qkv.bias", 3 * D);
+    L.out = mat(p + "attn_out.weight", D, D);
+    L.b_out = vec(p + "attn_out.bias", D);
+    L.ln2_g = vec(p + "ln2.weight", D);
+    L.ln2_b = vec(p + "ln2.bias", D);
+    L.up = mat(p + "ffn_up.weight", Mh, D);
+    L.b_up = vec(p + "ffn_up.bias", Mh);
+    L.down = mat(p + "ffn_down.weight", D, Mh);
+    L.b_down = vec(p + "ffn_down.bias", D);
+  }
+};
+
+void free_list(std::vector<void*>& v) {
+  for (void* p : v) cudaFree(p);
+  v.clear();
+}
+
+int validate_config(const jepa_b200_config* c) {
+  if (!c) return JEPA_B200_ERR_ARG;
+  if (c->dim < 64 || c->heads < 1 || c->dim != 64 * c->heads || c->dim % 64 || c->depth < 0 || c->mlp < 64 ||
+      c->mlp % 64)
+    return JEPA_B200_ERR_SHAPE;
+  if (c->patch < 1 || c->tubelet < 1 || c->img_h < c->patch || c->img_w < c->patch || c->img_h % c->patch ||
+      c->img_w % c->patch || c->frames < c->tubelet || c->frames % c->tubelet)
+    return JEPA_B200_ERR_SHAPE;
+  if (c->mask != JEPA_B200_MASK_BIDIR && c->mask != JEPA_B200_MASK_BLOCK_CAUSAL) return JEPA_B200_ERR_ARG;
+  if (c->dim > 4096 || c->mlp > 16384) return JEPA_B200_ERR_SHAPE;
+  if (c->n_classes < 0 || c->head_sa_blocks < 0) return JEPA_B200_ERR_ARG;
+  if (!(c->ln_eps > 0.0f)) return JEPA_B200_ERR_ARG;
+  return JEPA_B200_OK;
+}
+
+int alloc_ws(jepa_b200_model* m, void** p, size_t bytes) {
+  if (cudaMalloc(p, bytes) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+  m->ws_allocs.push_back(*p);
+  return JEPA_B200_OK;
+}
+
+int prepare_block_ops(jepa_b200_model* m, const LayerW& L, BlockOps& ops, float* Xres, int R) {
+  const int D = m->cfg.dim, Mh = m->cfg.mlp;
+  QkvDst qd;
+  qd.q = m->Q;
+  qd.k = m->Kb;
+  qd.vt = m->Vt;
+  qd.ntok = m->N;
+  qd.heads = m->cfg.heads;
+  qd.npad = m->npad;
+  qd.first_part = 0;
+  qd.dim = D;
+  int s;
+  if ((s = gemm_prepare(&ops.qkv, m->Y, R, D, L.qkv, L.b_qkv, EPI_QKV, m->Q, 3 * D, &qd, nullptr))) return s;
+  if ((s = gemm_prepare(&ops.out, m->O, R, D, L.out, L.b_out, EPI_RESID_F32, Xres, D, nullptr, nullptr))) return s;
+  if ((s = gemm_prepare(&ops.up, m->Y, R, D, L.up, L.b_up, EPI_GELU_F16, m->H, Mh, nullptr, nullptr))) return s;
+  if ((s = gemm_prepare(&ops.down, m->H, R, Mh, L.down, L.b_down, EPI_RESID_F32, Xres, D, nullptr, nullptr)))
+    return s;
+  return JEPA_B200_OK;
+}
+
+int ensure_workspace(jepa_b200_model* m, int B) {
+  if (B <= m->ws_B) return JEPA_B200_OK;
+  cudaDeviceSynchronize();
+  free_list(m->ws_allocs);
+  m->ws_B = 0;
+  const jepa_b200_config& c = m->cfg;
+  const size_t R = static_cast<size_t>(B) * m->N;
+  const size_t D = c.dim;
+  int s = JEPA_B200_OK;
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->X), R * D * 4);
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->Y), R * D * 2);
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->Q), R * D * 2);
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->Kb), R * D * 2);
+  const size_t vt_bytes = static_cast<size_t>(B) * c.heads * 64 * m->npad * 2;
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->Vt), vt_bytes);
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->O), R * D * 2);
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->H), R * c.mlp * 2);
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->Yf), R * D * 4);
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->partial), static_cast<size_t>(mean_pool_partial_floats(B, c.dim)) * 4);
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->hq), D * 4);
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->hattn), B * D * 4);
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->hz), B * D * 4);
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->hzn), B * D * 4);
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->hu), static_cast<size_t>(B) * c.mlp * 4);
+  if (s) {
+    free_list(m->ws_allocs);
+    return s;
+  }
+  // V^T columns past the last token stay zero: the attention multiplies them by p = 0
+  if (cudaMemset(m->Vt, 0, vt_bytes) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+  const int Ri = static_cast<int>(R);
+  m->enc_ops.assign(m->enc.size(), BlockOps());
+  for (size_t l = 0; l < m->enc.size(); ++l)
+    if ((s = prepare_block_ops(m, m->enc[l], m->enc_ops[l], m->X, Ri))) return s;
+  m->head_ops.assign(m->head.size(), BlockOps());
+  for (size_t l = 0; l < m->head.size(); ++l)
+    if ((s = prepare_block_ops(m, m->head[l], m->head_ops[l], m->Yf, Ri))) return s;
+  PatchSrc ps;
+  ps.pixels = nullptr;
+  ps.T = c.frames;
+  ps.H = c.img_h;
+  ps.W = c.img_w;
+  ps.patch = c.patch;
+  ps.tubelet = c.tubelet;
+  ps.n_patches = m->Np;
+  ps.k_real = m->Kpe;
+  ps.pos = m->pos;
+  ps.ntok = m->N;
+  ps.has_cls = c.has_cls ? 1 : 0;
+  if ((s = gemm_prepare(&m->pe_op, nullptr, B * m->Np, m->Kpe_pad, m->pe, m->b_pe, EPI_PATCH, m->X, c.dim, nullptr,
+                        &ps)))
+    return s;
+  if ((s = attn_prepare(&m->attn_enc, m->Q, m->Kb, m->Vt, B, c.heads, m->N, m->npad, c.mask, c.has_cls, m->ppf,
+                        m->O)))
+    return s;
+  if ((s = attn_prepare(&m->attn_head, m->Q, m->Kb, m->Vt, B, c.heads, m->N, m->npad, JEPA_B200_MASK_BIDIR, 0, 1,
+                        m->O)))
+    return s;
+  if (m->has_head) {
+    QkvDst qd;
+    qd.q = nullptr;
+    qd.k = m->Kb;
+    qd.vt = m->Vt;
+    qd.ntok = m->N;
+    qd.heads = c.heads;
+    qd.npad = m->npad;
+    qd.first_part = 1;
+    qd.dim = c.dim;
+    if ((s = gemm_prepare(&m->kv_op, m->Y, Ri, c.dim, m->xkv, m->b_xkv, EPI_QKV, m->Kb, 2 * c.dim, &qd, nullptr)))
+      return s;
+  }
+  m->ws_B = B;
+  return JEPA_B200_OK;
+}
+
+// Event pair around one launch while profiling is on.
+size_t prof_event(jepa_b200_model* m) {
+  if (m->prof_used == m->prof_events.size()) {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return SIZE_MAX;
+    m->prof_events.push_back(e);
+  }
+  return m->prof_used++;
+}
+
+struct ProfScope {
+  jepa_b200_model* m;
+  int cls;
+  cudaStream_t st;
+  size_t e0 = SIZE_MAX;
+  ProfScope(jepa_b200_model* m_, int cls_, cudaStream_t st_) : m(m_), cls(cls_), st(st_) {
+    if (m->prof) {
+      e0 = prof_event(m);
+      if (e0 != SIZE_MAX) cudaEventRecord(m->prof_events[e0], st);
+    }
+  }
+  ~ProfScope() {
+    if (m->prof && e0 != SIZE_MAX) {
+      const size_t e1 = prof_event(m);
+      if (e1 != SIZE_MAX) {
+        cudaEventRecord(m->prof_events[e1], st);
+        m->prof_recs.push_back({cls, e0, e1});
+      }
+    }
+  }
+};
+
+#define JB_TRY(expr)            \
+  do {                          \
+    const int _s = (expr);      \
+    if (_s != JEPA_B200_OK) return _s; \
+  } while (0)
+
+int run_block(jepa_b200_model* m, const LayerW& L, const BlockOps& ops, const AttnOp& at, float* Xres, int R,
+              cudaStream_t st) {
+  const int D = m->cfg.dim;
+  const float eps = m->cfg.ln_eps;
+  {
+    ProfScope ps(m, JEPA_B200_KC_LAYERNORM, st);
+    JB_TRY(launch_layernorm(Xres, R, D, 1, L.ln1_g, L.ln1_b, eps, m->Y, true, st));
+  }
+  {
+    ProfScope ps(m, JEPA_B200_KC_GEMM_QKV, st);
+    JB_TRY(gemm_launch(ops.qkv, st, m->err, m->timeout_ns));
+  }
+  {
+    ProfScope ps(m, JEPA_B200_KC_ATTENTION, st);
+    JB_TRY(attn_launch(at, st, m->err, m->timeout_ns));
+  }
+  {
+    ProfScope ps(m, JEPA_B200_KC_GEMM_OUT, st);
+    JB_TRY(gemm_launch(ops.out, st, m->err, m->timeout_ns));
+  }
+  {
+    ProfScope ps(m, JEPA_B200_KC_LAYERNORM, st);
+    JB_TRY(launch_layernorm(Xres, R, D, 1, L.ln2_g, L.ln2_b, eps, m->Y, true, st));
+  }
+  {
+    ProfScope ps(m, JEPA_B200_KC_GEMM_UP, st);
+    JB_TRY(gemm_launch(ops.up, st, m->err, m->timeout_ns));
+  }
+  {
+    ProfScope ps(m, JEPA_B200_KC_GEMM_DOWN, st);
+    JB_TRY(gemm_launch(ops.down, st, m->err, m->timeout_ns));
+  }
+  m->launches += 7;
+  return JEPA_B200_OK;
+}
+
+int run_embed_and_blocks(jepa_b200_model* m, const float* pixels, int B, int n_layers, cudaStream_t st) {
+  const jepa_b200_config& c = m->cfg;
+  const int R = B * m->N;
+  GemmOp pe = m->pe_op;
+  pe.p.patch.pixels = pixels;
+  {
+    ProfScope ps(m, JEPA_B200_KC_PATCH_EMBED, st);
+    JB_TRY(gemm_launch(pe, st, m->err, m->timeout_ns));
+    m->launches += 1;
+    if (c.has_cls) {
+      JB_TRY(launch_cls_rows(m->X, B, m->N, c.dim, m->cls, m->pos, st));
+      m->launches += 1;
+    }
+  }
+  for (int l = 0; l < n_layers; ++l) JB_TRY(run_block(m, m->enc[l], m->enc_ops[l], m->attn_enc, m->X, R, st));
+  return JEPA_B200_OK;
+}
+
+int run_head(jepa_b200_model* m, int B, float* out, cudaStream_t st) {
+  const jepa_b200_config& c = m->cfg;
+  const int R = B * m->N, D = c.dim;
+  const float eps = c.ln_eps;
+  for (size_t l = 0; l < m->head.size(); ++l)
+    JB_TRY(run_block(m, m->head[l], m->head_ops[l], m->attn_head, m->Yf, R, st));
+  ProfScope ps(m, JEPA_B200_KC_POOL_HEAD, st);
+  JB_TRY(launch_layernorm(m->Yf, R, D, 1, m->lnkv_g, m->lnkv_b, eps, m->Y, true, st));
+  JB_TRY(gemm_launch(m->kv_op, st, m->err, m->timeout_ns));
+  // q = W_q query + b_q (the learned query, shared by every clip)
+  JB_TRY(launch_gemv(m->query, 1, D, m->xq, m->b_xq, 0, nullptr, 0, m->hq, st));
+  JB_TRY(launch_xattn_1q(m->hq, m->Kb, m->Vt, B, c.heads, m->N, m->npad, m->hattn, st));
+  // z = query + W_out attn + b_out
+  JB_TRY(launch_gemv(m->hattn, B, D, m->xout, m->b_xout, 2, m->query, 0, m->hz, st));
+  JB_TRY(launch_layernorm(m->hz, B, D, 1, m->ln2x_g, m->ln2x_b, eps, m->hzn, false, st));
+  JB_TRY(launch_gemv(m->hzn, B, D, m->xup, m->b_xup, 1, nullptr, 0, m->hu, st));
+  JB_TRY(launch_gemv(m->hu, B, c.mlp, m->xdown, m->b_xdown, 2, m->hz, D, m->hz, st));
+  JB_TRY(launch_gemv(m->hz, B, D, m->hcls, m->b_cls, 0, nullptr, 0, out, st));
+  m->launches += 9;
+  return JEPA_B200_OK;
+}
+
+size_t out_elems(const jepa_b200_model* m, int B, int pool) {
+  switch (pool) {
+    case JEPA_B200_POOL_NONE: return static_cast<size_t>(B) * m->N * m->cfg.dim;
+    case JEPA_B200_POOL_MEAN:
+    case JEPA_B200_POOL_CLS: return static_cast<size_t>(B) * m->cfg.dim;
+    case JEPA_B200_POOL_ATTENTIVE: return static_cast<size_t>(B) * m->cfg.n_classes;
+    default: return 0;
+  }
+}
+
+int check_encode_args(jepa_b200_model* m, const void* pixels, int B, int pool, const void* out, size_t out_bytes) {
+  if (!m || !pixels || !out || B < 1) return JEPA_B200_ERR_ARG;
+  if (pool < JEPA_B200_POOL_NONE || pool > JEPA_B200_POOL_ATTENTIVE) return JEPA_B200_ERR_ARG;
+  if (pool == JEPA_B200_POOL_ATTENTIVE && !m->has_head) return JEPA_B200_ERR_MISSING_TENSOR;
+  if (pool == JEPA_B200_POOL_CLS && !m->cfg.has_cls) return JEPA_B200_ERR_ARG;
+  if (static_cast<long long>(B) * m->N > (1ll << 31) / 4096) return JEPA_B200_ERR_SHAPE;
+  if (out_bytes < out_elems(m, B, pool) * 4) return JEPA_B200_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(pixels) & 15) || (reinterpret_cast<uintptr_t>(out) & 15)) return JEPA_B200_ERR_ARG;
+  return JEPA_B200_OK;
+}
+
+}  // namespace
+
+static void load_sequence(Loader& L);
+
+extern "C" {
+
+const char* jepa_b200_status_str(int s) {
+  switch (s) {
+    case JEPA_B200_OK: return "ok";
+    case JEPA_B200_ERR_ARG: return "invalid argument";
+    case JEPA_B200_ERR_MISSING_TENSOR: return "missing tensor";
+    case JEPA_B200_ERR_SHAPE: return "wrong shape or size";
+    case JEPA_B200_ERR_DTYPE: return "dtype not allowed for this tensor";
+    case JEPA_B200_ERR_CUDA: return "CUDA call failed";
+    case JEPA_B200_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+    case JEPA_B200_ERR_UNSUPPORTED: return "not supported";
+    default: return "unknown status";
+  }
+}
+
+int jepa_b200_load_weights(const jepa_b200_config* cfg, const jepa_b200_tensor* table, int n_tensors, int device,
+                           jepa_b200_model** out_model) {
+  if (!out_model) return JEPA_B200_ERR_ARG;
+  *out_model = nullptr;
+  int s = validate_config(cfg);
+  if (s) return s;
+  if (!table || n_tensors < 1) return JEPA_B200_ERR_ARG;
+  if (device < 0) return JEPA_B200_ERR_ARG;
+  jepa_b200_model* m = new jepa_b200_model();
+  m->cfg = *cfg;
+  m->device = device;
+  const jepa_b200_config& c = *cfg;
+  m->ppf = (c.img_h / c.patch) * (c.img_w / c.patch);
+  m->Np = (c.frames / c.tubelet) * m->ppf;
+  m->N = m->Np + (c.has_cls ? 1 : 0);
+  m->npad = (m->N + 127) / 128 * 128;
+  m->Kpe = 3 * c.tubelet * c.patch * c.patch;
+  m->Kpe_pad = (m->Kpe + 63) / 64 * 64;
+  m->has_head = c.n_classes > 0;
+
+  for (int i = 0; i < n_tensors; ++i)
+    if (!table[i].name) {
+      delete m;
+      return JEPA_B200_ERR_ARG;
+    }
+  // pass 1 validates the whole table on the host; pass 2 converts and uploads
+  {
+    jepa_b200_model probe;
+    probe.cfg = m->cfg;
+    probe.N = m->N;
+    probe.Np = m->Np;
+    probe.Kpe = m->Kpe;
+    probe.Kpe_pad = m->Kpe_pad;
+    probe.has_head = m->has_head;
+    Loader V;
+    V.m = &probe;
+    V.dry = true;
+    for (int i = 0; i < n_tensors; ++i) V.tab[table[i].name] = &table[i];
+    load_sequence(V);
+    if (V.status != JEPA_B200_OK) {
+      delete m;
+      return V.status;
+    }
+  }
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    delete m;
+    return JEPA_B200_ERR_CUDA;
+  }
+  DeviceGuard guard(device);
+  Loader L;
+  L.m = m;
+  for (int i = 0; i < n_tensors; ++i) L.tab[table[i].name] = &table[i];
+  load_sequence(L);
+  if (L.status == JEPA_B200_OK) {
+    if (cudaMalloc(&m->err, sizeof(DevErr)) != cudaSuccess || cudaMemset(m->err, 0, sizeof(DevErr)) != cudaSuccess ||
+        cudaEventCreate(&m->ev0) != cudaSuccess || cudaEventCreate(&m->ev1) != cudaSuccess)
+      L.status = JEPA_B200_ERR_CUDA;
+  }
+  if (L.status != JEPA_B200_OK) {
+    jepa_b200_free(m);
+    return L.status;
+  }
+  *out_model = m;
+  return JEPA_B200_OK;
+}
+
+}  // extern "C"
+
+static void load_sequence(Loader& L) {
+  jepa_b200_model* m = L.m;
+  const jepa_b200_config& c = m->cfg;
+  const int64_t D = c.dim, Mh = c.mlp;
+  {
+    const jepa_b200_tensor* t = L.get("enc.patch_embed.weight", {D, 3, c.tubelet, c.patch, c.patch});
+    if (t && t->dtype != JEPA_B200_F32 && t->dtype != JEPA_B200_F16) L.status = JEPA_B200_ERR_DTYPE;
+    if (t && L.status == JEPA_B200_OK) m->pe = L.matrix({t}, m->Kpe, m->Kpe_pad);
+  }
+  m->b_pe = L.vec("enc.patch_embed.bias", D);
+  m->pos = L.table2d("enc.pos_embed", m->N, D);
+  if (c.has_cls) m->cls = L.vec("enc.cls_token", D);
+  m->enc.resize(c.depth);
+  for (int l = 0; l < c.depth; ++l) L.block(m->enc[l], "enc.blk." + std::to_string(l) + ".", D, Mh);
+  m->norm_g = L.vec("enc.norm.weight", D);
+  m->norm_b = L.vec("enc.norm.bias", D);
+  if (m->has_head) {
+    m->head.resize(c.head_sa_blocks);
+    for (int l = 0; l < c.head_sa_blocks; ++l) L.block(m->head[l], "head.blk." + std::to_string(l) + ".", D, Mh);
+    m->query = L.vec("head.query", D);
+    m->lnkv_g = L.vec("head.ln_kv.weight", D);
+    m->lnkv_b = L.vec("head.ln_kv.bias", D);
+    m->xq = L.mat("head.xattn.q.weight", D, D);
+    m->b_xq = L.vec("head.xattn.q.bias", D);
+    {
+      const jepa_b200_tensor* tk = L.get("head.xattn.k.weight", {D, D});
+      const jepa_b200_tensor* tv = L.get("head.xattn.v.weight", {D, D});
+      if (tk && tv) m->xkv = L.matrix({tk, tv}, D, D);
+      const jepa_b200_tensor* bk = L.get("head.xattn.k.bias", {D});
+      const jepa_b200_tensor* bv = L.get("head.xattn.v.bias", {D});
+      if (bk && bv) {
+        std::vector<float> v = L.host_floats(bk), w = L.host_floats(bv);
+        v.insert(v.end(), w.begin(), w.end());
+        m->b_xkv = static_cast<float*>(L.dalloc(v.size() * 4));
+        if (m->b_xkv) L.upload(m->b_xkv, v.data(), v.size() * 4);
+      }
+    }
+    m->xout = L.mat("head.xattn.out.weight", D, D);
+    m->b_xout = L.vec("head.xattn.out.bias", D);
+    m->ln2x_g = L.vec("head.xattn.ln2.weight", D);
+    m->ln2x_b = L.vec("head.xattn.ln2.bias", D);
+    m->xup = L.mat("head.xattn.ffn_up.weight", Mh, D);
+    m->b_xup = L.vec("head.xattn.ffn_up.bias", Mh);
+    m->xdown = L.mat("head.xattn.ffn_down.weight", D, Mh);
+    m->b_xdown = L.vec("head.xattn.ffn_down.bias", D);
+    m->hcls = L.mat("head.cls.weight", c.n_classes, D);
+    m->b_cls = L.vec("head.cls.bias", c.n_classes);
+  }
+}
+
+extern "C" {
+
+int jepa_b200_out_shape(const jepa_b200_model* m, int B, int pool, int64_t shape[3]) {
+  if (!m || !shape || B < 1) return JEPA_B200_ERR_ARG;
+  shape[0] = B;
+  shape[1] = shape[2] = 0;
+  switch (pool) {
+    case JEPA_B200_POOL_NONE:
+      shape[1] = m->N;
+      shape[2] = m->cfg.dim;
+      return 3;
+    case JEPA_B200_POOL_MEAN:
+      shape[1] = m->cfg.dim;
+      return 2;
+    case JEPA_B200_POOL_CLS:
+      if (!m->cfg.has_cls) return JEPA_B200_ERR_ARG;
+      shape[1] = m->cfg.dim;
+      return 2;
+    case JEPA_B200_POOL_ATTENTIVE:
+      if (!m->has_head) return JEPA_B200_ERR_MISSING_TENSOR;
+      shape[1] = m->cfg.n_classes;
+      return 2;
+    default:
+      return JEPA_B200_ERR_ARG;
+  }
+}
+
+int jepa_b200_encode(jepa_b200_model* m, const float* pixels, int B, int pool, float* out, size_t out_bytes,
+                     void* stream) {
+  int s = check_encode_args(m, pixels, B, pool, out, out_bytes);
+  if (s) return s;
+  DeviceGuard guard(m->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = ensure_workspace(m, B))) return s;
+  const jepa_b200_config& c = m->cfg;
+  const int R = B * m->N, D = c.dim;
+  m->launches = 0;
+  m->have_timing = false;
+  if (cudaEventRecord(m->ev0, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+  if ((s = run_embed_and_blocks(m, pixels, B, c.depth, st))) return s;
+  {
+    ProfScope ps(m, JEPA_B200_KC_LAYERNORM, st);
+    if (pool == JEPA_B200_POOL_NONE)
+      s = launch_layernorm(m->X, R, D, 1, m->norm_g, m->norm_b, c.ln_eps, out, false, st);
+    else if (pool == JEPA_B200_POOL_CLS)
+      s = launch_layernorm(m->X, B, D, m->N, m->norm_g, m->norm_b, c.ln_eps, out, false, st);
+    else
+      s = launch_layernorm(m->X, R, D, 1, m->norm_g, m->norm_b, c.ln_eps, m->Yf, false, st);
+    m->launches += 1;
+  }
+  if (!s && pool == JEPA_B200_POOL_MEAN) {
+    ProfScope ps(m, JEPA_B200_KC_POOL_HEAD, st);
+    s = launch_mean_pool(m->Yf, B, m->N, D, c.has_cls ? 1 : 0, m->partial, out, st);
+    m->launches += 2;
+  }
+  if (!s && pool == JEPA_B200_POOL_ATTENTIVE) s = run_head(m, B, out, st);
+  if (s) return s;
+  if (cudaEventRecord(m->ev1, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+  m->have_timing = true;
+  return JEPA_B200_OK;
+}
+
+int jepa_b200_encode_host(jepa_b200_model* m, const float* pixels, int B, int pool, float* out, size_t out_bytes,
+                          void* stream) {
+  int s = check_encode_args(m, pixels, B, pool, out, out_bytes);
+  if (s) return s;
+  DeviceGuard guard(m->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const jepa_b200_config& c = m->cfg;
+  const size_t pix_bytes = static_cast<size_t>(B) * c.frames * 3 * c.img_h * c.img_w * 4;
+  const size_t res_bytes = out_elems(m, B, pool) * 4;
+  if (pix_bytes > m->stage_pix_bytes) {
+    cudaDeviceSynchronize();
+    if (m->stage_pix) cudaFree(m->stage_pix);
+    m->stage_pix = nullptr;
+    m->stage_pix_bytes = 0;
+    if (cudaMalloc(&m->stage_pix, pix_bytes) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+    m->stage_pix_bytes = pix_bytes;
+  }
+  if (res_bytes > m->stage_out_bytes) {
+    cudaDeviceSynchronize();
+    if (m->stage_out) cudaFree(m->stage_out);
+    m->stage_out = nullptr;
+    m->stage_out_bytes = 0;
+    if (cudaMalloc(&m->stage_out, res_bytes) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+    m->stage_out_bytes = res_bytes;
+  }
+  if (cudaMemcpyAsync(m->stage_pix, pixels, pix_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return JEPA_B200_ERR_CUDA;
+  if ((s = jepa_b200_encode(m, m->stage_pix, B, pool, m->stage_out, res_bytes, stream))) return s;
+  if (cudaMemcpyAsync(out, m->stage_out, res_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return JEPA_B200_ERR_CUDA;
+  return jepa_b200_sync_status(m, stream);
+}
+
+int jepa_b200_debug_stage(jepa_b200_model* m, const float* pixels, int B, int layer, int stage, float* out,
+                          size_t out_bytes, void* stream) {
+  if (!m || !pixels || !out || B < 1 || stage != 0) return JEPA_B200_ERR_ARG;
+  if (layer < 0 || layer > m->cfg.depth) return JEPA_B200_ERR_ARG;
+  const size_t need = static_cast<size_t>(B) * m->N * m->cfg.dim * 4;
+  if (out_bytes < need) return JEPA_B200_ERR_SHAPE;
+  DeviceGuard guard(m->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int s;
+  if ((s = ensure_workspace(m, B))) return s;
+  m->launches = 0;
+  if ((s = run_embed_and_blocks(m, pixels, B, layer, st))) return s;
+  if (cudaMemcpyAsync(out, m->X, need, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+  return JEPA_B200_OK;
+}
+
+int jepa_b200_sync_status(jepa_b200_model* m, void* stream) {
+  if (!m) return JEPA_B200_ERR_ARG;
+  DeviceGuard guard(m->device);
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+  DevErr e{0, 0};
+  if (cudaMemcpy(&e, m->err, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+  if (e.code != DERR_NONE) {
+    cudaMemset(m->err, 0, sizeof(DevErr));
+    return e.code == DERR_TIMEOUT ? JEPA_B200_ERR_TIMEOUT : JEPA_B200_ERR_CUDA;
+  }
+  return JEPA_B200_OK;
+}
+
+double jepa_b200_last_ms(jepa_b200_model* m) {
+  if (!m || !m->have_timing) return -1.0;
+  DeviceGuard guard(m->device);
+  if (cudaEventSynchronize(m->ev1) != cudaSuccess) return -1.0;
+  float ms = 0.0f;
+  if (cudaEventElapsedTime(&ms, m->ev0, m->ev1) != cudaSuccess) return -1.0;
+  return ms;
+}
+
+size_t jepa_b200_model_n_bytes(const jepa_b200_model* m) { return m ? m->weight_bytes : 0; }
+
+int jepa_b200_set_timeout_ns(jepa_b200_model* m, unsigned long long ns) {
+  if (!m) return JEPA_B200_ERR_ARG;
+  m->timeout_ns = ns;
+  return JEPA_B200_OK;
+}
+
+int jepa_b200_last_launch_count(const jepa_b200_model* m) { return m ? m->launches : -1; }
+
+int jepa_b200_set_profiling(jepa_b200_model* m, int enable) {
+  if (!m) return JEPA_B200_ERR_ARG;
+  m->prof = enable != 0;
+  return JEPA_B200_OK;
+}
+
+int jepa_b200_profile_read(jepa_b200_model* m, double* ms, int* launches, int n) {
+  if (!m || !ms || !launches || n < JEPA_B200_KC_COUNT) return JEPA_B200_ERR_ARG;
+  DeviceGuard guard(m->device);
+  for (int i = 0; i < n; ++i) {
+    ms[i] = 0.0;
+    launches[i] = 0;
+  }
+  int s = JEPA_B200_OK;
+  for (const auto& r : m->prof_recs) {
+    float t = 0.0f;
+    if (cudaEventSynchronize(m->prof_events[r.e1]) != cudaSuccess ||
+        cudaEventElapsedTime(&t, m->prof_events[r.e0], m->prof_events[r.e1]) != cudaSuccess) {
+      s = JEPA_B200_ERR_CUDA;
+      continue;
+    }
+    ms[r.cls] += t;
+    launches[r.cls] += 1;
+  }
+  m->prof_recs.clear();
+  m->prof_used = 0;
+  return s;
+}
+
+void jepa_b200_free(jepa_b200_model* m) {
+  if (!m) return;
+  DeviceGuard guard(m->device);
+  cudaDeviceSynchronize();
+  free_list(m->ws_allocs);
+  free_list(m->allocs);
+  if (m->stage_pix) cudaFree(m->stage_pix);
+  if (m->stage_out) cudaFree(m->stage_out);
+  if (m->err) cudaFree(m->err);
+  if (m->ev0) cudaEventDestroy(m->ev0);
+  if (m->ev1) cudaEventDestroy(m->ev1);
+  for (cudaEvent_t e : m->prof_events) cudaEventDestroy(e);
+  delete m;
+}
+
+}  // extern "C"

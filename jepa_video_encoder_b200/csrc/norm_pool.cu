@@ -1,0 +1,175 @@
+// Memory-bound kernels of the encoder forward: the fused LayerNorm (pre-LN
+// block norms, the final `norm`, the head's ln_kv / ln2), the CLS rows of the
+// embedding, mean pooling over the patch tokens, and the byte repack of
+// q8_0 / q4_0 blocks into the GEMM's layout.
+//
+// LayerNorm: y = (x - mean) / sqrt(var + eps) * gamma + beta over each row,
+// biased variance, statistics in f32 from a row held in registers (two
+// passes over registers, one pass over HBM).  One warp per row.
+#include <algorithm>
+
+#include "internal.h"
+
+namespace jb {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int MAXV, bool OUT_F16>
+__global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict__ x, int rows, int D,
+                                                       long long in_stride, const float* __restrict__ g,
+                                                       const float* __restrict__ b, float eps, void* out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= rows) return;
+  const int nv = D >> 2;
+  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(row) * in_stride * D);
+  float4 v[MAXV];
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int idx = lane + 32 * i;
+    if (idx < nv) {
+      v[i] = __ldg(xr + idx);
+      s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+    } else {
+      v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  const float mean = warp_sum(s) / static_cast<float>(D);
+  float q = 0.0f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    if (lane + 32 * i < nv) {
+      const float a = v[i].x - mean, bb = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
+      q += (a * a + bb * bb) + (c * c + d * d);
+    }
+  }
+  const float rstd = rsqrtf(warp_sum(q) / static_cast<float>(D) + eps);
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  const float4* b4 = reinterpret_cast<const float4*>(b);
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int idx = lane + 32 * i;
+    if (idx < nv) {
+      const float4 gg = __ldg(g4 + idx), bb = __ldg(b4 + idx);
+      const float y0 = (v[i].x - mean) * rstd * gg.x + bb.x;
+      const float y1 = (v[i].y - mean) * rstd * gg.y + bb.y;
+      const float y2 = (v[i].z - mean) * rstd * gg.z + bb.z;
+      const float y3 = (v[i].w - mean) * rstd * gg.w + bb.w;
+      if (OUT_F16) {
+        uint2* o = reinterpret_cast<uint2*>(static_cast<__half*>(out) + static_cast<size_t>(row) * D) + idx;
+        *o = make_uint2(pack_half2(y0, y1), pack_half2(y2, y3));
+      } else {
+        float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + static_cast<size_t>(row) * D) + idx;
+        *o = make_float4(y0, y1, y2, y3);
+      }
+    }
+  }
+}
+
+int launch_layernorm(const float* x, int rows, int D, long long in_stride, const float* g, const float* b,
+                     float eps, void* out, bool out_f16, cudaStream_t st) {
+  if (!x || !g || !b || !out) return JEPA_B200_ERR_ARG;
+  if (rows < 1 || D < 4 || D % 4 != 0 || D > 4096 || in_stride < 1) return JEPA_B200_ERR_SHAPE;
+  const dim3 grid((rows + 7) / 8);
+  if (D <= 1024) {
+    if (out_f16)
+      layernorm_kernel<8, true><<<grid, 256, 0, st>>>(x, rows, D, in_stride, g, b, eps, out);
+    else
+      layernorm_kernel<8, false><<<grid, 256, 0, st>>>(x, rows, D, in_stride, g, b, eps, out);
+  } else {
+    if (out_f16)
+      layernorm_kernel<32, true><<<grid, 256, 0, st>>>(x, rows, D, in_stride, g, b, eps, out);
+    else
+      layernorm_kernel<32, false><<<grid, 256, 0, st>>>(x, rows, D, in_stride, g, b, eps, out);
+  }
+  return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+}
+
+// x[b, 0, :] = cls + pos[0]
+__global__ void cls_rows_kernel(float* x, int B, int ntok, int D, const float* cls, const float* pos) {
+  const int b = blockIdx.y;
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < D; c += gridDim.x * blockDim.x)
+    x[static_cast<size_t>(b) * ntok * D + c] = cls[c] + pos[c];
+}
+
+int launch_cls_rows(float* x, int B, int ntok, int D, const float* cls, const float* pos, cudaStream_t st) {
+  if (!x || !cls || !pos) return JEPA_B200_ERR_ARG;
+  cls_rows_kernel<<<dim3((D + 255) / 256, B), 256, 0, st>>>(x, B, ntok, D, cls, pos);
+  return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+}
+
+// Mean pooling over rows first..ntok-1 of each clip, deterministic two-stage
+// reduction: column sums over row chunks, then the chunk sums.
+constexpr int kPoolSplits = 32;
+
+__global__ void mean_pool_partial_kernel(const float* __restrict__ y, int ntok, int D, int first,
+                                         float* __restrict__ partial) {
+  const int col = blockIdx.x * 256 + threadIdx.x;
+  const int sp = blockIdx.y, b = blockIdx.z;
+  if (col >= D) return;
+  const int n_rows = ntok - first;
+  const int per = (n_rows + kPoolSplits - 1) / kPoolSplits;
+  const int r0 = first + sp * per, r1 = min(ntok, r0 + per);
+  const float* base = y + static_cast<size_t>(b) * ntok * D + col;
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+  int r = r0;
+  for (; r + 3 < r1; r += 4) {
+    s0 += __ldg(base + static_cast<size_t>(r) * D);
+    s1 += __ldg(base + static_cast<size_t>(r + 1) * D);
+    s2 += __ldg(base + static_cast<size_t>(r + 2) * D);
+    s3 += __ldg(base + static_cast<size_t>(r + 3) * D);
+  }
+  for (; r < r1; ++r) s0 += __ldg(base + static_cast<size_t>(r) * D);
+  partial[(static_cast<size_t>(b) * kPoolSplits + sp) * D + col] = (s0 + s1) + (s2 + s3);
+}
+
+__global__ void mean_pool_final_kernel(const float* __restrict__ partial, int B, int D, float inv_count,
+                                       float* __restrict__ out) {
+  const int i = blockIdx.x * 256 + threadIdx.x;
+  if (i >= B * D) return;
+  const int b = i / D, col = i % D;
+  float s = 0.f;
+  for (int sp = 0; sp < kPoolSplits; ++sp) s += partial[(static_cast<size_t>(b) * kPoolSplits + sp) * D + col];
+  out[i] = s * inv_count;
+}
+
+int mean_pool_partial_floats(int B, int D) { return B * kPoolSplits * D; }
+
+int launch_mean_pool(const float* y, int B, int ntok, int D, int first, float* partial, float* out,
+                     cudaStream_t st) {
+  if (!y || !partial || !out) return JEPA_B200_ERR_ARG;
+  if (B < 1 || D < 1 || first < 0 || first >= ntok || B > 65535) return JEPA_B200_ERR_SHAPE;
+  mean_pool_partial_kernel<<<dim3((D + 255) / 256, kPoolSplits, B), 256, 0, st>>>(y, ntok, D, first, partial);
+  mean_pool_final_kernel<<<(B * D + 255) / 256, 256, 0, st>>>(partial, B, D, 1.0f / (ntok - first), out);
+  return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+}
+
+// Repack [N, K/32] q8_0 (34-byte) or q4_0 (18-byte) blocks into
+// qs [N, K] int8 or [N, K/2] nibble bytes (block order kept) + scales [N, K/32].
+__global__ void repack_kernel(int bmode, const uint8_t* __restrict__ blocks, long long nblocks, uint8_t* qs,
+                              uint16_t* scales) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= nblocks) return;
+  const int bsz = bmode == B_Q8 ? 34 : 18;
+  const int qbytes = bmode == B_Q8 ? 32 : 16;
+  const uint8_t* src = blocks + i * bsz;
+  scales[i] = static_cast<uint16_t>(src[0] | (src[1] << 8));
+  uint8_t* dst = qs + i * qbytes;
+  for (int j = 0; j < qbytes; ++j) dst[j] = src[2 + j];
+}
+
+int launch_repack(int bmode, const uint8_t* blocks, int N, int K, void* qs, __half* scales, cudaStream_t st) {
+  if (!blocks || !qs || !scales) return JEPA_B200_ERR_ARG;
+  if ((bmode != B_Q8 && bmode != B_Q4) || N < 1 || K < 32 || K % 32 != 0) return JEPA_B200_ERR_SHAPE;
+  const long long nb = static_cast<long long>(N) * (K / 32);
+  repack_kernel<<<static_cast<unsigned>((nb + 255) / 256), 256, 0, st>>>(
+      bmode, blocks, nb, static_cast<uint8_t*>(qs), reinterpret_cast<uint16_t*>(scales));
+  return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+}
+
+}  // namespace jb

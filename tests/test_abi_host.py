@@ -1,0 +1,147 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol include/jepa_b200.h declares, and rejects bad arguments and bad
+tensor tables before any device work."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+from jepa_video_encoder_b200 import _abi, build, synth, make_config
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "jepa_b200.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _abi.load_library()
+
+
+def header_functions():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"JEPA_B200_API\s+[^;(]*?\b(jepa_b200_\w+)\s*\(", txt)))
+
+
+def test_header_declares_functions():
+    names = header_functions()
+    assert "jepa_b200_load_weights" in names and "jepa_b200_encode" in names
+    assert len(names) >= 20
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = header_functions()
+    out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(l.split()[-1] for l in out.splitlines() if " T " in l)
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(lib, n)
+    # the binding declares exactly the header's functions
+    assert sorted(_abi.SIGNATURES) == names
+
+
+def test_status_strings(lib):
+    for s in range(0, -8, -1):
+        assert _abi.status_str(s)
+    assert _abi.status_str(_abi.ERR_TIMEOUT).startswith("a bounded")
+
+
+def _tiny_cfg(**kw):
+    base = synth.EncoderConfig(name="t", dim=128, depth=1, heads=2, mlp=256, patch=8, tubelet=1, img_h=16,
+                               img_w=16, frames=2, has_cls=True, mask="block_causal", weights="f16", batch=1,
+                               pool="cls")
+    return base.with_(**kw)
+
+
+def _load(lib, cfg, table):
+    entries = (_abi.TensorEntry * len(table))()
+    keep = []
+    for i, t in enumerate(table):
+        nm = t.name.encode()
+        keep.append(nm)
+        entries[i].name = nm
+        entries[i].dtype = t.dtype
+        entries[i].ndim = len(t.shape)
+        for j, s in enumerate(t.shape):
+            entries[i].shape[j] = s
+        entries[i].data = t.data.ctypes.data
+        entries[i].nbytes = t.nbytes
+    c = make_config(cfg)
+    h = ctypes.c_void_p()
+    st = lib.jepa_b200_load_weights(ctypes.byref(c), entries, len(table), 0, ctypes.byref(h))
+    if st == 0:
+        lib.jepa_b200_free(h)
+    return st
+
+
+def _has_gpu():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+def test_table_validation(lib):
+    cfg = _tiny_cfg()
+    table = synth.make_tensor_table(cfg)
+    full = _load(lib, cfg, table)
+    # a complete table passes validation; without a device the upload then fails
+    assert full == (0 if _has_gpu() else _abi.ERR_CUDA)
+    assert _load(lib, cfg, [t for t in table if t.name != "enc.blk.0.ffn_up.bias"]) == _abi.ERR_MISSING_TENSOR
+    bad = list(table)
+    i = [t.name for t in bad].index("enc.blk.0.ln1.weight")
+    bad[i] = synth.Tensor(bad[i].name, synth.DT_Q8_0, bad[i].shape,
+                          synth.quantize_q8_0(np.ones(cfg.dim, np.float32)))
+    assert _load(lib, cfg, bad) == _abi.ERR_DTYPE
+    bad = list(table)
+    i = [t.name for t in bad].index("enc.pos_embed")
+    bad[i] = synth.Tensor(bad[i].name, synth.DT_F32, (cfg.n_tokens - 1, cfg.dim),
+                          np.zeros((cfg.n_tokens - 1, cfg.dim), np.float32))
+    assert _load(lib, cfg, bad) == _abi.ERR_SHAPE
+    bad = list(table)
+    i = [t.name for t in bad].index("enc.blk.0.attn_out.weight")
+    bad[i] = synth.Tensor(bad[i].name, bad[i].dtype, bad[i].shape, bad[i].data[:-1])   # nbytes off by one row
+    assert _load(lib, cfg, bad) == _abi.ERR_SHAPE
+
+
+def test_quantised_table_validation(lib):
+    cfg = _tiny_cfg(weights="q8_0")
+    table = synth.make_tensor_table(cfg)
+    assert _load(lib, cfg, table) == (0 if _has_gpu() else _abi.ERR_CUDA)
+    # quantised blocks are refused outside the re-typed matrices
+    bad = list(table)
+    i = [t.name for t in bad].index("enc.patch_embed.weight")
+    w = np.zeros((cfg.dim, 3 * 8 * 8), np.float32)
+    bad[i] = synth.Tensor(bad[i].name, synth.DT_Q8_0, bad[i].shape, synth.quantize_q8_0(w))
+    assert _load(lib, cfg, bad) == _abi.ERR_DTYPE
+
+
+def test_bad_config(lib):
+    cfg = _tiny_cfg()
+    table = synth.make_tensor_table(cfg)
+    assert _load(lib, cfg.with_(heads=3), table) == _abi.ERR_SHAPE       # dim != 64 * heads
+    assert _load(lib, cfg.with_(img_h=20), table) == _abi.ERR_SHAPE      # not a multiple of the patch
+    c = make_config(cfg)
+    c.mask = 7
+    h = ctypes.c_void_p()
+    assert lib.jepa_b200_load_weights(ctypes.byref(c), None, 0, 0, ctypes.byref(h)) == _abi.ERR_ARG
+
+
+def test_null_arguments(lib):
+    shp = (ctypes.c_int64 * 3)()
+    assert lib.jepa_b200_out_shape(None, 1, 0, shp) == _abi.ERR_ARG
+    assert lib.jepa_b200_encode(None, None, 1, 0, None, 0, None) == _abi.ERR_ARG
+    assert lib.jepa_b200_encode_host(None, None, 1, 0, None, 0, None) == _abi.ERR_ARG
+    assert lib.jepa_b200_debug_stage(None, None, 1, 0, 0, None, 0, None) == _abi.ERR_ARG
+    assert lib.jepa_b200_op_layernorm(None, 4, 64, 1, None, None, 1e-6, None, 1, None) == _abi.ERR_ARG
+    assert lib.jepa_b200_op_linear(None, 4, 64, None, None, 1, 128, None, 0, None, 128, None) == _abi.ERR_ARG
+    assert lib.jepa_b200_op_linear(None, 4, 64, None, None, 5, 128, None, 0, None, 128, None) == _abi.ERR_ARG
+    assert lib.jepa_b200_op_gemv(None, 1, 64, None, None, 1, 8, None, 7, None, 0, None, None) == _abi.ERR_ARG
+    assert lib.jepa_b200_model_n_bytes(None) == 0
+    assert lib.jepa_b200_last_ms(None) < 0
+    lib.jepa_b200_free(None)
