@@ -218,6 +218,13 @@ def run_ours(args, cfg, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     if model.sync_status(stream) != 0:
         raise RuntimeError("device error during warm-up")
+    if args.forward_only:   # a fixed number of plain forwards, for profiler launch lists
+        for _ in range(args.steps):
+            step()
+        torch.cuda.synchronize(dev)
+        st = model.sync_status(stream)
+        model.close()
+        return 0 if st == 0 else 1
 
     # ---- timed region: K steps, each between CUDA events, L2 flushed between steps
     clock_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv") if os.path.isdir(
@@ -346,6 +353,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
+    ap.add_argument("--forward-only", action="store_true",
+                    help="run warm-up + --steps forwards and exit (no timing, no JSON): for ncu launch lists")
     args = ap.parse_args()
     cfg = synth.WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -245,8 +245,11 @@ __global__ void __launch_bounds__(192, 2)
           break;
         }
         tc_fence_after();
-        if (m_new > m_run && m_run != -INFINITY) {
-          const float alpha = ex2_approx(m_run - m_new);
+        // tcgen05.ld / st are warp-collective: the whole warp rescales its
+        // rows when any of them saw a larger max (the others scale by 1).
+        const bool grow = m_new > m_run && m_run != -INFINITY;
+        if (__any_sync(0xffffffffu, grow)) {
+          const float alpha = grow ? ex2_approx(m_run - m_new) : 1.0f;
           l_run *= alpha;
 #pragma unroll 1
           for (int c = 0; c < 2; ++c) {

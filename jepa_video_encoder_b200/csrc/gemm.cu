@@ -14,10 +14,11 @@
 //   warp 1      MMA issuer: tcgen05.mma kind::f16 M=128 N=BN K=16, f32
 //               accumulators in TMEM, two accumulator buffers so the
 //               epilogue of tile i overlaps the main loop of tile i+1;
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator rows, bias, then
+//   warps 2-9   epilogue: tcgen05.ld of the accumulator rows (two warps per
+//               TMEM lane quadrant, each half of the columns), bias, then
 //               f16 store / GELU / f32 residual add / QKV head scatter /
 //               patch-embed + pos_embed;
-//   warps 6-9   (quantised weights or patch-embed only) converters: unpack
+//   warps 10-13 (quantised weights or patch-embed only) converters: unpack
 //               q8_0 (q*d) or q4_0 ((q-8)*d) blocks, or gather pixels, into
 //               the swizzled operand tile in shared memory.
 #include <cudaTypedefs.h>
@@ -211,7 +212,7 @@ __device__ __forceinline__ void fill_a_patch(uint8_t* sA, const GemmParams& p, i
 }
 
 template <int BN, int BMODE, bool GATHER>
-__global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 320 : 192, 1)
+__global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
   using C = GemmCfg<BN>;
@@ -234,7 +235,7 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 320 : 192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 128);
+      mbar_init(&tempty_bar[a], 256);
     }
     mbar_init(&drain_bar, 1);
     abort_sh = 0;
@@ -339,8 +340,11 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 320 : 192, 1)
       tc_commit(&drain_bar);
       mbar_wait_drain(&drain_bar, 0);
     }
-  } else if (warp < 6) {
+  } else if (warp < 10) {
+    // 8 epilogue warps: warps w and w+4 read the same TMEM lane quadrant
+    // (w % 4) and split the tile's columns in two halves.
     const int quad = warp & 3;
+    const int chalf = (warp - 2) >> 2;
     int acc = 0;
     uint32_t aphase = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
@@ -352,7 +356,7 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 320 : 192, 1)
       const int row = mb * 128 + quad * 32 + lane;
       const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = chalf * (BN / 64); c < (chalf + 1) * (BN / 64); ++c) {
         uint32_t r[32];
         tmem_ld32(tb + static_cast<uint32_t>(c * 32), r);
         if (row < p.M) epilogue_chunk(p, row, nb * BN + c * 32, r);
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 320 : 192, 1)
       }
     }
   } else if (CONV) {
-    const int ct = threadIdx.x - 192;
+    const int ct = threadIdx.x - 320;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -499,7 +503,7 @@ static int launch_impl(const GemmOp& op, cudaStream_t st) {
       return JEPA_B200_ERR_CUDA;
     attr_done |= 1ull << dev;
   }
-  constexpr int threads = (BMODE != B_F16 || GATHER) ? 320 : 192;
+  constexpr int threads = (BMODE != B_F16 || GATHER) ? 448 : 320;
   kern<<<op.grid, threads, GemmCfg<BN>::SMEM, st>>>(op.tmA, op.tmB, op.p);
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
