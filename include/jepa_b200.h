@@ -279,6 +279,24 @@ JEPA_B200_API int jepa_b200_op_xattn_1q(const float *q, const void *k, const voi
 /* Mean over rows first..ntok-1 of each clip of y f32 [B, ntok, D] -> out f32 [B, D]. */
 JEPA_B200_API int jepa_b200_op_mean_pool(const float *y, int B, int ntok, int D, int first, float *out, void *stream);
 
+/* Mean pooling that allocates nothing, for callers that cannot call
+ * cudaMalloc (work recorded into a CUDA graph, serving loops under a fixed
+ * device-memory budget or that must not synchronise the device, hosts whose
+ * allocator belongs to another framework).  There is no counterpart on the
+ * pages: it is jepa_b200_op_mean_pool with its partial sums kept in a fixed
+ * file-scope device array (4 MiB on every GPU that loads the library, held
+ * until exit) instead of a buffer grown with cudaMalloc.
+ * y f32 [B, ntok, D] -> out f32 [B, D] (mean over rows first..ntok-1), device
+ * pointers.  Limit: B * D <= 32768; larger sizes return ERR_SHAPE before any
+ * device work.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  Every call shares the array and overwrites
+ * the partial sums it reads, so its previous contents never matter, but calls
+ * that overlap on the GPU (two streams, two host threads) race on it.
+ * Returns OK, ERR_ARG, ERR_SHAPE or ERR_CUDA. */
+JEPA_B200_API int jepa_b200_op_mean_pool_noalloc(const float *y, int B, int ntok, int D, int first, float *out,
+                                                 void *stream);
+
 /* Synchronise `stream`, return and clear the device status of the op calls
  * (OK, ERR_TIMEOUT, ERR_CUDA). */
 JEPA_B200_API int jepa_b200_op_sync_status(void *stream);

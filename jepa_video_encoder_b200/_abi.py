@@ -59,6 +59,7 @@ SIGNATURES = {
     "jepa_b200_op_xattn_1q": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p,
                                       c_void_p]),
     "jepa_b200_op_mean_pool": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p]),
+    "jepa_b200_op_mean_pool_noalloc": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p]),
     "jepa_b200_op_sync_status": (c_int, [c_void_p]),
     "jepa_b200_op_set_timeout_ns": (None, [c_ulonglong]),
 }
