@@ -196,7 +196,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     import jepa_video_encoder_b200 as jb
     from jepa_video_encoder_b200 import build as jbuild
 
-    if rank == 0 or not os.path.exists(jbuild.LIB):
+    if rank == 0 and not os.path.exists(jbuild.LIB):
         jbuild.build()
     if world > 1:
         torch.distributed.barrier()

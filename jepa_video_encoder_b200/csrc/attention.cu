@@ -7,18 +7,28 @@
 // every query row the allowed keys form one interval [lo, hi]:
 //   CLS row:            [0, N-1]
 //   patch of slot s:    [c, c + (s+1) * P_f - 1]   (c = 1 with a CLS row)
-// so a query tile only visits KV tiles up to its largest hi; tiles past it
-// are never loaded (the skipped, fully masked tiles).
+// so a query tile only visits KV tiles up to its largest hi (the fully masked
+// tiles past it are never loaded), and only tiles that cut an interval need
+// the per-element mask.  The CLS row, the one row that reads every key, gets
+// a CTA of its own (scheduled first), so that its query tile in the regular
+// CTAs stays as short as the first frame's.
 //
-// One CTA per (128-query tile, clip*head); two CTAs per SM so one CTA's
-// softmax overlaps the other's tensor-core work.
-//   warp 0     TMA: Q tile once, K tiles (2 stages) and V^T tiles;
-//   warp 1     MMA: S = Q K^T into TMEM (M=128, N=128), then O += P V into
-//              TMEM (M=128, N=64) with P from shared memory;
-//   warps 2-5  softmax, one thread per query row: row max from TMEM, O
-//              rescaled in TMEM when the max grows, P = exp2(.) written as
-//              f16 into the swizzled A tile of the PV product, row sum in f32;
-//              at the end O / l is written token-major for the out-projection.
+// One CTA per (pair of 128-query tiles, clip*head), one CTA per SM:
+//   warp 0      TMA: both Q tiles once, then K and V^T tiles through a
+//               2-stage ring shared by the two query tiles;
+//   warps 1,10  MMA, one issuer per query tile g: for each KV tile j,
+//               S_g = Q_g K_j^T into TMEM (M=128, N=128) and O_g += P_g V_{j-1}
+//               into TMEM (M=128, N=64, P from shared memory); the tensor core
+//               works on one tile while the other tile's softmax runs;
+//   warps 2-5   softmax of query tile 0, warps 6-9 of query tile 1, one
+//               thread per query row: scores read once from TMEM into
+//               registers (S is released at once for the next KV tile), row
+//               max, O rescaled in TMEM only when the max grew by more than
+//               2^8 (lazy rescaling: P stays <= 256, exact after the final
+//               division by the row sum), P = exp2(s*c - m) written as f16
+//               into the swizzled A tile of the PV product; two P buffers per
+//               query tile, so tile j's softmax only waits for the PV product
+//               of tile j-2 (and for tile j-1's when it has to rescale O).
 #include <string.h>
 
 #include <algorithm>
@@ -28,11 +38,14 @@
 namespace jb {
 
 namespace {
-constexpr int kQBytes = 128 * 64 * 2;   // Q tile [128 x 64]
-constexpr int kKBytes = 128 * 64 * 2;   // K tile [128 keys x 64]
-constexpr int kVBytes = 64 * 128 * 2;   // V^T tile [64 dims x 128 keys] as two [64 x 64] halves
-constexpr int kPBytes = 128 * 128 * 2;  // P tile [128 x 128 keys] as two [128 x 64] halves
-constexpr int kAttnSmem = kQBytes + 2 * kKBytes + kVBytes + kPBytes + 1024;
+constexpr int kTile = 128 * 64 * 2;  // one [128 x 64] f16 tile, 16 KB
+constexpr int kStages = 2;
+constexpr int kOffQ = 0;                           // Q0, Q1
+constexpr int kOffK = kOffQ + 2 * kTile;           // K ring
+constexpr int kOffV = kOffK + kStages * kTile;     // V^T ring, each [64 dims x 128 keys] as two [64 x 64]
+constexpr int kOffP = kOffV + kStages * kTile;     // P[g][b]: query tile g, buffer b, each [128 x 128 keys]
+constexpr int kAttnSmem = kOffP + 2 * 2 * 2 * kTile + 1024;  // as two [128 x 64] halves
+constexpr float kRescaleLog2 = 8.0f;  // rescale O when the row max grew by more than 2^8
 }  // namespace
 
 __device__ __forceinline__ void key_range(const AttnParams& p, int i, int& lo, int& hi) {
@@ -40,11 +53,11 @@ __device__ __forceinline__ void key_range(const AttnParams& p, int i, int& lo, i
   hi = p.N - 1;
   if (p.mask == JEPA_B200_MASK_BLOCK_CAUSAL && i < p.N) {
     if (p.has_cls) {
-      if (i > 0) {
-        const int s = (i - 1) / p.ppf;
-        lo = 1;
-        hi = (s + 1) * p.ppf;
-      }
+      // row 0 (CLS) reads every key; its own CTA computes it, and in the
+      // pair CTAs it takes slot 0's range so that its tile stays short
+      const int s = i > 0 ? (i - 1) / p.ppf : 0;
+      lo = 1;
+      hi = (s + 1) * p.ppf;
     } else {
       const int s = i / p.ppf;
       hi = (s + 1) * p.ppf - 1;
@@ -53,57 +66,68 @@ __device__ __forceinline__ void key_range(const AttnParams& p, int i, int& lo, i
   }
 }
 
-__global__ void __launch_bounds__(192, 2)
+// Number of KV tiles query tile starting at q0 must visit (0: no valid row).
+__device__ __forceinline__ int kv_tiles(const AttnParams& p, int q0) {
+  if (q0 >= p.N) return 0;
+  int lo_a, hi_a, lo_b, hi_b;
+  key_range(p, q0, lo_a, hi_a);
+  key_range(p, min(q0 + 127, p.N - 1), lo_b, hi_b);
+  return (max(hi_a, hi_b) + 1 + 127) / 128;
+}
+
+__global__ void __launch_bounds__(352, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   extern __shared__ uint8_t dsmem[];
-  __shared__ uint64_t q_full, k_full[2], k_empty[2], v_full, v_empty, s_full, p_full, pv_done, drain_bar;
+  __shared__ uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  // per query tile g: S ready / S taken, and per P buffer b: P written / PV done
+  __shared__ uint64_t s_full[2], s_free[2], p_full[2][2], pv_done[2][2], drain_bar[2];
   __shared__ uint32_t tmem_sh;
   __shared__ int abort_sh;
 
   const uint32_t raw = smem_u32(dsmem);
   uint8_t* sm = dsmem + ((1024u - (raw & 1023u)) & 1023u);
-  uint8_t* sQ = sm;
-  uint8_t* sK0 = sm + kQBytes;
-  uint8_t* sV = sK0 + 2 * kKBytes;
-  uint8_t* sP = sV + kVBytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = p.n_q_tiles - 1 - static_cast<int>(blockIdx.x);  // late (heavier) tiles first
+  const int n_pairs = (p.n_q_tiles + 1) / 2;
   const int bh = blockIdx.y;
-  const int q0 = qt * 128;
-
-  // KV tiles this query tile needs: up to the largest hi over its rows.
-  int lo_a, hi_a, lo_b, hi_b;
-  key_range(p, q0, lo_a, hi_a);
-  key_range(p, min(q0 + 127, p.N - 1), lo_b, hi_b);
-  const int kv_end = max(hi_a, hi_b) + 1;
-  const int n_kv = (kv_end + 127) / 128;
+  // With a separate CLS row, CTA 0 computes the CLS row alone (query tile 0
+  // against every KV tile); the pair CTAs follow, later (heavier) tiles first.
+  const bool cls_cta = p.cls_separate && blockIdx.x == 0;
+  const int pair = n_pairs - 1 - (static_cast<int>(blockIdx.x) - p.cls_separate);
+  const int q00 = cls_cta ? 0 : 2 * pair * 128, q01 = q00 + 128;  // first rows of query tiles 0 and 1
+  const int nkv0 = cls_cta ? (p.N + 127) / 128 : kv_tiles(p, q00);
+  const int nkv1 = cls_cta ? 0 : kv_tiles(p, q01);
+  const int nkv_all = max(nkv0, nkv1);
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 2);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 2);
     }
-    mbar_init(&v_full, 1);
-    mbar_init(&v_empty, 1);
-    mbar_init(&s_full, 1);
-    mbar_init(&p_full, 128);
-    mbar_init(&pv_done, 1);
-    mbar_init(&drain_bar, 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&s_full[g], 1);
+      mbar_init(&s_free[g], 128);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&p_full[g][b], 128);
+        mbar_init(&pv_done[g][b], 1);
+      }
+      mbar_init(&drain_bar[g], 1);
+    }
     abort_sh = 0;
     mbar_fence_init();
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_sh, 256);
+    tmem_alloc(&tmem_sh, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tS = tmem_sh;         // S: columns 0..127
-  const uint32_t tO = tmem_sh + 128;   // O: columns 128..191
+  const uint32_t tmem = tmem_sh;  // S_g: columns 128g..128g+127; O_g: 256+64g..256+64g+63
 
   WaitCtl w;
   w.abort = reinterpret_cast<volatile int*>(&abort_sh);
@@ -115,199 +139,242 @@ __global__ void __launch_bounds__(192, 2)
     if (lane == 0) {
       bool ok = true;
       uint32_t karmed = 0, kpar = 0, varmed = 0, vpar = 0;
-      mbar_expect_tx(&q_full, kQBytes);
-      tma_load_3d(sQ, &tmQ, &q_full, 0, q0, bh);
-      for (int j = 0; j < n_kv; ++j) {
-        const int ks = j & 1;
-        const uint32_t kph = (j >> 1) & 1;
-        if (!mbar_wait(&k_empty[ks], kph ^ 1, w)) {
+      mbar_expect_tx(&q_full, nkv1 > 0 ? 2 * kTile : kTile);
+      tma_load_3d(sm + kOffQ, &tmQ, &q_full, 0, q00, bh);
+      if (nkv1 > 0) tma_load_3d(sm + kOffQ + kTile, &tmQ, &q_full, 0, q01, bh);
+      for (int j = 0; j < nkv_all; ++j) {
+        const int s = j % kStages;
+        const uint32_t ph = (j / kStages) & 1;
+        if (!mbar_wait(&k_empty[s], ph ^ 1, w)) {
           ok = false;
           break;
         }
-        mbar_expect_tx(&k_full[ks], kKBytes);
-        tma_load_3d(sK0 + ks * kKBytes, &tmK, &k_full[ks], 0, j * 128, bh);
-        karmed |= 1u << ks;
-        kpar = (kpar & ~(1u << ks)) | (kph << ks);
-        if (!mbar_wait(&v_empty, (j & 1) ^ 1, w)) {
+        mbar_expect_tx(&k_full[s], kTile);
+        tma_load_3d(sm + kOffK + s * kTile, &tmK, &k_full[s], 0, j * 128, bh);
+        karmed |= 1u << s;
+        kpar = (kpar & ~(1u << s)) | (ph << s);
+        if (!mbar_wait(&v_empty[s], ph ^ 1, w)) {
           ok = false;
           break;
         }
-        mbar_expect_tx(&v_full, kVBytes);
-        tma_load_3d(sV, &tmV, &v_full, j * 128, 0, bh);
-        tma_load_3d(sV + kVBytes / 2, &tmV, &v_full, j * 128 + 64, 0, bh);
-        varmed = 1;
-        vpar = j & 1;
+        mbar_expect_tx(&v_full[s], kTile);
+        tma_load_3d(sm + kOffV + s * kTile, &tmV, &v_full[s], j * 128, 0, bh);
+        tma_load_3d(sm + kOffV + s * kTile + kTile / 2, &tmV, &v_full[s], j * 128 + 64, 0, bh);
+        varmed |= 1u << s;
+        vpar = (vpar & ~(1u << s)) | (ph << s);
       }
-      if (!ok) {
+      if (!ok) {  // let the copies already issued land before the CTA exits
         mbar_wait_drain(&q_full, 0);
-        for (int s = 0; s < 2; ++s)
+        for (int s = 0; s < kStages; ++s) {
           if ((karmed >> s) & 1u) mbar_wait_drain(&k_full[s], (kpar >> s) & 1u);
-        if (varmed) mbar_wait_drain(&v_full, vpar);
+          if ((varmed >> s) & 1u) mbar_wait_drain(&v_full[s], (vpar >> s) & 1u);
+        }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 10) {
+    // one MMA issuer per query tile, so each tile's S / PV products follow
+    // its own softmax without waiting on the other tile's
     if (lane == 0) {
+      const int g = warp == 1 ? 0 : 1;
+      const int nkv_g = g == 0 ? nkv0 : nkv1;
       constexpr uint32_t idesc_s = idesc_f16_f32(128, 128);
       constexpr uint32_t idesc_o = idesc_f16_f32(128, 64);
-      const uint64_t qd = sdesc_kmajor_sw128(smem_u32(sQ));
-      const uint64_t pd0 = sdesc_kmajor_sw128(smem_u32(sP));
-      const uint64_t pd1 = sdesc_kmajor_sw128(smem_u32(sP + kPBytes / 2));
-      const uint64_t vd0 = sdesc_kmajor_sw128(smem_u32(sV));
-      const uint64_t vd1 = sdesc_kmajor_sw128(smem_u32(sV + kVBytes / 2));
+      const uint64_t qd = sdesc_kmajor_sw128(smem_u32(sm + kOffQ + g * kTile));
       bool ok = mbar_wait(&q_full, 0, w);
-      // O += P_j V_j (j = tile index), after softmax published P_j
-      auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(&p_full, j & 1, w)) return false;
-        if (!mbar_wait(&v_full, j & 1, w)) return false;
-        tc_fence_after();
+      // Every issuer waits for each K / V tile to land and then arrives on
+      // its release barrier (count 2), also for tiles it does not use: a
+      // stage is only refilled once both issuers are done with it.
+      for (int j = 0; ok && j <= nkv_all; ++j) {
+        const int ks = j % kStages;
+        if (j < nkv_all) {
+          if (!mbar_wait(&k_full[ks], (j / kStages) & 1, w)) {
+            ok = false;
+            break;
+          }
+          if (j < nkv_g) {  // S_g = Q_g K_j^T once softmax g has taken S_g of tile j-1
+            if (j > 0 && !mbar_wait(&s_free[g], (j - 1) & 1, w)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t kd = sdesc_kmajor_sw128(smem_u32(sm + kOffK + ks * kTile));
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint64_t ad = (k < 4 ? pd0 : pd1) + static_cast<uint64_t>(2 * (k & 3));
-          const uint64_t bd = (k < 4 ? vd0 : vd1) + static_cast<uint64_t>(2 * (k & 3));
-          tc_mma_f16_ss(tO, ad, bd, idesc_o, (j > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < 4; ++k)
+              tc_mma_f16_ss(tmem + 128 * g, qd + static_cast<uint64_t>(2 * k), kd + static_cast<uint64_t>(2 * k),
+                            idesc_s, k > 0 ? 1u : 0u);
+            tc_commit(&s_full[g]);
+          }
+          tc_commit(&k_empty[ks]);
         }
-        tc_commit(&v_empty);
-        tc_commit(&pv_done);
-        return true;
-      };
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int ks = j & 1;
-        if (!mbar_wait(&k_full[ks], (j >> 1) & 1, w)) {
-          ok = false;
-          break;
-        }
-        // S is free once softmax published P_{j-1} (it has read S_{j-1})
-        if (j > 0 && !mbar_wait(&p_full, (j - 1) & 1, w)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint64_t kd = sdesc_kmajor_sw128(smem_u32(sK0 + ks * kKBytes));
+        if (j >= 1) {
+          const int vs = (j - 1) % kStages;
+          if (!mbar_wait(&v_full[vs], ((j - 1) / kStages) & 1, w)) {
+            ok = false;
+            break;
+          }
+          if (j <= nkv_g) {  // O_g += P_g V_{j-1} once softmax g published P_g of tile j-1
+            const int pbuf = (j - 1) & 1;
+            if (!mbar_wait(&p_full[g][pbuf], ((j - 1) >> 1) & 1, w)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t pb = smem_u32(sm + kOffP + (g * 2 + pbuf) * 2 * kTile);
+            const uint32_t vb = smem_u32(sm + kOffV + vs * kTile);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          tc_mma_f16_ss(tS, qd + static_cast<uint64_t>(2 * k), kd + static_cast<uint64_t>(2 * k), idesc_s,
-                        k > 0 ? 1u : 0u);
-        tc_commit(&k_empty[ks]);
-        tc_commit(&s_full);
-        if (j > 0 && !issue_pv(j - 1)) {
-          ok = false;
-          break;
+            for (int k = 0; k < 8; ++k) {
+              const uint64_t ad = sdesc_kmajor_sw128(pb + (k >> 2) * kTile) + static_cast<uint64_t>(2 * (k & 3));
+              const uint64_t bd = sdesc_kmajor_sw128(vb + (k >> 2) * (kTile / 2)) + static_cast<uint64_t>(2 * (k & 3));
+              tc_mma_f16_ss(tmem + 256 + 64 * g, ad, bd, idesc_o, (j > 1 || k > 0) ? 1u : 0u);
+            }
+            tc_commit(&pv_done[g][pbuf]);
+          }
+          tc_commit(&v_empty[vs]);
         }
       }
-      if (ok) issue_pv(n_kv - 1);
-      tc_commit(&drain_bar);
-      mbar_wait_drain(&drain_bar, 0);
+      tc_commit(&drain_bar[g]);
+      mbar_wait_drain(&drain_bar[g], 0);
     }
-  } else {
-    // softmax: one thread per query row
+  } else if (warp < 10) {
+    // softmax: warps 2-5 take query tile 0, warps 6-9 query tile 1
+    const int g = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const int i = q0 + r;
+    const int i = (g == 0 ? q00 : q01) + r;
+    const int n_my = g == 0 ? nkv0 : nkv1;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tS = tmem + 128 * g + lane_off;
+    const uint32_t tO = tmem + 256 + 64 * g + lane_off;
+    const uint32_t pbase0 = smem_u32(sm + kOffP + g * 2 * 2 * kTile);
     int lo, hi;
     key_range(p, i, lo, hi);
-    if (i >= p.N) {
+    if (i >= p.N || (cls_cta && i == 0)) {
       lo = 0;
       hi = p.N - 1;
     }
-    const float sc = p.scale_log2;
+    // rows this CTA writes: the CLS CTA only row 0; pair CTAs every valid row
+    // but a separately computed CLS row
+    const bool store_row = cls_cta ? (i == 0) : (i < p.N && !(i == 0 && p.cls_separate));
+    const float c = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.0f;
-    const uint32_t pbase = smem_u32(sP);
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      bool okw = mbar_wait(&s_full, j & 1, w);
+    for (int j = 0; j < n_my; ++j) {
+      bool okw = mbar_wait(&s_full[g], j & 1, w);
       okw = __all_sync(0xffffffffu, okw);
       if (!okw) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int kbase = j * 128;
-      // pass 1: masked row max of the scaled scores (log2 domain)
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t s[32];
-        tmem_ld32(tS + lane_off + static_cast<uint32_t>(c * 32), s);
+      float s[128];
+      {
+        uint32_t u[128];
+        tmem_ld128(tS, u);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int key = kbase + c * 32 + e;
-          const float v = __uint_as_float(s[e]) * sc;
-          if (key >= lo && key <= hi) mx = fmaxf(mx, v);
-        }
+        for (int e = 0; e < 128; ++e) s[e] = __uint_as_float(u[e]);
       }
-      const float m_new = fmaxf(m_run, mx);
-      if (j > 0) {  // P buffer free and O stable once PV_{j-1} is done
-        okw = mbar_wait(&pv_done, (j - 1) & 1, w);
+      tc_fence_before();
+      mbar_arrive(&s_free[g]);  // S_g may now be overwritten by the next KV tile
+      const int kbase = j * 128;
+      const bool full = lo <= kbase && hi >= kbase + 127;
+      if (!__all_sync(0xffffffffu, full)) {
+        const int rlo = lo - kbase, rhi = hi - kbase;
+#pragma unroll
+        for (int e = 0; e < 128; ++e) s[e] = (e >= rlo && e <= rhi) ? s[e] : -INFINITY;
+      }
+      // row max as 8 independent chains (short dependency chains: two
+      // softmax warps per scheduler must hide the latency)
+      float mxv[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) mxv[t] = s[t];
+#pragma unroll
+      for (int e = 8; e < 128; ++e) mxv[e & 7] = fmaxf(mxv[e & 7], s[e]);
+      const float mx = fmaxf(fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])),
+                             fmaxf(fmaxf(mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7])));
+      const float m_new = fmaxf(m_run, mx * c);
+      const int pbuf = j & 1;
+      if (j > 1) {  // P buffer pbuf is free once the PV product of tile j-2 is done
+        okw = mbar_wait(&pv_done[g][pbuf], ((j - 2) >> 1) & 1, w);
         okw = __all_sync(0xffffffffu, okw);
         if (!okw) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        // tcgen05.ld / st are warp-collective: the whole warp rescales its
-        // rows when any of them saw a larger max (the others scale by 1).
-        const bool grow = m_new > m_run && m_run != -INFINITY;
-        if (__any_sync(0xffffffffu, grow)) {
-          const float alpha = grow ? ex2_approx(m_run - m_new) : 1.0f;
-          l_run *= alpha;
-#pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + lane_off + static_cast<uint32_t>(c * 32), o);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + lane_off + static_cast<uint32_t>(c * 32), o);
-          }
+      }
+      const bool grow = m_new > m_run + kRescaleLog2;
+      // tcgen05.ld / st are warp-collective: the warp rescales together,
+      // after every PV product so far (the one of tile j-1 last) is done
+      const bool rescale = j > 0 && __any_sync(0xffffffffu, grow);
+      if (rescale) {
+        okw = mbar_wait(&pv_done[g][pbuf ^ 1], ((j - 1) >> 1) & 1, w);
+        okw = __all_sync(0xffffffffu, okw);
+        if (!okw) {
+          ok = false;
+          break;
         }
       }
-      // a row may still see no allowed key (m = -inf): then every p is 0
-      m_run = m_new;
+      tc_fence_after();
+      if (rescale) {
+        const float alpha = grow ? ex2_approx(m_run - m_new) : 1.0f;
+        l_run *= alpha;
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t o[16];
+          tmem_ld16(tO + static_cast<uint32_t>(q * 16), o);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st16(tO + static_cast<uint32_t>(q * 16), o);
+        }
+      }
+      if (grow) m_run = m_new;
+      // a row that has seen no allowed key yet keeps m = -inf: all its p are 0
       const float m_use = m_run == -INFINITY ? 0.0f : m_run;
-      // pass 2: P = exp2(s - m), row sum, f16 into the swizzled P tile
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t s[32];
-        tmem_ld32(tS + lane_off + static_cast<uint32_t>(c * 32), s);
-        uint32_t h[16];
+      float lsv[8];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int key = kbase + c * 32 + e;
-          float pa = 0.0f, pb = 0.0f;
-          if (key >= lo && key <= hi) pa = ex2_approx(__uint_as_float(s[e]) * sc - m_use);
-          if (key + 1 >= lo && key + 1 <= hi) pb = ex2_approx(__uint_as_float(s[e + 1]) * sc - m_use);
-          l_run += pa + pb;
-          h[e >> 1] = pack_half2(pa, pb);
-        }
-        const uint32_t half_base = pbase + static_cast<uint32_t>((c >> 1) * (kPBytes / 2));
+      for (int t = 0; t < 8; ++t) lsv[t] = 0.0f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int kk = (c & 1) * 32 + u * 8;
-          st_shared_v4(half_base + sw128_offset(r, kk), h[4 * u], h[4 * u + 1], h[4 * u + 2], h[4 * u + 3]);
+      for (int h = 0; h < 2; ++h) {  // two [128 x 64] halves of the P tile
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int k = h * 64 + u * 8 + 2 * e;
+            const float pa = ex2_approx(fmaf(s[k], c, -m_use));
+            const float pb = ex2_approx(fmaf(s[k + 1], c, -m_use));
+            lsv[(2 * e) & 7] += pa;
+            lsv[(2 * e + 1) & 7] += pb;
+            pk[e] = pack_half2(pa, pb);
+          }
+          st_shared_v4(pbase0 + static_cast<uint32_t>((pbuf * 2 + h) * kTile) + sw128_offset(r, u * 8), pk[0], pk[1],
+                       pk[2], pk[3]);
         }
       }
+      l_run += ((lsv[0] + lsv[1]) + (lsv[2] + lsv[3])) + ((lsv[4] + lsv[5]) + (lsv[6] + lsv[7]));
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full);
+      mbar_arrive(&p_full[g][pbuf]);
     }
-    if (ok) {
-      bool okw = mbar_wait(&pv_done, (n_kv - 1) & 1, w);
+    if (ok && n_my > 0) {  // the last PV product completes after all earlier ones
+      bool okw = mbar_wait(&pv_done[g][(n_my - 1) & 1], ((n_my - 1) >> 1) & 1, w);
       okw = __all_sync(0xffffffffu, okw);
       if (okw) {
         tc_fence_after();
         const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
         const int b = bh / p.heads, hd = bh % p.heads;
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        for (int q = 0; q < 2; ++q) {
           uint32_t o[32];
-          tmem_ld32(tO + lane_off + static_cast<uint32_t>(c * 32), o);
-          if (i < p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(b) * p.N + i) * p.ldo + hd * 64 + c * 32);
+          tmem_ld32(tO + static_cast<uint32_t>(q * 32), o);
+          if (store_row) {
+            uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(b) * p.N + i) * p.ldo + hd * 64 + q * 32);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              const float* f = reinterpret_cast<const float*>(o) + 8 * u;
-              dst[u] = make_uint4(pack_half2(f[0] * inv_l, f[1] * inv_l), pack_half2(f[2] * inv_l, f[3] * inv_l),
-                                  pack_half2(f[4] * inv_l, f[5] * inv_l), pack_half2(f[6] * inv_l, f[7] * inv_l));
+              uint32_t h[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                h[e] = pack_half2(__uint_as_float(o[8 * u + 2 * e]) * inv_l, __uint_as_float(o[8 * u + 2 * e + 1]) * inv_l);
+              dst[u] = make_uint4(h[0], h[1], h[2], h[3]);
             }
           }
         }
@@ -318,7 +385,7 @@ __global__ void __launch_bounds__(192, 2)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_sh, 256);
+    tmem_dealloc(tmem_sh, 512);
   }
 }
 
@@ -355,6 +422,11 @@ int attn_prepare(AttnOp* op, const __half* q, const __half* k, const __half* vt,
   p.scale_log2 = 1.4426950408889634f / 8.0f;
   p.out = out;
   p.ldo = heads * 64;
+  p.cls_separate = (mask == JEPA_B200_MASK_BLOCK_CAUSAL && has_cls) ? 1 : 0;
+  op->q = q;
+  op->k = k;
+  op->vt = vt;
+  op->npad = npad;
   op->B = B;
   op->smem = kAttnSmem;
   return JEPA_B200_OK;
@@ -373,8 +445,8 @@ int attn_launch(const AttnOp& op, cudaStream_t st, DevErr* err, unsigned long lo
   AttnParams p = op.p;
   p.err = err;
   p.timeout_ns = timeout_ns;
-  dim3 grid(p.n_q_tiles, op.B * p.heads);
-  attn_fwd_kernel<<<grid, 192, kAttnSmem, st>>>(op.tmQ, op.tmK, op.tmV, p);
+  dim3 grid((p.n_q_tiles + 1) / 2 + p.cls_separate, op.B * p.heads);
+  attn_fwd_kernel<<<grid, 352, kAttnSmem, st>>>(op.tmQ, op.tmK, op.tmV, p);
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 

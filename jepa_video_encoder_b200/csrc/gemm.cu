@@ -36,9 +36,9 @@ struct GemmCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = BN == 256 ? 4 : (BN == 192 ? 5 : 6);
+  static constexpr int STAGES = BN == 256 ? 4 : (BN == 192 ? 4 : 6);
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 8 * 4096 + 1024;  // + epilogue staging
 };
 
 __device__ __forceinline__ float gelu_erf(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
@@ -183,6 +183,9 @@ __device__ __forceinline__ void fill_a_patch(uint8_t* sA, const GemmParams& p, i
   const int ppf = (s.H / s.patch) * wp;
   const int pp = s.patch * s.patch;
   const int ktpp = s.tubelet * pp;
+  // patch rows of 8-multiple width on 16-byte aligned image rows and planes
+  const bool vec8 = (s.patch % 8 == 0) && (s.W % 4 == 0) && ((s.H * s.W) % 4 == 0) &&
+                    ((reinterpret_cast<uintptr_t>(s.pixels) & 15) == 0);
   const uint32_t sbase = smem_u32(sA);
   for (int idx = ct; idx < 128 * 8; idx += 128) {
     const int r = idx >> 3, u = idx & 7;
@@ -190,7 +193,24 @@ __device__ __forceinline__ void fill_a_patch(uint8_t* sA, const GemmParams& p, i
     float f[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) f[e] = 0.0f;
-    if (m < p.M) {
+    if (m < p.M && vec8) {
+      // 8 consecutive k = 8 consecutive pixels of one image row: two 16-byte loads
+      const int b = m / s.n_patches, i = m % s.n_patches;
+      const int tp = i / ppf, rem = i % ppf;
+      const int hp = rem / wp, wq = rem % wp;
+      const int k = kb * 64 + u * 8;
+      if (k < s.k_real) {
+        const int c = k / ktpp, rk = k % ktpp;
+        const int dt = rk / pp, rk2 = rk % pp;
+        const int kh = rk2 / s.patch, kw = rk2 % s.patch;
+        const size_t plane = (static_cast<size_t>(b) * s.T + tp * s.tubelet + dt) * 3 + c;
+        const float4* src =
+            reinterpret_cast<const float4*>(s.pixels + (plane * s.H + hp * s.patch + kh) * s.W + wq * s.patch + kw);
+        const float4 a = __ldg(src), bb = __ldg(src + 1);
+        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+        f[4] = bb.x; f[5] = bb.y; f[6] = bb.z; f[7] = bb.w;
+      }
+    } else if (m < p.M) {
       const int b = m / s.n_patches, i = m % s.n_patches;
       const int tp = i / ppf, rem = i % ppf;
       const int hp = rem / wp, wq = rem % wp;
@@ -211,10 +231,153 @@ __device__ __forceinline__ void fill_a_patch(uint8_t* sA, const GemmParams& p, i
   }
 }
 
+// Epilogue of one output tile for one thread: its row, half of the BN
+// columns (chalf), read from TMEM at tb (lane quadrant already applied).
+template <int BN>
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tb, int row, int nb, int chalf) {
+  if (p.epi == EPI_RESID_F32) {
+    // residual add: the residual's loads are issued before the TMEM load
+    // so the two latencies overlap
+#pragma unroll 1
+    for (int c = chalf * (BN / 64); c < (chalf + 1) * (BN / 64); ++c) {
+      const int col0 = nb * BN + c * 32;
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + static_cast<size_t>(row) * p.ldo + col0);
+      float4 x[8];
+      if (row < p.M) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) x[j] = dst[j];
+      }
+      uint32_t r[32];
+      tmem_ld32(tb + static_cast<uint32_t>(c * 32), r);
+      if (row < p.M) {
+        const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 b = p.bias ? __ldg(b4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+          x[j].x += __uint_as_float(r[4 * j]) + b.x;
+          x[j].y += __uint_as_float(r[4 * j + 1]) + b.y;
+          x[j].z += __uint_as_float(r[4 * j + 2]) + b.z;
+          x[j].w += __uint_as_float(r[4 * j + 3]) + b.w;
+          dst[j] = x[j];
+        }
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int c = chalf * (BN / 64); c < (chalf + 1) * (BN / 64); ++c) {
+      uint32_t r[32];
+      tmem_ld32(tb + static_cast<uint32_t>(c * 32), r);
+      if (row < p.M) epilogue_chunk(p, row, nb * BN + c * 32, r);
+    }
+  }
+}
+
+// TMA epilogue of one output tile for one warp: 32 rows starting at row0,
+// half of the BN columns (chalf).  Each 32-row x 128-byte chunk (32 f32
+// columns, or 64 f16 columns) is written to the warp's staging buffer in the
+// 128-byte-swizzled layout and sent with one TMA store (f16 / f32 outputs)
+// or one TMA reduce-add (f32 residual: X += A W^T + b), so every global
+// write is a full, coalesced line.
+template <int BN>
+__device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUtensorMap* tmC, uint32_t tb,
+                                                  int row0, int nb, int chalf, uint8_t* stage_buf, int lane,
+                                                  bool& pending) {
+  const uint32_t sb = smem_u32(stage_buf);
+  const uint32_t row_off = static_cast<uint32_t>(lane) * 128u;
+  const bool live = row0 < p.M;
+  const int c_begin = chalf * (BN / 64), c_end = (chalf + 1) * (BN / 64);
+  if (p.epi == EPI_F32 || p.epi == EPI_RESID_F32) {
+#pragma unroll 1
+    for (int c = c_begin; c < c_end; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tb + static_cast<uint32_t>(c * 32), r);
+      const int col0 = nb * BN + c * 32;
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+      if (p.bias) {
+        const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 b = __ldg(b4 + j);
+          v[4 * j] += b.x;
+          v[4 * j + 1] += b.y;
+          v[4 * j + 2] += b.z;
+          v[4 * j + 3] += b.w;
+        }
+      }
+      if (pending) {  // the previous chunk's store must have read the buffer
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        st_shared_v4(sb + row_off + static_cast<uint32_t>(((u ^ (lane & 7)) & 7) << 4), __float_as_uint(v[4 * u]),
+                     __float_as_uint(v[4 * u + 1]), __float_as_uint(v[4 * u + 2]), __float_as_uint(v[4 * u + 3]));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && live) {
+        if (p.epi == EPI_RESID_F32)
+          tma_reduce_add_2d(tmC, stage_buf, col0, row0);
+        else
+          tma_store_2d(tmC, stage_buf, col0, row0);
+        bulk_commit();
+      }
+      pending = true;
+    }
+  } else {  // f16 output: two 32-column TMEM chunks per 128-byte staging row
+#pragma unroll 1
+    for (int c = c_begin; c < c_end; c += 2) {
+      uint32_t w[32];
+      const int col0 = nb * BN + c * 32;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t r[32];
+        tmem_ld32(tb + static_cast<uint32_t>((c + h) * 32), r);
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        if (p.bias) {
+          const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0 + h * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 b = __ldg(b4 + j);
+            v[4 * j] += b.x;
+            v[4 * j + 1] += b.y;
+            v[4 * j + 2] += b.z;
+            v[4 * j + 3] += b.w;
+          }
+        }
+        if (p.epi == EPI_GELU_F16) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) w[h * 16 + j] = pack_half2(v[2 * j], v[2 * j + 1]);
+      }
+      if (pending) {
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        st_shared_v4(sb + row_off + static_cast<uint32_t>(((u ^ (lane & 7)) & 7) << 4), w[4 * u], w[4 * u + 1],
+                     w[4 * u + 2], w[4 * u + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && live) {
+        tma_store_2d(tmC, stage_buf, col0, row0);
+        bulk_commit();
+      }
+      pending = true;
+    }
+  }
+}
+
 template <int BN, int BMODE, bool GATHER>
 __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
   using C = GemmCfg<BN>;
   constexpr bool CONV = (BMODE != B_F16) || GATHER;
   constexpr int S = C::STAGES;
@@ -268,7 +431,7 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
       uint32_t phase = 0, armed = 0, armed_par = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const int mb = t % p.m_tiles, nb = t / p.m_tiles;
+        const int nb = t % p.n_tiles, mb = t / p.n_tiles;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, w)) {
             ok = false;
@@ -345,6 +508,8 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
     // (w % 4) and split the tile's columns in two halves.
     const int quad = warp & 3;
     const int chalf = (warp - 2) >> 2;
+    uint8_t* stage_buf = smem + S * C::STAGE_BYTES + (warp - 2) * 4096;
+    bool pending = false;
     int acc = 0;
     uint32_t aphase = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
@@ -352,15 +517,13 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int mb = t % p.m_tiles, nb = t / p.m_tiles;
+      const int nb = t % p.n_tiles, mb = t / p.n_tiles;
       const int row = mb * 128 + quad * 32 + lane;
       const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
-#pragma unroll 1
-      for (int c = chalf * (BN / 64); c < (chalf + 1) * (BN / 64); ++c) {
-        uint32_t r[32];
-        tmem_ld32(tb + static_cast<uint32_t>(c * 32), r);
-        if (row < p.M) epilogue_chunk(p, row, nb * BN + c * 32, r);
-      }
+      if (p.tma_epi)
+        epilogue_tile_tma<BN>(p, &tmC, tb, mb * 128 + quad * 32, nb, chalf, stage_buf, lane, pending);
+      else
+        epilogue_tile<BN>(p, tb, row, nb, chalf);
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
       if (++acc == 2) {
@@ -368,13 +531,14 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
         aphase ^= 1;
       }
     }
+    if (pending && lane == 0) bulk_wait0();
   } else if (CONV) {
     const int ct = threadIdx.x - 320;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      const int mb = t % p.m_tiles, nb = t / p.m_tiles;
+      const int nb = t % p.n_tiles, mb = t / p.n_tiles;
       for (int kb = 0; kb < kblocks; ++kb) {
         bool okw = mbar_wait(&empty_bar[stage], phase ^ 1, w);
         okw = __all_sync(0xffffffffu, okw);
@@ -405,6 +569,192 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// CTA-pair variant (f16 weights): a cluster of two CTAs on two SMs computes a
+// 256 x BN tile with tcgen05.mma.cta_group::2 (M = 256).  Each CTA loads the
+// 128 A rows of its half and half of the B tile (BN/2 rows), so per SM a
+// stage is 16 KB + BN*64 bytes instead of 16 KB + BN*128: the same MMA work
+// per SM with two thirds of the shared-memory traffic and more stages in
+// flight.  The leader CTA (rank 0) issues the MMAs; its commits arrive on the
+// barriers of both CTAs (multicast commit).  TMA loads are plain (no
+// multicast): each CTA loads its own tiles, the bytes counted on the
+// leader's barrier.
+template <int BN>
+struct Gemm2Cfg {
+  static constexpr int A_BYTES = 128 * 64 * 2;
+  static constexpr int B_BYTES = (BN / 2) * 64 * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = BN == 256 ? 6 : (BN == 192 ? 6 : 8);
+  static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 8 * 4096 + 1024;  // + epilogue staging
+};
+
+template <int BN>
+__global__ void __launch_bounds__(320, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+  using C = Gemm2Cfg<BN>;
+  constexpr int S = C::STAGES;
+  extern __shared__ uint8_t dsmem[];
+  __shared__ uint64_t full_bar[S], empty_bar[S], tfull_bar[2], tempty_bar[2], drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  const uint32_t raw = smem_u32(dsmem);
+  uint8_t* smem = dsmem + ((1024u - (raw & 1023u)) & 1023u);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: leader (issues the MMAs), 1: peer
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_bar[s], 1);     // leader: one expect-tx arrival + the bytes of both CTAs
+      mbar_init(&empty_bar[s], 1);    // both: the leader's multicast commit
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);    // both: the leader's multicast commit
+      mbar_init(&tempty_bar[a], 16);  // leader: one arrival per epilogue warp of both CTAs
+    }
+    mbar_init(&drain_bar, 1);
+    abort_sh = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&tmem_base_sh, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_sh;
+
+  WaitCtl w;
+  w.abort = reinterpret_cast<volatile int*>(&abort_sh);
+  w.err = p.err;
+  w.timeout_ns = p.timeout_ns;
+  w.where = (KID_GEMM << 8) | 0x80u | static_cast<unsigned>(warp);
+  const int num_tiles = ((p.M + 255) / 256) * p.n_tiles;
+  const int n_clusters = gridDim.x >> 1;
+  const int cid = blockIdx.x >> 1;
+  const int kblocks = p.K / 64;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t leader_full0 = mapa_shared(smem_u32(&full_bar[0]), 0);
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_par = 0;
+      bool ok = true;
+      for (int t = cid; t < num_tiles && ok; t += n_clusters) {
+        const int nb = t % p.n_tiles, mb = t / p.n_tiles;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, w)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sA = smem + stage * C::STAGE_BYTES;
+          uint8_t* sB = sA + C::A_BYTES;
+          if (rank == 0) mbar_expect_tx(&full_bar[stage], 2u * C::STAGE_BYTES);
+          const uint32_t fb = leader_full0 + static_cast<uint32_t>(stage * sizeof(uint64_t));
+          tma_load_2d_pair(sA, &tmA, fb, kb * 64, mb * 256 + static_cast<int>(rank) * 128);
+          tma_load_2d_pair(sB, &tmB, fb, kb * 64, nb * BN + static_cast<int>(rank) * (BN / 2));
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok && rank == 0) {  // let the copies already counted on the leader's barriers land
+        for (int s = 0; s < S; ++s)
+          if ((armed >> s) & 1u) mbar_wait_drain(&full_bar[s], (armed_par >> s) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(256, BN);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, aphase = 0;
+      bool ok = true;
+      for (int t = cid; t < num_tiles && ok; t += n_clusters) {
+        if (!mbar_wait(&tempty_bar[acc], aphase ^ 1, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dtm = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, w)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint64_t ad = sdesc_kmajor_sw128(a0);
+          const uint64_t bd = sdesc_kmajor_sw128(a0 + C::A_BYTES);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma_f16_ss_pair(dtm, ad + static_cast<uint64_t>(2 * k), bd + static_cast<uint64_t>(2 * k), idesc,
+                               (kb | k) != 0 ? 1u : 0u);
+          tc_commit_pair_mc(&empty_bar[stage], 0x3);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(&tfull_bar[acc], 0x3);
+        if (++acc == 2) {
+          acc = 0;
+          aphase ^= 1;
+        }
+      }
+      tc_commit_pair_mc(&drain_bar, 0x1);
+      mbar_wait_drain(&drain_bar, 0);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int chalf = (warp - 2) >> 2;
+    const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
+    uint8_t* stage_buf = smem + S * C::STAGE_BYTES + (warp - 2) * 4096;
+    bool pending = false;
+    int acc = 0;
+    uint32_t aphase = 0;
+    for (int t = cid; t < num_tiles; t += n_clusters) {
+      bool ok = mbar_wait(&tfull_bar[acc], aphase, w);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int nb = t % p.n_tiles, mb = t / p.n_tiles;
+      const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quad * 32;
+      const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
+      if (p.tma_epi)
+        epilogue_tile_tma<BN>(p, &tmC, tb, row0, nb, chalf, stage_buf, lane, pending);
+      else
+        epilogue_tile<BN>(p, tb, row0 + lane, nb, chalf);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_tempty0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+      if (++acc == 2) {
+        acc = 0;
+        aphase ^= 1;
+      }
+    }
+    if (pending && lane == 0) bulk_wait0();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while the pair's MMAs or arrivals may touch it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ host --
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -432,6 +782,18 @@ bool make_tmap_f16(CUtensorMap* m, const void* base, int rank, const uint64_t* d
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank, const_cast<void*>(base), d, s, b, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_2d(CUtensorMap* m, const void* base, int esize, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+                  uint32_t box_cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn || (esize != 2 && esize != 4)) return false;
+  cuuint64_t d[2] = {cols, rows}, st[1] = {row_bytes};
+  cuuint32_t b[2] = {box_cols, box_rows}, es[2] = {1, 1};
+  CUresult r = fn(m, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                  const_cast<void*>(base), d, st, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -481,14 +843,35 @@ int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& W, 
     const uint32_t box[2] = {64, 128};
     if (!make_tmap_f16(&op->tmA, A, 2, dims, str, box)) return JEPA_B200_ERR_CUDA;
   }
+  // TMA epilogue: f32 outputs and residual adds in 32-column chunks, f16
+  // outputs in 64-column chunks (two per warp-half of the tile)
+  if (epi == EPI_F32 || epi == EPI_RESID_F32) {
+    if (!make_tmap_2d(&op->tmC, out, 4, static_cast<uint64_t>(ldo), static_cast<uint64_t>(M),
+                      static_cast<uint64_t>(ldo) * 4, 32, 32))
+      return JEPA_B200_ERR_CUDA;
+    p.tma_epi = 1;
+  } else if ((epi == EPI_F16 || epi == EPI_GELU_F16) && (bn / 64) % 2 == 0) {
+    if (!make_tmap_2d(&op->tmC, out, 2, static_cast<uint64_t>(ldo), static_cast<uint64_t>(M),
+                      static_cast<uint64_t>(ldo) * 2, 64, 32))
+      return JEPA_B200_ERR_CUDA;
+    p.tma_epi = 1;
+  }
+  // f16 weights and at least two 128-row blocks: the CTA-pair kernel
+  op->pair = (W.bmode == B_F16 && !patch && M >= 256) ? 1 : 0;
   if (W.bmode == B_F16) {
     const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
     const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
-    const uint32_t box[2] = {64, static_cast<uint32_t>(bn)};
+    const uint32_t box[2] = {64, static_cast<uint32_t>(op->pair ? bn / 2 : bn)};
     if (!make_tmap_f16(&op->tmB, W.data, 2, dims, str, box)) return JEPA_B200_ERR_CUDA;
   }
-  op->grid = std::min(p.m_tiles * p.n_tiles, num_sms());
-  op->smem = bn == 256 ? GemmCfg<256>::SMEM : (bn == 192 ? GemmCfg<192>::SMEM : GemmCfg<128>::SMEM);
+  if (op->pair) {
+    const int cluster_tiles = ((M + 255) / 256) * p.n_tiles;
+    op->grid = 2 * std::min(cluster_tiles, num_sms() / 2);
+    op->smem = bn == 256 ? Gemm2Cfg<256>::SMEM : (bn == 192 ? Gemm2Cfg<192>::SMEM : Gemm2Cfg<128>::SMEM);
+  } else {
+    op->grid = std::min(p.m_tiles * p.n_tiles, num_sms());
+    op->smem = bn == 256 ? GemmCfg<256>::SMEM : (bn == 192 ? GemmCfg<192>::SMEM : GemmCfg<128>::SMEM);
+  }
   return JEPA_B200_OK;
 }
 
@@ -504,7 +887,34 @@ static int launch_impl(const GemmOp& op, cudaStream_t st) {
     attr_done |= 1ull << dev;
   }
   constexpr int threads = (BMODE != B_F16 || GATHER) ? 448 : 320;
-  kern<<<op.grid, threads, GemmCfg<BN>::SMEM, st>>>(op.tmA, op.tmB, op.p);
+  kern<<<op.grid, threads, GemmCfg<BN>::SMEM, st>>>(op.tmA, op.tmB, op.tmC, op.p);
+  return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+}
+
+template <int BN>
+static int launch_pair(const GemmOp& op, cudaStream_t st) {
+  auto kern = gemm_pair_kernel<BN>;
+  static unsigned long long attr_done = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !((attr_done >> dev) & 1ull)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Gemm2Cfg<BN>::SMEM) != cudaSuccess)
+      return JEPA_B200_ERR_CUDA;
+    attr_done |= 1ull << dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(op.grid);
+  cfg.blockDim = dim3(320);
+  cfg.dynamicSmemBytes = Gemm2Cfg<BN>::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, op.tmA, op.tmB, op.tmC, op.p) != cudaSuccess) return JEPA_B200_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 
@@ -512,6 +922,13 @@ int gemm_launch(const GemmOp& op_in, cudaStream_t st, DevErr* err, unsigned long
   GemmOp op = op_in;
   op.p.err = err;
   op.p.timeout_ns = timeout_ns;
+  if (op.pair) {
+    switch (op.bn) {
+      case 256: return launch_pair<256>(op, st);
+      case 192: return launch_pair<192>(op, st);
+      default: return launch_pair<128>(op, st);
+    }
+  }
   if (op.gather) {
     switch (op.bn) {
       case 256: return launch_impl<256, B_F16, true>(op, st);

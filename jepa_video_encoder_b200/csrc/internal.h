@@ -45,6 +45,7 @@ struct PatchSrc {
 
 struct GemmParams {
   int M, N, K;
+  int tma_epi;  // 1: the epilogue stages 32-row chunks in shared memory and writes them with TMA
   int m_tiles, n_tiles;
   const float* bias;
   int epi;
@@ -62,8 +63,10 @@ struct GemmParams {
 struct GemmOp {
   CUtensorMap tmA;
   CUtensorMap tmB;
+  CUtensorMap tmC;  // output map of the TMA epilogue
   GemmParams p;
   int bn = 0, bmode = 0, gather = 0, grid = 0, smem = 0;
+  int pair = 0;  // 1: CTA-pair kernel (tcgen05 cta_group::2, 256-row tiles)
 };
 
 // Build a GEMM op.  A: f16 [M, K] (ignored when patch != nullptr: the patch
@@ -74,6 +77,7 @@ int gemm_launch(const GemmOp& op, cudaStream_t st, DevErr* err, unsigned long lo
 
 struct AttnParams {
   int N, heads, n_q_tiles, mask, has_cls, ppf;
+  int cls_separate;  // block-causal with CLS: row 0 by the one-query kernel
   float scale_log2;
   __half* out;
   int ldo;
@@ -84,6 +88,10 @@ struct AttnParams {
 struct AttnOp {
   CUtensorMap tmQ, tmK, tmV;
   AttnParams p;
+  const __half* q = nullptr;
+  const __half* k = nullptr;
+  const __half* vt = nullptr;
+  int npad = 0;
   int B = 0, smem = 0;
 };
 
@@ -108,6 +116,9 @@ int launch_xattn_1q(const float* q, const __half* k, const __half* vt, int B, in
 // Driver entry point for tensor maps (resolved once through the runtime).
 bool make_tmap_f16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
                    const uint32_t* box);
+// 2-D map with 128-byte swizzle of f16 (esize 2) or f32 (esize 4) elements.
+bool make_tmap_2d(CUtensorMap* m, const void* base, int esize, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+                  uint32_t box_cols, uint32_t box_rows);
 
 int num_sms();
 
