@@ -15,20 +15,19 @@
 //
 // One CTA per (pair of 128-query tiles, clip*head), one CTA per SM:
 //   warp 0      TMA: both Q tiles once, then K and V^T tiles through a
-//               2-stage ring shared by the two query tiles;
-//   warps 1,10  MMA, one issuer per query tile g: for each KV tile j,
-//               S_g = Q_g K_j^T into TMEM (M=128, N=128) and O_g += P_g V_{j-1}
-//               into TMEM (M=128, N=64, P from shared memory); the tensor core
-//               works on one tile while the other tile's softmax runs;
-//   warps 2-5   softmax of query tile 0, warps 6-9 of query tile 1, one
-//               thread per query row: scores read once from TMEM into
-//               registers (S is released at once for the next KV tile), row
-//               max, O rescaled in TMEM only when the max grew by more than
-//               2^8 (lazy rescaling: P stays <= 256, exact after the final
-//               division by the row sum), P = exp2(s*c - m) written as f16
-//               into the swizzled A tile of the PV product; two P buffers per
-//               query tile, so tile j's softmax only waits for the PV product
-//               of tile j-2 (and for tile j-1's when it has to rescale O).
+//               4-stage ring shared by the two query tiles;
+//   warps 1,18  MMA, one issuer per query tile g: for each KV tile j,
+//               S_g = Q_g K_j^T into TMEM (M=128, N=128, both operands in
+//               shared memory) and O_g += P_g V_{j-1} into TMEM (M=128, N=64,
+//               P read from TMEM);
+//   warps 2-9   softmax of query tile 0, warps 10-17 of query tile 1, two
+//               threads per query row, each with 64 of the tile's 128 keys:
+//               scores read once from TMEM into registers (S is released at
+//               once for the next KV tile), row max combined through shared
+//               memory, O rescaled in TMEM only when the max grew by more
+//               than 2^8 (lazy rescaling: P stays <= 256, exact after the
+//               final division by the row sum), P = exp2(s*c - m) packed as
+//               f16 pairs into TMEM for the PV product.
 #include <string.h>
 
 #include <algorithm>
@@ -39,13 +38,15 @@ namespace jb {
 
 namespace {
 constexpr int kTile = 128 * 64 * 2;  // one [128 x 64] f16 tile, 16 KB
-constexpr int kStages = 2;
-constexpr int kOffQ = 0;                           // Q0, Q1
-constexpr int kOffK = kOffQ + 2 * kTile;           // K ring
-constexpr int kOffV = kOffK + kStages * kTile;     // V^T ring, each [64 dims x 128 keys] as two [64 x 64]
-constexpr int kOffP = kOffV + kStages * kTile;     // P[g][b]: query tile g, buffer b, each [128 x 128 keys]
-constexpr int kAttnSmem = kOffP + 2 * 2 * 2 * kTile + 1024;  // as two [128 x 64] halves
+constexpr int kStages = 4;
+constexpr int kOffQ = 0;                        // Q0, Q1
+constexpr int kOffK = kOffQ + 2 * kTile;        // K ring
+constexpr int kOffV = kOffK + kStages * kTile;  // V^T ring, each [64 dims x 128 keys] as two [64 x 64]
+constexpr int kAttnSmem = kOffV + kStages * kTile + 1024;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O when the row max grew by more than 2^8
+// TMEM columns: S_g (f32, 128 keys), O_g (f32, 64 dims), P_g (f16 pairs, 128 keys)
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+constexpr int kThreads = 19 * 32;  // producer, 2 MMA issuers, 2 x 8 softmax warps
 }  // namespace
 
 __device__ __forceinline__ void key_range(const AttnParams& p, int i, int& lo, int& hi) {
@@ -75,13 +76,16 @@ __device__ __forceinline__ int kv_tiles(const AttnParams& p, int q0) {
   return (max(hi_a, hi_b) + 1 + 127) / 128;
 }
 
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   extern __shared__ uint8_t dsmem[];
   __shared__ uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  // per query tile g: S ready / S taken, and per P buffer b: P written / PV done
-  __shared__ uint64_t s_full[2], s_free[2], p_full[2][2], pv_done[2][2], drain_bar[2];
+  // per query tile g: S ready / S taken / P written / PV done
+  __shared__ uint64_t s_full[2], s_free[2], p_full[2], pv_done[2], drain_bar[2];
+  __shared__ uint64_t x_bar[2];         // per query tile: both halves of every row posted their partial
+  __shared__ float xmax[2][2][2][128];  // [tile parity][g][column half][row]: partial row maxima
+  __shared__ float xsum[2][2][128];     // [g][column half][row]: partial row sums
   __shared__ uint32_t tmem_sh;
   __shared__ int abort_sh;
 
@@ -110,12 +114,11 @@ __global__ void __launch_bounds__(352, 1)
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(&s_full[g], 1);
-      mbar_init(&s_free[g], 128);
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(&p_full[g][b], 128);
-        mbar_init(&pv_done[g][b], 1);
-      }
+      mbar_init(&s_free[g], 256);
+      mbar_init(&p_full[g], 256);
+      mbar_init(&pv_done[g], 1);
       mbar_init(&drain_bar[g], 1);
+      mbar_init(&x_bar[g], 256);
     }
     abort_sh = 0;
     mbar_fence_init();
@@ -127,7 +130,7 @@ __global__ void __launch_bounds__(352, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = tmem_sh;  // S_g: columns 128g..128g+127; O_g: 256+64g..256+64g+63
+  const uint32_t tmem = tmem_sh;
 
   WaitCtl w;
   w.abort = reinterpret_cast<volatile int*>(&abort_sh);
@@ -171,7 +174,7 @@ __global__ void __launch_bounds__(352, 1)
         }
       }
     }
-  } else if (warp == 1 || warp == 10) {
+  } else if (warp == 1 || warp == 18) {
     // one MMA issuer per query tile, so each tile's S / PV products follow
     // its own softmax without waiting on the other tile's
     if (lane == 0) {
@@ -200,8 +203,8 @@ __global__ void __launch_bounds__(352, 1)
             const uint64_t kd = sdesc_kmajor_sw128(smem_u32(sm + kOffK + ks * kTile));
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              tc_mma_f16_ss(tmem + 128 * g, qd + static_cast<uint64_t>(2 * k), kd + static_cast<uint64_t>(2 * k),
-                            idesc_s, k > 0 ? 1u : 0u);
+              tc_mma_f16_ss(tmem + kColS + 128 * g, qd + static_cast<uint64_t>(2 * k),
+                            kd + static_cast<uint64_t>(2 * k), idesc_s, k > 0 ? 1u : 0u);
             tc_commit(&s_full[g]);
           }
           tc_commit(&k_empty[ks]);
@@ -212,22 +215,20 @@ __global__ void __launch_bounds__(352, 1)
             ok = false;
             break;
           }
-          if (j <= nkv_g) {  // O_g += P_g V_{j-1} once softmax g published P_g of tile j-1
-            const int pbuf = (j - 1) & 1;
-            if (!mbar_wait(&p_full[g][pbuf], ((j - 1) >> 1) & 1, w)) {
+          if (j <= nkv_g) {  // O_g += P_g V_{j-1} (P from TMEM) once softmax g published P_g
+            if (!mbar_wait(&p_full[g], (j - 1) & 1, w)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t pb = smem_u32(sm + kOffP + (g * 2 + pbuf) * 2 * kTile);
             const uint32_t vb = smem_u32(sm + kOffV + vs * kTile);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-              const uint64_t ad = sdesc_kmajor_sw128(pb + (k >> 2) * kTile) + static_cast<uint64_t>(2 * (k & 3));
               const uint64_t bd = sdesc_kmajor_sw128(vb + (k >> 2) * (kTile / 2)) + static_cast<uint64_t>(2 * (k & 3));
-              tc_mma_f16_ss(tmem + 256 + 64 * g, ad, bd, idesc_o, (j > 1 || k > 0) ? 1u : 0u);
+              tc_mma_f16_ts(tmem + kColO + 64 * g, tmem + kColP + 64 * g + 8 * k, bd, idesc_o,
+                            (j > 1 || k > 0) ? 1u : 0u);
             }
-            tc_commit(&pv_done[g][pbuf]);
+            tc_commit(&pv_done[g]);
           }
           tc_commit(&v_empty[vs]);
         }
@@ -235,17 +236,20 @@ __global__ void __launch_bounds__(352, 1)
       tc_commit(&drain_bar[g]);
       mbar_wait_drain(&drain_bar[g], 0);
     }
-  } else if (warp < 10) {
-    // softmax: warps 2-5 take query tile 0, warps 6-9 query tile 1
-    const int g = (warp - 2) >> 2;
+  } else {
+    // softmax: warps 2-9 take query tile 0, warps 10-17 query tile 1; two
+    // threads per query row, each with half of the 128 keys of a tile (and
+    // half of the 64 output columns)
+    const int g = (warp - 2) >> 3;
+    const int ch = ((warp - 2) >> 2) & 1;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int i = (g == 0 ? q00 : q01) + r;
     const int n_my = g == 0 ? nkv0 : nkv1;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tS = tmem + 128 * g + lane_off;
-    const uint32_t tO = tmem + 256 + 64 * g + lane_off;
-    const uint32_t pbase0 = smem_u32(sm + kOffP + g * 2 * 2 * kTile);
+    const uint32_t tS = tmem + kColS + 128 * g + 64 * ch + lane_off;
+    const uint32_t tO = tmem + kColO + 64 * g + 32 * ch + lane_off;
+    const uint32_t tP = tmem + kColP + 64 * g + 32 * ch + lane_off;
     int lo, hi;
     key_range(p, i, lo, hi);
     if (i >= p.N || (cls_cta && i == 0)) {
@@ -266,47 +270,46 @@ __global__ void __launch_bounds__(352, 1)
         break;
       }
       tc_fence_after();
-      float s[128];
+      float s[64];
       {
-        uint32_t u[128];
-        tmem_ld128(tS, u);
+        uint32_t u[64];
+        tmem_ld64(tS, u);
 #pragma unroll
-        for (int e = 0; e < 128; ++e) s[e] = __uint_as_float(u[e]);
+        for (int e = 0; e < 64; ++e) s[e] = __uint_as_float(u[e]);
       }
       tc_fence_before();
       mbar_arrive(&s_free[g]);  // S_g may now be overwritten by the next KV tile
-      const int kbase = j * 128;
-      const bool full = lo <= kbase && hi >= kbase + 127;
+      const int kbase = j * 128 + 64 * ch;
+      const bool full = lo <= kbase && hi >= kbase + 63;
       if (!__all_sync(0xffffffffu, full)) {
         const int rlo = lo - kbase, rhi = hi - kbase;
 #pragma unroll
-        for (int e = 0; e < 128; ++e) s[e] = (e >= rlo && e <= rhi) ? s[e] : -INFINITY;
+        for (int e = 0; e < 64; ++e) s[e] = (e >= rlo && e <= rhi) ? s[e] : -INFINITY;
       }
-      // row max as 8 independent chains (short dependency chains: two
-      // softmax warps per scheduler must hide the latency)
-      float mxv[8];
+      float mxv[4];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) mxv[t] = s[t];
+      for (int t = 0; t < 4; ++t) mxv[t] = fmax3(s[t], s[4 + t], s[8 + t]);
 #pragma unroll
-      for (int e = 8; e < 128; ++e) mxv[e & 7] = fmaxf(mxv[e & 7], s[e]);
-      const float mx = fmaxf(fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])),
-                             fmaxf(fmaxf(mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7])));
+      for (int e = 12; e < 60; e += 8) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) mxv[t] = fmax3(mxv[t], s[e + t], s[e + 4 + t]);
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) mxv[t] = fmaxf(mxv[t], s[60 + t]);
+      // the other half of the row: exchange partial maxima through shared
+      // memory (double-buffered by tile parity; bounded barrier wait)
+      xmax[j & 1][g][ch][r] = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
+      mbar_arrive(&x_bar[g]);
+      okw = mbar_wait(&x_bar[g], j & 1, w);
+      okw = __all_sync(0xffffffffu, okw);
+      if (!okw) {
+        ok = false;
+        break;
+      }
+      const float mx = fmaxf(xmax[j & 1][g][0][r], xmax[j & 1][g][1][r]);
       const float m_new = fmaxf(m_run, mx * c);
-      const int pbuf = j & 1;
-      if (j > 1) {  // P buffer pbuf is free once the PV product of tile j-2 is done
-        okw = mbar_wait(&pv_done[g][pbuf], ((j - 2) >> 1) & 1, w);
-        okw = __all_sync(0xffffffffu, okw);
-        if (!okw) {
-          ok = false;
-          break;
-        }
-      }
-      const bool grow = m_new > m_run + kRescaleLog2;
-      // tcgen05.ld / st are warp-collective: the warp rescales together,
-      // after every PV product so far (the one of tile j-1 last) is done
-      const bool rescale = j > 0 && __any_sync(0xffffffffu, grow);
-      if (rescale) {
-        okw = mbar_wait(&pv_done[g][pbuf ^ 1], ((j - 1) >> 1) & 1, w);
+      if (j > 0) {  // P_g free and O_g stable once the PV product of tile j-1 is done
+        okw = mbar_wait(&pv_done[g], (j - 1) & 1, w);
         okw = __all_sync(0xffffffffu, okw);
         if (!okw) {
           ok = false;
@@ -314,11 +317,13 @@ __global__ void __launch_bounds__(352, 1)
         }
       }
       tc_fence_after();
-      if (rescale) {
+      const bool grow = m_new > m_run + kRescaleLog2;
+      // tcgen05.ld / st are warp-collective: the warp rescales together
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
         const float alpha = grow ? ex2_approx(m_run - m_new) : 1.0f;
         l_run *= alpha;
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
           uint32_t o[16];
           tmem_ld16(tO + static_cast<uint32_t>(q * 16), o);
 #pragma unroll
@@ -329,53 +334,50 @@ __global__ void __launch_bounds__(352, 1)
       if (grow) m_run = m_new;
       // a row that has seen no allowed key yet keeps m = -inf: all its p are 0
       const float m_use = m_run == -INFINITY ? 0.0f : m_run;
+      // P = exp2(s*c - m): arguments and the row sum two lanes at a time,
+      // packed as f16 pairs into TMEM for the PV product
+      const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
+      uint64_t lsv2[4] = {0ull, 0ull, 0ull, 0ull};
+      uint32_t pk[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        float xa, xb;
+        f2_unpack(f2_fma(f2_pack(s[2 * e], s[2 * e + 1]), c2, nm2), xa, xb);
+        const float pa = ex2_approx(xa);
+        const float pb = ex2_approx(xb);
+        lsv2[e & 3] = f2_add(lsv2[e & 3], f2_pack(pa, pb));
+        pk[e] = pack_half2(pa, pb);
+      }
+      tmem_st32(tP, pk);
       float lsv[8];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) lsv[t] = 0.0f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {  // two [128 x 64] halves of the P tile
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int k = h * 64 + u * 8 + 2 * e;
-            const float pa = ex2_approx(fmaf(s[k], c, -m_use));
-            const float pb = ex2_approx(fmaf(s[k + 1], c, -m_use));
-            lsv[(2 * e) & 7] += pa;
-            lsv[(2 * e + 1) & 7] += pb;
-            pk[e] = pack_half2(pa, pb);
-          }
-          st_shared_v4(pbase0 + static_cast<uint32_t>((pbuf * 2 + h) * kTile) + sw128_offset(r, u * 8), pk[0], pk[1],
-                       pk[2], pk[3]);
-        }
-      }
+      for (int t = 0; t < 4; ++t) f2_unpack(lsv2[t], lsv[2 * t], lsv[2 * t + 1]);
       l_run += ((lsv[0] + lsv[1]) + (lsv[2] + lsv[3])) + ((lsv[4] + lsv[5]) + (lsv[6] + lsv[7]));
-      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[g][pbuf]);
+      mbar_arrive(&p_full[g]);
     }
     if (ok && n_my > 0) {  // the last PV product completes after all earlier ones
-      bool okw = mbar_wait(&pv_done[g][(n_my - 1) & 1], ((n_my - 1) >> 1) & 1, w);
+      bool okw = mbar_wait(&pv_done[g], (n_my - 1) & 1, w);
+      xsum[g][ch][r] = l_run;
+      mbar_arrive(&x_bar[g]);
+      okw = okw && mbar_wait(&x_bar[g], n_my & 1, w);
       okw = __all_sync(0xffffffffu, okw);
       if (okw) {
         tc_fence_after();
-        const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+        const float l_row = xsum[g][0][r] + xsum[g][1][r];
+        const float inv_l = l_row > 0.0f ? 1.0f / l_row : 0.0f;
         const int b = bh / p.heads, hd = bh % p.heads;
-#pragma unroll 1
-        for (int q = 0; q < 2; ++q) {
-          uint32_t o[32];
-          tmem_ld32(tO + static_cast<uint32_t>(q * 32), o);
-          if (store_row) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(b) * p.N + i) * p.ldo + hd * 64 + q * 32);
+        uint32_t o[32];
+        tmem_ld32(tO, o);
+        if (store_row) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(b) * p.N + i) * p.ldo + hd * 64 + ch * 32);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              uint32_t h[4];
+          for (int u = 0; u < 4; ++u) {
+            uint32_t h[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                h[e] = pack_half2(__uint_as_float(o[8 * u + 2 * e]) * inv_l, __uint_as_float(o[8 * u + 2 * e + 1]) * inv_l);
-              dst[u] = make_uint4(h[0], h[1], h[2], h[3]);
-            }
+            for (int e = 0; e < 4; ++e)
+              h[e] = pack_half2(__uint_as_float(o[8 * u + 2 * e]) * inv_l, __uint_as_float(o[8 * u + 2 * e + 1]) * inv_l);
+            dst[u] = make_uint4(h[0], h[1], h[2], h[3]);
           }
         }
       }
@@ -446,7 +448,7 @@ int attn_launch(const AttnOp& op, cudaStream_t st, DevErr* err, unsigned long lo
   p.err = err;
   p.timeout_ns = timeout_ns;
   dim3 grid((p.n_q_tiles + 1) / 2 + p.cls_separate, op.B * p.heads);
-  attn_fwd_kernel<<<grid, 352, kAttnSmem, st>>>(op.tmQ, op.tmK, op.tmV, p);
+  attn_fwd_kernel<<<grid, kThreads, kAttnSmem, st>>>(op.tmQ, op.tmK, op.tmV, p);
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 
