@@ -183,9 +183,6 @@ __device__ __forceinline__ void fill_a_patch(uint8_t* sA, const GemmParams& p, i
   const int ppf = (s.H / s.patch) * wp;
   const int pp = s.patch * s.patch;
   const int ktpp = s.tubelet * pp;
-  // patch rows of 8-multiple width on 16-byte aligned image rows and planes
-  const bool vec8 = (s.patch % 8 == 0) && (s.W % 4 == 0) && ((s.H * s.W) % 4 == 0) &&
-                    ((reinterpret_cast<uintptr_t>(s.pixels) & 15) == 0);
   const uint32_t sbase = smem_u32(sA);
   for (int idx = ct; idx < 128 * 8; idx += 128) {
     const int r = idx >> 3, u = idx & 7;
@@ -193,24 +190,7 @@ __device__ __forceinline__ void fill_a_patch(uint8_t* sA, const GemmParams& p, i
     float f[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) f[e] = 0.0f;
-    if (m < p.M && vec8) {
-      // 8 consecutive k = 8 consecutive pixels of one image row: two 16-byte loads
-      const int b = m / s.n_patches, i = m % s.n_patches;
-      const int tp = i / ppf, rem = i % ppf;
-      const int hp = rem / wp, wq = rem % wp;
-      const int k = kb * 64 + u * 8;
-      if (k < s.k_real) {
-        const int c = k / ktpp, rk = k % ktpp;
-        const int dt = rk / pp, rk2 = rk % pp;
-        const int kh = rk2 / s.patch, kw = rk2 % s.patch;
-        const size_t plane = (static_cast<size_t>(b) * s.T + tp * s.tubelet + dt) * 3 + c;
-        const float4* src =
-            reinterpret_cast<const float4*>(s.pixels + (plane * s.H + hp * s.patch + kh) * s.W + wq * s.patch + kw);
-        const float4 a = __ldg(src), bb = __ldg(src + 1);
-        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-        f[4] = bb.x; f[5] = bb.y; f[6] = bb.z; f[7] = bb.w;
-      }
-    } else if (m < p.M) {
+    if (m < p.M) {
       const int b = m / s.n_patches, i = m % s.n_patches;
       const int tp = i / ppf, rem = i % ppf;
       const int hp = rem / wp, wq = rem % wp;
@@ -228,6 +208,65 @@ __device__ __forceinline__ void fill_a_patch(uint8_t* sA, const GemmParams& p, i
     }
     st_shared_v4(sbase + sw128_offset(r, u * 8), pack_half2(f[0], f[1]), pack_half2(f[2], f[3]),
                  pack_half2(f[4], f[5]), pack_half2(f[6], f[7]));
+  }
+}
+
+// Fast gather for patches whose rows are multiples of 8 pixels on 16-byte
+// aligned image rows: a converter thread always fills the same 8-column unit
+// (u = ct % 8) of the same 8 tile rows, so the pixel offset of each of its
+// rows is computed once per tile (rowbase) and the offset of its unit once
+// per K block; each unit is two 16-byte loads.
+__device__ __forceinline__ bool patch_vec8(const PatchSrc& s) {
+  return (s.patch % 8 == 0) && (s.W % 4 == 0) && ((s.H * s.W) % 4 == 0) &&
+         ((reinterpret_cast<uintptr_t>(s.pixels) & 15) == 0);
+}
+
+__device__ __forceinline__ void patch_rowbases(const GemmParams& p, int m0, int ct, long long (&rowbase)[8]) {
+  const PatchSrc& s = p.patch;
+  const int wp = s.W / s.patch;
+  const int ppf = (s.H / s.patch) * wp;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int m = m0 + (ct >> 3) + 16 * it;
+    if (m < p.M) {
+      const int b = m / s.n_patches, i = m % s.n_patches;
+      const int tp = i / ppf, rem = i % ppf;
+      const int hp = rem / wp, wq = rem % wp;
+      rowbase[it] = ((static_cast<long long>(b) * s.T + tp * s.tubelet) * 3) * s.H * s.W +
+                    static_cast<long long>(hp * s.patch) * s.W + wq * s.patch;
+    } else {
+      rowbase[it] = -1;
+    }
+  }
+}
+
+__device__ __forceinline__ void fill_a_patch_vec8(uint8_t* sA, const GemmParams& p, int kb, int ct,
+                                                  const long long (&rowbase)[8]) {
+  const PatchSrc& s = p.patch;
+  const int u = ct & 7;
+  const int k = kb * 64 + u * 8;
+  long long koff = -1;
+  if (k < s.k_real) {
+    const int pp = s.patch * s.patch, ktpp = s.tubelet * pp;
+    const int c = k / ktpp, rk = k % ktpp;
+    const int dt = rk / pp, rk2 = rk % pp;
+    const int kh = rk2 / s.patch, kw = rk2 % s.patch;
+    koff = static_cast<long long>(dt * 3 + c) * s.H * s.W + static_cast<long long>(kh) * s.W + kw;
+  }
+  const uint32_t sbase = smem_u32(sA);
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int r = (ct >> 3) + 16 * it;
+    uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;
+    if (rowbase[it] >= 0 && koff >= 0) {
+      const float4* src = reinterpret_cast<const float4*>(s.pixels + rowbase[it] + koff);
+      const float4 a = __ldg(src), b = __ldg(src + 1);
+      w0 = pack_half2(a.x, a.y);
+      w1 = pack_half2(a.z, a.w);
+      w2 = pack_half2(b.x, b.y);
+      w3 = pack_half2(b.z, b.w);
+    }
+    st_shared_v4(sbase + sw128_offset(r, u * 8), w0, w1, w2, w3);
   }
 }
 
@@ -534,11 +573,14 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
     if (pending && lane == 0) bulk_wait0();
   } else if (CONV) {
     const int ct = threadIdx.x - 320;
+    const bool vec8 = GATHER && patch_vec8(p.patch);
+    long long rowbase[8];
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       const int nb = t % p.n_tiles, mb = t / p.n_tiles;
+      if (vec8) patch_rowbases(p, mb * 128, ct, rowbase);
       for (int kb = 0; kb < kblocks; ++kb) {
         bool okw = mbar_wait(&empty_bar[stage], phase ^ 1, w);
         okw = __all_sync(0xffffffffu, okw);
@@ -548,7 +590,9 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
         }
         uint8_t* sA = smem + stage * C::STAGE_BYTES;
         uint8_t* sB = sA + C::A_BYTES;
-        if (GATHER)
+        if (GATHER && vec8)
+          fill_a_patch_vec8(sA, p, kb, ct, rowbase);
+        else if (GATHER)
           fill_a_patch(sA, p, mb * 128, kb, ct);
         else
           fill_b_quant<BMODE, BN>(sB, p, nb * BN, kb, ct);

@@ -23,49 +23,50 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
                                                        long long in_stride, const float* __restrict__ g,
                                                        const float* __restrict__ b, float eps, void* out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + warp;
-  if (row >= rows) return;
   const int nv = D >> 2;
-  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(row) * in_stride * D);
-  float4 v[MAXV];
-  float s = 0.0f;
+  // grid-stride over rows: the grid is sized to the resident capacity
+  for (int row = blockIdx.x * 8 + warp; row < rows; row += gridDim.x * 8) {
+    const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(row) * in_stride * D);
+    float4 v[MAXV];
+    float s = 0.0f;
 #pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    const int idx = lane + 32 * i;
-    if (idx < nv) {
-      v[i] = __ldg(xr + idx);
-      s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
-    } else {
-      v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  }
-  const float mean = warp_sum(s) / static_cast<float>(D);
-  float q = 0.0f;
-#pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    if (lane + 32 * i < nv) {
-      const float a = v[i].x - mean, bb = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
-      q += (a * a + bb * bb) + (c * c + d * d);
-    }
-  }
-  const float rstd = rsqrtf(warp_sum(q) / static_cast<float>(D) + eps);
-  const float4* g4 = reinterpret_cast<const float4*>(g);
-  const float4* b4 = reinterpret_cast<const float4*>(b);
-#pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    const int idx = lane + 32 * i;
-    if (idx < nv) {
-      const float4 gg = __ldg(g4 + idx), bb = __ldg(b4 + idx);
-      const float y0 = (v[i].x - mean) * rstd * gg.x + bb.x;
-      const float y1 = (v[i].y - mean) * rstd * gg.y + bb.y;
-      const float y2 = (v[i].z - mean) * rstd * gg.z + bb.z;
-      const float y3 = (v[i].w - mean) * rstd * gg.w + bb.w;
-      if (OUT_F16) {
-        uint2* o = reinterpret_cast<uint2*>(static_cast<__half*>(out) + static_cast<size_t>(row) * D) + idx;
-        *o = make_uint2(pack_half2(y0, y1), pack_half2(y2, y3));
+    for (int i = 0; i < MAXV; ++i) {
+      const int idx = lane + 32 * i;
+      if (idx < nv) {
+        v[i] = __ldg(xr + idx);
+        s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
       } else {
-        float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + static_cast<size_t>(row) * D) + idx;
-        *o = make_float4(y0, y1, y2, y3);
+        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    const float mean = warp_sum(s) / static_cast<float>(D);
+    float q = 0.0f;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      if (lane + 32 * i < nv) {
+        const float a = v[i].x - mean, bb = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
+        q += (a * a + bb * bb) + (c * c + d * d);
+      }
+    }
+    const float rstd = rsqrtf(warp_sum(q) / static_cast<float>(D) + eps);
+    const float4* g4 = reinterpret_cast<const float4*>(g);
+    const float4* b4 = reinterpret_cast<const float4*>(b);
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int idx = lane + 32 * i;
+      if (idx < nv) {
+        const float4 gg = __ldg(g4 + idx), bb = __ldg(b4 + idx);
+        const float y0 = (v[i].x - mean) * rstd * gg.x + bb.x;
+        const float y1 = (v[i].y - mean) * rstd * gg.y + bb.y;
+        const float y2 = (v[i].z - mean) * rstd * gg.z + bb.z;
+        const float y3 = (v[i].w - mean) * rstd * gg.w + bb.w;
+        if (OUT_F16) {
+          uint2* o = reinterpret_cast<uint2*>(static_cast<__half*>(out) + static_cast<size_t>(row) * D) + idx;
+          *o = make_uint2(pack_half2(y0, y1), pack_half2(y2, y3));
+        } else {
+          float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + static_cast<size_t>(row) * D) + idx;
+          *o = make_float4(y0, y1, y2, y3);
+        }
       }
     }
   }
@@ -75,7 +76,7 @@ int launch_layernorm(const float* x, int rows, int D, long long in_stride, const
                      float eps, void* out, bool out_f16, cudaStream_t st) {
   if (!x || !g || !b || !out) return JEPA_B200_ERR_ARG;
   if (rows < 1 || D < 4 || D % 4 != 0 || D > 4096 || in_stride < 1) return JEPA_B200_ERR_SHAPE;
-  const dim3 grid((rows + 7) / 8);
+  const dim3 grid(std::min((rows + 7) / 8, num_sms() * 8));
   if (D <= 1024) {
     if (out_f16)
       layernorm_kernel<8, true><<<grid, 256, 0, st>>>(x, rows, D, in_stride, g, b, eps, out);
