@@ -94,11 +94,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_pairs = (p.n_q_tiles + 1) / 2;
-  const int bh = blockIdx.y;
-  // With a separate CLS row, CTA 0 computes the CLS row alone (query tile 0
-  // against every KV tile); the pair CTAs follow, later (heavier) tiles first.
-  const bool cls_cta = p.cls_separate && blockIdx.x == 0;
-  const int pair = n_pairs - 1 - (static_cast<int>(blockIdx.x) - p.cls_separate);
+  // Grid: (unit, clip*head), or (clip*head, unit) under the block-causal mask
+  // so that the hardware starts the heaviest units of every head first.  With
+  // a separate CLS row, unit 0 computes the CLS row alone (query tile 0
+  // against every KV tile); the pair units follow, later (heavier) tiles first.
+  const int unit = p.mask == JEPA_B200_MASK_BLOCK_CAUSAL ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
+  const int bh = p.mask == JEPA_B200_MASK_BLOCK_CAUSAL ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.y);
+  const bool cls_cta = p.cls_separate && unit == 0;
+  const int pair = n_pairs - 1 - (unit - p.cls_separate);
   const int q00 = cls_cta ? 0 : 2 * pair * 128, q01 = q00 + 128;  // first rows of query tiles 0 and 1
   const int nkv0 = cls_cta ? (p.N + 127) / 128 : kv_tiles(p, q00);
   const int nkv1 = cls_cta ? 0 : kv_tiles(p, q01);
@@ -447,7 +450,8 @@ int attn_launch(const AttnOp& op, cudaStream_t st, DevErr* err, unsigned long lo
   AttnParams p = op.p;
   p.err = err;
   p.timeout_ns = timeout_ns;
-  dim3 grid((p.n_q_tiles + 1) / 2 + p.cls_separate, op.B * p.heads);
+  const int units = (p.n_q_tiles + 1) / 2 + p.cls_separate;
+  const dim3 grid = p.mask == JEPA_B200_MASK_BLOCK_CAUSAL ? dim3(op.B * p.heads, units) : dim3(units, op.B * p.heads);
   attn_fwd_kernel<<<grid, kThreads, kAttnSmem, st>>>(op.tmQ, op.tmK, op.tmV, p);
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
