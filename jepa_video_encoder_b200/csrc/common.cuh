@@ -399,6 +399,51 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// GELU in its erf form, x * Phi(x), Phi the standard normal CDF: the
+// activation between ffn_up and ffn_down ("Quantization" page, "The rule";
+// the pages name no GELU variant, and the erf form is the one read here).
+// With u = |x|:  x * Phi(x) = max(x, 0) - u * Phi(-u)  for either sign of x,
+// and Phi(-u) = 2^q(u) with q a degree-11 polynomial fitted to log2 Phi(-u)
+// on [0, 6] (weighted least squares driven to equal ripple; q(0) = -1 so
+// that Phi(0) = 1/2 exactly; the fit is reproduced by gelu_fit.py next to
+// this file).  Evaluated in f32 with one ex2 per element the absolute error
+// is below 4e-8 on [-8, 8].  u is clamped to 6 in q: for x < -6 the result
+// is x * Phi(-6) (about 1e-9 |x|) instead of x * Phi(x), both zero once
+// rounded to f16 for |x| < 30.
+__device__ __forceinline__ float gelu_q(int k) {
+  constexpr float c[12] = {-1.000000000e+00f, -1.151105762e+00f, -4.592085183e-01f, -5.247146264e-02f,
+                           6.975546945e-03f,  -5.228150712e-06f, -2.895472280e-04f, 8.469620661e-05f,
+                           -1.389817317e-05f, 1.411672088e-06f,  -8.283102204e-08f, 2.152039880e-09f};
+  return c[k];
+}
+
+__device__ __forceinline__ float gelu1(float x) {
+  const float u = fabsf(x), c = fminf(u, 6.0f);
+  float q = gelu_q(11);
+#pragma unroll
+  for (int k = 10; k >= 0; --k) q = fmaf(q, c, gelu_q(k));
+  return fmaf(-u, ex2_approx(q), fmaxf(x, 0.0f));
+}
+
+// Two GELUs per call, the polynomial in packed f32x2 arithmetic.
+__device__ __forceinline__ void gelu2(float& x0, float& x1) {
+  const float u0 = fabsf(x0), u1 = fabsf(x1);
+  const uint64_t c = f2_pack(fminf(u0, 6.0f), fminf(u1, 6.0f));
+  uint64_t q = f2_pack(gelu_q(11), gelu_q(11));
+#pragma unroll
+  for (int k = 10; k >= 0; --k) q = f2_fma(q, c, f2_pack(gelu_q(k), gelu_q(k)));
+  float q0, q1;
+  f2_unpack(q, q0, q1);
+  x0 = fmaf(-u0, ex2_approx(q0), fmaxf(x0, 0.0f));
+  x1 = fmaf(-u1, ex2_approx(q1), fmaxf(x1, 0.0f));
+}
+
 // max of three floats in one instruction
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;

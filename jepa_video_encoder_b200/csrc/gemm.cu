@@ -41,9 +41,21 @@ struct GemmCfg {
   static constexpr int SMEM = STAGES * STAGE_BYTES + 8 * 4096 + 1024;  // + epilogue staging
 };
 
-__device__ __forceinline__ float gelu_erf(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
+// Two GELUs: packed polynomial, or (LOWREG, kernels launched with 448
+// threads and so at most 128 registers a thread) the scalar one whose
+// coefficients are instruction immediates rather than register pairs.
+template <bool LOWREG>
+__device__ __forceinline__ void gelu_pair(float& a, float& b) {
+  if (LOWREG) {
+    a = gelu1(a);
+    b = gelu1(b);
+  } else {
+    gelu2(a, b);
+  }
+}
 
 // Epilogue for 32 consecutive output columns col0..col0+31 of one row.
+template <bool LOWREG>
 __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int col0, const uint32_t (&r)[32]) {
   float v[32];
 #pragma unroll
@@ -62,7 +74,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int
   switch (p.epi) {
     case EPI_GELU_F16:
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+      for (int j = 0; j < 16; ++j) gelu_pair<LOWREG>(v[2 * j], v[2 * j + 1]);
       // fall through
     case EPI_F16: {
       uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(p.out) + static_cast<size_t>(row) * p.ldo + col0);
@@ -272,7 +284,7 @@ __device__ __forceinline__ void fill_a_patch_vec8(uint8_t* sA, const GemmParams&
 
 // Epilogue of one output tile for one thread: its row, half of the BN
 // columns (chalf), read from TMEM at tb (lane quadrant already applied).
-template <int BN>
+template <int BN, bool LOWREG>
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tb, int row, int nb, int chalf) {
   if (p.epi == EPI_RESID_F32) {
     // residual add: the residual's loads are issued before the TMEM load
@@ -306,7 +318,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tb, 
     for (int c = chalf * (BN / 64); c < (chalf + 1) * (BN / 64); ++c) {
       uint32_t r[32];
       tmem_ld32(tb + static_cast<uint32_t>(c * 32), r);
-      if (row < p.M) epilogue_chunk(p, row, nb * BN + c * 32, r);
+      if (row < p.M) epilogue_chunk<LOWREG>(p, row, nb * BN + c * 32, r);
     }
   }
 }
@@ -317,7 +329,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tb, 
 // 128-byte-swizzled layout and sent with one TMA store (f16 / f32 outputs)
 // or one TMA reduce-add (f32 residual: X += A W^T + b), so every global
 // write is a full, coalesced line.
-template <int BN>
+template <int BN, bool LOWREG>
 __device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUtensorMap* tmC, uint32_t tb,
                                                   int row0, int nb, int chalf, uint8_t* stage_buf, int lane,
                                                   bool& pending) {
@@ -373,26 +385,26 @@ __device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUt
       for (int h = 0; h < 2; ++h) {
         uint32_t r[32];
         tmem_ld32(tb + static_cast<uint32_t>((c + h) * 32), r);
-        float v[32];
+        const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0 + h * 32);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        if (p.bias) {
-          const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0 + h * 32);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 b = __ldg(b4 + j);
-            v[4 * j] += b.x;
-            v[4 * j + 1] += b.y;
-            v[4 * j + 2] += b.z;
-            v[4 * j + 3] += b.w;
+        for (int j = 0; j < 8; ++j) {
+          uint64_t lo = f2_pack(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]));
+          uint64_t hi = f2_pack(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+          if (p.bias) {
+            const float4 bb = __ldg(b4 + j);
+            lo = f2_add(lo, f2_pack(bb.x, bb.y));
+            hi = f2_add(hi, f2_pack(bb.z, bb.w));
           }
+          float x0, x1, x2, x3;
+          f2_unpack(lo, x0, x1);
+          f2_unpack(hi, x2, x3);
+          if (p.epi == EPI_GELU_F16) {
+            gelu_pair<LOWREG>(x0, x1);
+            gelu_pair<LOWREG>(x2, x3);
+          }
+          w[h * 16 + 2 * j] = pack_half2(x0, x1);
+          w[h * 16 + 2 * j + 1] = pack_half2(x2, x3);
         }
-        if (p.epi == EPI_GELU_F16) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
-        }
-#pragma unroll
-        for (int j = 0; j < 16; ++j) w[h * 16 + j] = pack_half2(v[2 * j], v[2 * j + 1]);
       }
       if (pending) {
         if (lane == 0) bulk_wait_read0();
@@ -560,9 +572,10 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
       const int row = mb * 128 + quad * 32 + lane;
       const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
       if (p.tma_epi)
-        epilogue_tile_tma<BN>(p, &tmC, tb, mb * 128 + quad * 32, nb, chalf, stage_buf, lane, pending);
+        epilogue_tile_tma<BN, (BMODE != B_F16 || GATHER)>(p, &tmC, tb, mb * 128 + quad * 32, nb, chalf, stage_buf, lane,
+                                                         pending);
       else
-        epilogue_tile<BN>(p, tb, row, nb, chalf);
+        epilogue_tile<BN, (BMODE != B_F16 || GATHER)>(p, tb, row, nb, chalf);
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
       if (++acc == 2) {
@@ -777,9 +790,9 @@ __global__ void __launch_bounds__(320, 1)
       const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quad * 32;
       const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
       if (p.tma_epi)
-        epilogue_tile_tma<BN>(p, &tmC, tb, row0, nb, chalf, stage_buf, lane, pending);
+        epilogue_tile_tma<BN, false>(p, &tmC, tb, row0, nb, chalf, stage_buf, lane, pending);
       else
-        epilogue_tile<BN>(p, tb, row0 + lane, nb, chalf);
+        epilogue_tile<BN, false>(p, tb, row0 + lane, nb, chalf);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tempty0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));

@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(256) gemv_kernel(const float* __restrict__ x, 
       float v = warp_sum_h(acc[m]);
       if (lane == 0) {
         if (bias) v += bias[n];
-        if (epi == 1) v = 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
+        if (epi == 1) v = gelu1(v);
         if (epi == 2) v += resid[static_cast<size_t>(m) * resid_stride + n];
         y[static_cast<size_t>(m) * N + n] = v;
       }
