@@ -311,34 +311,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float mx = fmaxf(xmax[j & 1][g][0][r], xmax[j & 1][g][1][r]);
       const float m_new = fmaxf(m_run, mx * c);
-      if (j > 0) {  // P_g free and O_g stable once the PV product of tile j-1 is done
-        okw = mbar_wait(&pv_done[g], (j - 1) & 1, w);
-        okw = __all_sync(0xffffffffu, okw);
-        if (!okw) {
-          ok = false;
-          break;
-        }
-      }
-      tc_fence_after();
       const bool grow = m_new > m_run + kRescaleLog2;
-      // tcgen05.ld / st are warp-collective: the warp rescales together
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        const float alpha = grow ? ex2_approx(m_run - m_new) : 1.0f;
-        l_run *= alpha;
-#pragma unroll 1
-        for (int q = 0; q < 2; ++q) {
-          uint32_t o[16];
-          tmem_ld16(tO + static_cast<uint32_t>(q * 16), o);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st16(tO + static_cast<uint32_t>(q * 16), o);
-        }
-      }
+      const float alpha = grow ? ex2_approx(m_run - m_new) : 1.0f;  // exp2(-inf) = 0 on the first tile
+      l_run *= alpha;
       if (grow) m_run = m_new;
       // a row that has seen no allowed key yet keeps m = -inf: all its p are 0
       const float m_use = m_run == -INFINITY ? 0.0f : m_run;
       // P = exp2(s*c - m): arguments and the row sum two lanes at a time,
-      // packed as f16 pairs into TMEM for the PV product
+      // packed as f16 pairs; computed before waiting for the previous PV
+      // product, which only the O rescale and the P store depend on
       const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
       uint64_t lsv2[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[32];
@@ -350,6 +331,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float pb = ex2_approx(xb);
         lsv2[e & 3] = f2_add(lsv2[e & 3], f2_pack(pa, pb));
         pk[e] = pack_half2(pa, pb);
+      }
+      if (j > 0) {  // P_g free and O_g stable once the PV product of tile j-1 is done
+        okw = mbar_wait(&pv_done[g], (j - 1) & 1, w);
+        okw = __all_sync(0xffffffffu, okw);
+        if (!okw) {
+          ok = false;
+          break;
+        }
+      }
+      tc_fence_after();
+      // tcgen05.ld / st are warp-collective: the warp rescales together
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+        for (int q = 0; q < 2; ++q) {
+          uint32_t o[16];
+          tmem_ld16(tO + static_cast<uint32_t>(q * 16), o);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st16(tO + static_cast<uint32_t>(q * 16), o);
+        }
       }
       tmem_st32(tP, pk);
       float lsv[8];
