@@ -109,10 +109,25 @@ def _clock_sampler_stop(proc, fh, path, gpu_index):
             "samples": len(sm)}
 
 
-def _src_hash():
+# The sources each kernel class is compiled from: a traffic figure stays valid
+# while these files are unchanged.
+_CLASS_SOURCES = {
+    "attention": ("attention.cu", "common.cuh", "internal.h"),
+    "layernorm": ("norm_pool.cu", "common.cuh", "internal.h"),
+    "pool_head": ("head.cu", "norm_pool.cu", "common.cuh", "internal.h"),
+}
+_GEMM_SOURCES = ("gemm.cu", "common.cuh", "internal.h")
+
+
+def _src_hash(kernel_class=None):
+    names = _CLASS_SOURCES.get(kernel_class, _GEMM_SOURCES if kernel_class and (
+        kernel_class.startswith("gemm_") or kernel_class == "patch_embed") else None)
+    csrc = os.path.join(ROOT, "jepa_video_encoder_b200", "csrc")
+    paths = [os.path.join(csrc, n) for n in names] if names else sorted(glob.glob(os.path.join(csrc, "*")))
+    paths.append(os.path.join(ROOT, "include", "jepa_b200.h"))
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "jepa_video_encoder_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
+    for path in paths:
+        with open(path, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
@@ -123,7 +138,7 @@ def _traffic(kernel_class, cfg_name):
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
-    src = _src_hash()
+    src = _src_hash(kernel_class)
     for line in open(p):
         parts = line.split()
         if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel_class and parts[1] == cfg_name \

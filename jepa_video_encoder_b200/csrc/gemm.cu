@@ -323,6 +323,13 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tb, 
   }
 }
 
+// Bias of 32 consecutive output columns (zeros without a bias).
+__device__ __forceinline__ void load_bias32(const float* bias, int col0, float4 (&bb)[8]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    bb[j] = bias ? __ldg(reinterpret_cast<const float4*>(bias + col0) + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
 // TMA epilogue of one output tile for one warp: 32 rows starting at row0,
 // half of the BN columns (chalf).  Each 32-row x 128-byte chunk (32 f32
 // columns, or 64 f16 columns) is written to the warp's staging buffer in the
@@ -340,17 +347,20 @@ __device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUt
   if (p.epi == EPI_F32 || p.epi == EPI_RESID_F32) {
 #pragma unroll 1
     for (int c = c_begin; c < c_end; ++c) {
+      const int col0 = nb * BN + c * 32;
+      // the bias loads are issued first so that their latency overlaps the
+      // TMEM load's (after it in the 128-register kernels)
+      float4 bb[8];
+      if (!LOWREG) load_bias32(p.bias, col0, bb);
       uint32_t r[32];
       tmem_ld32(tb + static_cast<uint32_t>(c * 32), r);
-      const int col0 = nb * BN + c * 32;
       float v[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-      if (p.bias) {
-        const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
+      if (!LOWREG || p.bias) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float4 b = __ldg(b4 + j);
+          const float4 b = LOWREG ? __ldg(reinterpret_cast<const float4*>(p.bias + col0) + j) : bb[j];
           v[4 * j] += b.x;
           v[4 * j + 1] += b.y;
           v[4 * j + 2] += b.z;
@@ -383,17 +393,21 @@ __device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUt
       const int col0 = nb * BN + c * 32;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
+        float4 bb[8];  // issued before the TMEM load so the two latencies overlap
+        if (!LOWREG) load_bias32(p.bias, col0 + h * 32, bb);
         uint32_t r[32];
         tmem_ld32(tb + static_cast<uint32_t>((c + h) * 32), r);
-        const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0 + h * 32);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           uint64_t lo = f2_pack(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]));
           uint64_t hi = f2_pack(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-          if (p.bias) {
-            const float4 bb = __ldg(b4 + j);
-            lo = f2_add(lo, f2_pack(bb.x, bb.y));
-            hi = f2_add(hi, f2_pack(bb.z, bb.w));
+          if (!LOWREG) {
+            lo = f2_add(lo, f2_pack(bb[j].x, bb[j].y));
+            hi = f2_add(hi, f2_pack(bb[j].z, bb[j].w));
+          } else if (p.bias) {
+            const float4 b = __ldg(reinterpret_cast<const float4*>(p.bias + col0 + h * 32) + j);
+            lo = f2_add(lo, f2_pack(b.x, b.y));
+            hi = f2_add(hi, f2_pack(b.z, b.w));
           }
           float x0, x1, x2, x3;
           f2_unpack(lo, x0, x1);
