@@ -20,14 +20,20 @@
 //               S_g = Q_g K_j^T into TMEM (M=128, N=128, both operands in
 //               shared memory) and O_g += P_g V_{j-1} into TMEM (M=128, N=64,
 //               P read from TMEM);
-//   warps 2-9   softmax of query tile 0, warps 10-17 of query tile 1, two
-//               threads per query row, each with 64 of the tile's 128 keys:
+//   warps 2-9   softmax of query tile 0, warps 10-17 of query tile 1:
 //               scores read once from TMEM into registers (S is released at
-//               once for the next KV tile), row max combined through shared
-//               memory, O rescaled in TMEM only when the max grew by more
-//               than 2^8 (lazy rescaling: P stays <= 256, exact after the
-//               final division by the row sum), P = exp2(s*c - m) packed as
-//               f16 pairs into TMEM for the PV product.
+//               once for the next KV tile), O rescaled in TMEM only when the
+//               row max grew by more than 2^8 (lazy rescaling: P stays <= 256,
+//               exact after the final division by the row sum), P =
+//               exp2(s*c - m) packed as f16 pairs into TMEM for the PV
+//               product.  Two row layouts (template ROWS_IN_WARP):
+//                 bidirectional: two threads per row in two warps of a lane
+//                 quadrant (32x32b TMEM shape), each with 64 keys, row max
+//                 and sum combined through shared memory;
+//                 block-causal: four threads per row in one warp (16x256b /
+//                 16x128b TMEM shapes), each with 32 keys of two rows, row
+//                 max and sum combined with shuffles -- no cross-warp barrier
+//                 per KV tile, which dominates the short block-causal tiles.
 #include <string.h>
 
 #include <algorithm>
@@ -76,6 +82,17 @@ __device__ __forceinline__ int kv_tiles(const AttnParams& p, int q0) {
   return (max(hi_a, hi_b) + 1 + 127) / 128;
 }
 
+// Allowed keys of tile row i in this CTA: rows past N (padding) and, in
+// the CLS CTA, row 0 take every key.
+__device__ __forceinline__ void row_keys(const AttnParams& p, bool cls_cta, int i, int& lo, int& hi) {
+  key_range(p, i, lo, hi);
+  if (i >= p.N || (cls_cta && i == 0)) {
+    lo = 0;
+    hi = p.N - 1;
+  }
+}
+
+template <bool ROWS_IN_WARP>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
@@ -83,7 +100,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   // per query tile g: S ready / S taken / P written / PV done
   __shared__ uint64_t s_full[2], s_free[2], p_full[2], pv_done[2], drain_bar[2];
-  __shared__ uint64_t x_bar[2];         // per query tile: both halves of every row posted their partial
+  // cross-warp row layout only: both halves of every row posted their partial
+  __shared__ uint64_t x_bar[2];
   __shared__ float xmax[2][2][2][128];  // [tile parity][g][column half][row]: partial row maxima
   __shared__ float xsum[2][2][128];     // [g][column half][row]: partial row sums
   __shared__ uint32_t tmem_sh;
@@ -239,10 +257,172 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(&drain_bar[g]);
       mbar_wait_drain(&drain_bar[g], 0);
     }
+  } else if constexpr (ROWS_IN_WARP) {
+    // softmax: warps 2-9 take query tile 0, warps 10-17 query tile 1.  The
+    // two warps of a TMEM lane quadrant take its 32 rows in halves of 16;
+    // through the 16-lane TMEM shapes four threads share a row, each with 32
+    // of a KV tile's 128 keys, and every thread holds two rows (ra, ra + 8),
+    // so row maxima and row sums are reduced with two shuffles in the warp.
+    const int g = (warp - 2) >> 3;
+    const int hh = ((warp - 2) >> 2) & 1;
+    const int quad = warp & 3;
+    const int lane_base = quad * 32 + hh * 16;
+    const int kq = lane & 3;  // this thread's keys in every group of 8: 2*kq, 2*kq + 1
+    const int ra = lane_base + (lane >> 2);
+    const int q0 = g == 0 ? q00 : q01;
+    const int ia = q0 + ra, ib = ia + 8;
+    const int n_my = g == 0 ? nkv0 : nkv1;
+    const uint32_t lane_off = static_cast<uint32_t>(lane_base) << 16;
+    const uint32_t tS = tmem + kColS + 128 * g + lane_off;
+    const uint32_t tO = tmem + kColO + 64 * g + lane_off;
+    const uint32_t tP = tmem + kColP + 64 * g + lane_off;
+    int loa, hia, lob, hib;
+    row_keys(p, cls_cta, ia, loa, hia);
+    row_keys(p, cls_cta, ib, lob, hib);
+    const float c = p.scale_log2;
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.0f, l_b = 0.0f;  // l: this thread's share of the row sum
+    bool ok = true;
+    for (int j = 0; j < n_my; ++j) {
+      bool okw = mbar_wait(&s_full[g], j & 1, w);
+      okw = __all_sync(0xffffffffu, okw);
+      if (!okw) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[64];
+      {
+        uint32_t u[64];
+        tmem_ld_16x256b_x16(tS, u);
+#pragma unroll
+        for (int e = 0; e < 64; ++e) s[e] = __uint_as_float(u[e]);
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[g]);  // S_g may now be overwritten by the next KV tile
+      const int kbase = j * 128;
+      const bool full = loa <= kbase && hia >= kbase + 127 && lob <= kbase && hib >= kbase + 127;
+      if (!__all_sync(0xffffffffu, full)) {
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const int key = kbase + 8 * m + 2 * kq;
+          s[4 * m] = (key >= loa && key <= hia) ? s[4 * m] : -INFINITY;
+          s[4 * m + 1] = (key + 1 >= loa && key + 1 <= hia) ? s[4 * m + 1] : -INFINITY;
+          s[4 * m + 2] = (key >= lob && key <= hib) ? s[4 * m + 2] : -INFINITY;
+          s[4 * m + 3] = (key + 1 >= lob && key + 1 <= hib) ? s[4 * m + 3] : -INFINITY;
+        }
+      }
+      float xa = fmaxf(s[0], s[1]), xb = fmaxf(s[2], s[3]);
+      float ya = fmaxf(s[4], s[5]), yb = fmaxf(s[6], s[7]);
+#pragma unroll
+      for (int m = 2; m < 16; m += 2) {
+        xa = fmax3(xa, s[4 * m], s[4 * m + 1]);
+        xb = fmax3(xb, s[4 * m + 2], s[4 * m + 3]);
+        ya = fmax3(ya, s[4 * m + 4], s[4 * m + 5]);
+        yb = fmax3(yb, s[4 * m + 6], s[4 * m + 7]);
+      }
+      float mxa = fmaxf(xa, ya), mxb = fmaxf(xb, yb);
+      mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
+      mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
+      mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
+      mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
+      const float mna = fmaxf(m_a, mxa * c), mnb = fmaxf(m_b, mxb * c);
+      const bool ga = mna > m_a + kRescaleLog2, gb = mnb > m_b + kRescaleLog2;
+      const float alpha_a = ga ? ex2_approx(m_a - mna) : 1.0f;  // exp2(-inf) = 0 on the first tile
+      const float alpha_b = gb ? ex2_approx(m_b - mnb) : 1.0f;
+      l_a *= alpha_a;
+      l_b *= alpha_b;
+      if (ga) m_a = mna;
+      if (gb) m_b = mnb;
+      // a row that has seen no allowed key yet keeps m = -inf: all its p are 0
+      const float mua = m_a == -INFINITY ? 0.0f : m_a, mub = m_b == -INFINITY ? 0.0f : m_b;
+      // P = exp2(s*c - m), two lanes at a time, packed as f16 pairs in the
+      // 16x128b order (one word per row and 4-column group); computed
+      // before waiting for the previous PV product, which only the O
+      // rescale and the P store depend on
+      const uint64_t c2 = f2_pack(c, c), nma = f2_pack(-mua, -mua), nmb = f2_pack(-mub, -mub);
+      uint64_t sa[2] = {0ull, 0ull}, sb[2] = {0ull, 0ull};
+      uint32_t pk[32];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        float x0, x1, x2, x3;
+        f2_unpack(f2_fma(f2_pack(s[4 * m], s[4 * m + 1]), c2, nma), x0, x1);
+        f2_unpack(f2_fma(f2_pack(s[4 * m + 2], s[4 * m + 3]), c2, nmb), x2, x3);
+        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+        const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+        sa[m & 1] = f2_add(sa[m & 1], f2_pack(p0, p1));
+        sb[m & 1] = f2_add(sb[m & 1], f2_pack(p2, p3));
+        pk[2 * m] = pack_half2(p0, p1);
+        pk[2 * m + 1] = pack_half2(p2, p3);
+      }
+      if (j > 0) {  // P_g free and O_g stable once the PV product of tile j-1 is done
+        okw = mbar_wait(&pv_done[g], (j - 1) & 1, w);
+        okw = __all_sync(0xffffffffu, okw);
+        if (!okw) {
+          ok = false;
+          break;
+        }
+      }
+      tc_fence_after();
+      // tcgen05.ld / st are warp-collective: the warp rescales together
+      if (j > 0 && __any_sync(0xffffffffu, ga || gb)) {
+        uint32_t o[32];
+        tmem_ld_16x256b_x8(tO, o);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          o[4 * m] = __float_as_uint(__uint_as_float(o[4 * m]) * alpha_a);
+          o[4 * m + 1] = __float_as_uint(__uint_as_float(o[4 * m + 1]) * alpha_a);
+          o[4 * m + 2] = __float_as_uint(__uint_as_float(o[4 * m + 2]) * alpha_b);
+          o[4 * m + 3] = __float_as_uint(__uint_as_float(o[4 * m + 3]) * alpha_b);
+        }
+        tmem_st_16x256b_x8(tO, o);
+      }
+      tmem_st_16x128b_x16(tP, pk);
+      float t0, t1, t2, t3;
+      f2_unpack(f2_add(sa[0], sa[1]), t0, t1);
+      f2_unpack(f2_add(sb[0], sb[1]), t2, t3);
+      l_a += t0 + t1;
+      l_b += t2 + t3;
+      tc_fence_before();
+      mbar_arrive(&p_full[g]);
+    }
+    if (ok && n_my > 0) {  // the last PV product completes after all earlier ones
+      bool okw = mbar_wait(&pv_done[g], (n_my - 1) & 1, w);
+      okw = __all_sync(0xffffffffu, okw);
+      l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+      l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+      l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+      l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+      if (okw) {
+        tc_fence_after();
+        const float inv_a = l_a > 0.0f ? 1.0f / l_a : 0.0f;
+        const float inv_b = l_b > 0.0f ? 1.0f / l_b : 0.0f;
+        const int b = bh / p.heads, hd = bh % p.heads;
+        uint32_t o[32];
+        tmem_ld_16x256b_x8(tO, o);
+        // rows this CTA writes: the CLS CTA only row 0; pair CTAs every
+        // valid row but a separately computed CLS row
+        const bool st_a = cls_cta ? (ia == 0) : (ia < p.N && !(ia == 0 && p.cls_separate));
+        const bool st_b = cls_cta ? (ib == 0) : (ib < p.N && !(ib == 0 && p.cls_separate));
+        if (st_a) {
+          uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (static_cast<size_t>(b) * p.N + ia) * p.ldo + hd * 64 + 2 * kq);
+#pragma unroll
+          for (int m = 0; m < 8; ++m)
+            dst[4 * m] = pack_half2(__uint_as_float(o[4 * m]) * inv_a, __uint_as_float(o[4 * m + 1]) * inv_a);
+        }
+        if (st_b) {
+          uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (static_cast<size_t>(b) * p.N + ib) * p.ldo + hd * 64 + 2 * kq);
+#pragma unroll
+          for (int m = 0; m < 8; ++m)
+            dst[4 * m] = pack_half2(__uint_as_float(o[4 * m + 2]) * inv_b, __uint_as_float(o[4 * m + 3]) * inv_b);
+        }
+      }
+    }
   } else {
-    // softmax: warps 2-9 take query tile 0, warps 10-17 query tile 1; two
-    // threads per query row, each with half of the 128 keys of a tile (and
-    // half of the 64 output columns)
+    // softmax, rows split across warps: warps 2-9 take query tile 0, warps
+    // 10-17 query tile 1; two threads per query row (in two warps of the
+    // same TMEM lane quadrant), each with half of the 128 keys of a tile
+    // (and half of the 64 output columns), row maxima and sums combined
+    // through shared memory behind a bounded barrier
     const int g = (warp - 2) >> 3;
     const int ch = ((warp - 2) >> 2) & 1;
     const int quad = warp & 3;
@@ -438,23 +618,33 @@ int attn_prepare(AttnOp* op, const __half* q, const __half* k, const __half* vt,
   return JEPA_B200_OK;
 }
 
-int attn_launch(const AttnOp& op, cudaStream_t st, DevErr* err, unsigned long long timeout_ns) {
-  static unsigned long long attr_done = 0;
+template <bool ROWS_IN_WARP>
+static int attn_launch_impl(const AttnParams& p, const AttnOp& op, cudaStream_t st) {
+  auto kern = attn_fwd_kernel<ROWS_IN_WARP>;
+  static unsigned long long attr_done = 0;  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !((attr_done >> dev) & 1ull)) {
-    if (cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) != cudaSuccess)
       return JEPA_B200_ERR_CUDA;
     attr_done |= 1ull << dev;
   }
+  const int units = (p.n_q_tiles + 1) / 2 + p.cls_separate;
+  const dim3 grid = p.mask == JEPA_B200_MASK_BLOCK_CAUSAL ? dim3(op.B * p.heads, units) : dim3(units, op.B * p.heads);
+  kern<<<grid, kThreads, kAttnSmem, st>>>(op.tmQ, op.tmK, op.tmV, p);
+  return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+}
+
+int attn_launch(const AttnOp& op, cudaStream_t st, DevErr* err, unsigned long long timeout_ns) {
   AttnParams p = op.p;
   p.err = err;
   p.timeout_ns = timeout_ns;
-  const int units = (p.n_q_tiles + 1) / 2 + p.cls_separate;
-  const dim3 grid = p.mask == JEPA_B200_MASK_BLOCK_CAUSAL ? dim3(op.B * p.heads, units) : dim3(units, op.B * p.heads);
-  attn_fwd_kernel<<<grid, kThreads, kAttnSmem, st>>>(op.tmQ, op.tmK, op.tmV, p);
-  return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+  // Block-causal query tiles visit few KV tiles, where the per-tile row-max
+  // exchange between warps is a large share: rows kept inside one warp.
+  // Bidirectional tiles are long and bound by the exponentials, where the
+  // cross-warp layout issues fewer instructions.
+  if (p.mask == JEPA_B200_MASK_BLOCK_CAUSAL) return attn_launch_impl<true>(p, op, st);
+  return attn_launch_impl<false>(p, op, st);
 }
 
 }  // namespace jb

@@ -439,10 +439,98 @@ __device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUt
   }
 }
 
+// QKV epilogue of one output tile for one warp (32 rows from row0, half of
+// the BN columns).  Per head and 32 token rows, Q and K are one 32 x 128-byte
+// tile of [B*h, N, 64]: staged like the f16 epilogue and sent with one 3-D
+// TMA store at (0, t0, b*h + head) when the 32 rows lie in one clip, else
+// written row by row.  V goes to V^T [B*h, 64, Npad] column by column (one
+// coalesced 64-byte store per dimension and warp).
+template <int BN, bool LOWREG>
+__device__ __forceinline__ void epilogue_tile_qkv(const GemmParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
+                                                  uint32_t tb, int row0, int nb, int chalf, uint8_t* stage_buf,
+                                                  int lane, bool& pending) {
+  const uint32_t sb = smem_u32(stage_buf);
+  const uint32_t row_off = static_cast<uint32_t>(lane) * 128u;
+  const int ntok = p.qkv.ntok, heads = p.qkv.heads;
+  const int row = row0 + lane;
+  const int b0 = row0 / ntok, t0 = row0 - b0 * ntok;
+  const bool one_clip = row0 + 31 < p.M && t0 + 31 < ntok;
+  const int c_begin = chalf * (BN / 64), c_end = (chalf + 1) * (BN / 64);
+#pragma unroll 1
+  for (int c = c_begin; c < c_end; c += 2) {
+    const int col0 = nb * BN + c * 32;
+    const int part = col0 / p.qkv.dim + p.qkv.first_part;
+    const int within = col0 % p.qkv.dim;
+    const int hd = within >> 6;
+    if (part == 2) {
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float4 bb[8];
+        if (!LOWREG) load_bias32(p.bias, col0 + h * 32, bb);
+        uint32_t r[32];
+        tmem_ld32(tb + static_cast<uint32_t>((c + h) * 32), r);
+        if (LOWREG) load_bias32(p.bias, col0 + h * 32, bb);
+        if (row < p.M && p.qkv.vt) {
+          const int b = row / ntok, t = row - b * ntok;
+          __half* base = p.qkv.vt + ((static_cast<size_t>(b) * heads + hd) * 64 + h * 32) * p.qkv.npad + t;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            base[static_cast<size_t>(4 * j) * p.qkv.npad] = __float2half_rn(__uint_as_float(r[4 * j]) + bb[j].x);
+            base[static_cast<size_t>(4 * j + 1) * p.qkv.npad] = __float2half_rn(__uint_as_float(r[4 * j + 1]) + bb[j].y);
+            base[static_cast<size_t>(4 * j + 2) * p.qkv.npad] = __float2half_rn(__uint_as_float(r[4 * j + 2]) + bb[j].z);
+            base[static_cast<size_t>(4 * j + 3) * p.qkv.npad] = __float2half_rn(__uint_as_float(r[4 * j + 3]) + bb[j].w);
+          }
+        }
+      }
+      continue;
+    }
+    __half* base = part == 0 ? p.qkv.q : p.qkv.k;
+    uint32_t w[32];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float4 bb[8];
+      if (!LOWREG) load_bias32(p.bias, col0 + h * 32, bb);
+      uint32_t r[32];
+      tmem_ld32(tb + static_cast<uint32_t>((c + h) * 32), r);
+      if (LOWREG) load_bias32(p.bias, col0 + h * 32, bb);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        w[h * 16 + 2 * j] = pack_half2(__uint_as_float(r[4 * j]) + bb[j].x, __uint_as_float(r[4 * j + 1]) + bb[j].y);
+        w[h * 16 + 2 * j + 1] =
+            pack_half2(__uint_as_float(r[4 * j + 2]) + bb[j].z, __uint_as_float(r[4 * j + 3]) + bb[j].w);
+      }
+    }
+    if (!base) continue;
+    if (one_clip) {  // warp-uniform
+      if (pending) {
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        st_shared_v4(sb + row_off + static_cast<uint32_t>(((u ^ (lane & 7)) & 7) << 4), w[4 * u], w[4 * u + 1],
+                     w[4 * u + 2], w[4 * u + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(part == 0 ? tmQ : tmK, stage_buf, 0, t0, b0 * heads + hd);
+        bulk_commit();
+      }
+      pending = true;
+    } else if (row < p.M) {
+      const int b = row / ntok, t = row - b * ntok;
+      uint4* dst = reinterpret_cast<uint4*>(base + ((static_cast<size_t>(b) * heads + hd) * ntok + t) * 64);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+    }
+  }
+}
+
 template <int BN, int BMODE, bool GATHER>
 __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
+                   const GemmParams p) {
   using C = GemmCfg<BN>;
   constexpr bool CONV = (BMODE != B_F16) || GATHER;
   constexpr int S = C::STAGES;
@@ -585,11 +673,19 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
       const int nb = t % p.n_tiles, mb = t / p.n_tiles;
       const int row = mb * 128 + quad * 32 + lane;
       const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
-      if (p.tma_epi)
-        epilogue_tile_tma<BN, (BMODE != B_F16 || GATHER)>(p, &tmC, tb, mb * 128 + quad * 32, nb, chalf, stage_buf, lane,
-                                                         pending);
+      constexpr bool kLowReg = BMODE != B_F16 || GATHER;
+      bool done = false;
+      if constexpr (!kLowReg) {  // the 128-register kernels keep the row-by-row QKV stores
+        if (p.tma_epi && p.epi == EPI_QKV) {
+          epilogue_tile_qkv<BN, false>(p, &tmC, &tmC2, tb, mb * 128 + quad * 32, nb, chalf, stage_buf, lane, pending);
+          done = true;
+        }
+      }
+      if (done) {
+      } else if (p.tma_epi && p.epi != EPI_QKV)
+        epilogue_tile_tma<BN, kLowReg>(p, &tmC, tb, mb * 128 + quad * 32, nb, chalf, stage_buf, lane, pending);
       else
-        epilogue_tile<BN, (BMODE != B_F16 || GATHER)>(p, tb, row, nb, chalf);
+        epilogue_tile<BN, kLowReg>(p, tb, row, nb, chalf);
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
       if (++acc == 2) {
@@ -664,7 +760,8 @@ struct Gemm2Cfg {
 template <int BN>
 __global__ void __launch_bounds__(320, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
+                     const GemmParams p) {
   using C = Gemm2Cfg<BN>;
   constexpr int S = C::STAGES;
   extern __shared__ uint8_t dsmem[];
@@ -803,7 +900,9 @@ __global__ void __launch_bounds__(320, 1)
       const int nb = t % p.n_tiles, mb = t / p.n_tiles;
       const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quad * 32;
       const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
-      if (p.tma_epi)
+      if (p.tma_epi && p.epi == EPI_QKV)
+        epilogue_tile_qkv<BN, true>(p, &tmC, &tmC2, tb, row0, nb, chalf, stage_buf, lane, pending);
+      else if (p.tma_epi)
         epilogue_tile_tma<BN, false>(p, &tmC, tb, row0, nb, chalf, stage_buf, lane, pending);
       else
         epilogue_tile<BN, false>(p, tb, row0 + lane, nb, chalf);
@@ -927,6 +1026,22 @@ int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& W, 
       return JEPA_B200_ERR_CUDA;
     p.tma_epi = 1;
   }
+  // QKV epilogue: Q and K as [B*h, N, 64] maps, 32 token rows per store
+  if (epi == EPI_QKV && qkv && (bn / 64) % 2 == 0 && qkv->ntok > 0 && M % qkv->ntok == 0 && qkv->dim % 64 == 0) {
+    const uint64_t BHn = static_cast<uint64_t>(M / qkv->ntok) * qkv->heads;
+    const uint64_t dims[3] = {64, static_cast<uint64_t>(qkv->ntok), BHn};
+    const uint64_t str[2] = {128, static_cast<uint64_t>(qkv->ntok) * 128};
+    const uint32_t box[3] = {64, 32, 1};
+    // a map is built for a missing destination too (on the other one's
+    // address); the epilogue never stores through it
+    const __half* qb = qkv->q ? qkv->q : qkv->k;
+    const __half* kb = qkv->k ? qkv->k : qkv->q;
+    if (qb && kb) {
+      if (!make_tmap_f16(&op->tmC, qb, 3, dims, str, box) || !make_tmap_f16(&op->tmC2, kb, 3, dims, str, box))
+        return JEPA_B200_ERR_CUDA;
+      p.tma_epi = 1;
+    }
+  }
   // f16 weights and at least two 128-row blocks: the CTA-pair kernel
   op->pair = (W.bmode == B_F16 && !patch && M >= 256) ? 1 : 0;
   if (W.bmode == B_F16) {
@@ -958,7 +1073,7 @@ static int launch_impl(const GemmOp& op, cudaStream_t st) {
     attr_done |= 1ull << dev;
   }
   constexpr int threads = (BMODE != B_F16 || GATHER) ? 448 : 320;
-  kern<<<op.grid, threads, GemmCfg<BN>::SMEM, st>>>(op.tmA, op.tmB, op.tmC, op.p);
+  kern<<<op.grid, threads, GemmCfg<BN>::SMEM, st>>>(op.tmA, op.tmB, op.tmC, op.tmC2, op.p);
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 
@@ -985,7 +1100,7 @@ static int launch_pair(const GemmOp& op, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, op.tmA, op.tmB, op.tmC, op.p) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, op.tmA, op.tmB, op.tmC, op.tmC2, op.p) != cudaSuccess) return JEPA_B200_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 

@@ -63,7 +63,8 @@ struct GemmParams {
 struct GemmOp {
   CUtensorMap tmA;
   CUtensorMap tmB;
-  CUtensorMap tmC;  // output map of the TMA epilogue
+  CUtensorMap tmC;   // output map of the TMA epilogue (Q for the QKV epilogue)
+  CUtensorMap tmC2;  // K map of the QKV epilogue
   GemmParams p;
   int bn = 0, bmode = 0, gather = 0, grid = 0, smem = 0;
   int pair = 0;  // 1: CTA-pair kernel (tcgen05 cta_group::2, 256-row tiles)
