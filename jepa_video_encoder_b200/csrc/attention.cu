@@ -9,9 +9,11 @@
 //   patch of slot s:    [c, c + (s+1) * P_f - 1]   (c = 1 with a CLS row)
 // so a query tile only visits KV tiles up to its largest hi (the fully masked
 // tiles past it are never loaded), and only tiles that cut an interval need
-// the per-element mask.  The CLS row, the one row that reads every key, gets
-// a CTA of its own (scheduled first), so that its query tile in the regular
-// CTAs stays as short as the first frame's.
+// the per-element mask.  The CLS row, the one row that reads every key, is
+// computed apart (a "CLS tile": the query tile at row 0 against every KV
+// tile, only row 0 kept) so that query tile 0 stays as short as the first
+// frame's: as the second tile of the last pair when the tile count is odd
+// (that pair has no second tile of its own), else in a CTA of its own.
 //
 // One CTA per (pair of 128-query tiles, clip*head), one CTA per SM:
 //   warp 0      TMA: both Q tiles once, then K and V^T tiles through a
@@ -84,9 +86,9 @@ __device__ __forceinline__ int kv_tiles(const AttnParams& p, int q0) {
 
 // Allowed keys of tile row i in this CTA: rows past N (padding) and, in
 // the CLS CTA, row 0 take every key.
-__device__ __forceinline__ void row_keys(const AttnParams& p, bool cls_cta, int i, int& lo, int& hi) {
+__device__ __forceinline__ void row_keys(const AttnParams& p, bool cls_tile, int i, int& lo, int& hi) {
   key_range(p, i, lo, hi);
-  if (i >= p.N || (cls_cta && i == 0)) {
+  if (i >= p.N || cls_tile) {
     lo = 0;
     hi = p.N - 1;
   }
@@ -118,11 +120,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   // against every KV tile); the pair units follow, later (heavier) tiles first.
   const int unit = p.mask == JEPA_B200_MASK_BLOCK_CAUSAL ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
   const int bh = p.mask == JEPA_B200_MASK_BLOCK_CAUSAL ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.y);
-  const bool cls_cta = p.cls_separate && unit == 0;
-  const int pair = n_pairs - 1 - (unit - p.cls_separate);
-  const int q00 = cls_cta ? 0 : 2 * pair * 128, q01 = q00 + 128;  // first rows of query tiles 0 and 1
+  // The CLS tile (query rows 0..127 against every key, only row 0 kept) is
+  // either the second tile of the last pair, whose own second tile does not
+  // exist when the tile count is odd, or the one tile of unit 0.
+  const int cls_unit = p.cls_separate && !p.cls_in_pair;
+  const bool cls_cta = cls_unit && unit == 0;
+  const int pair = n_pairs - 1 - (unit - cls_unit);
+  const int cls_g = cls_cta ? 0 : ((p.cls_in_pair && pair == n_pairs - 1) ? 1 : -1);  // query tile g holding CLS
+  const int q00 = cls_cta ? 0 : 2 * pair * 128;  // first rows of query tiles 0 and 1
+  const int q01 = cls_g == 1 ? 0 : q00 + 128;
   const int nkv0 = cls_cta ? (p.N + 127) / 128 : kv_tiles(p, q00);
-  const int nkv1 = cls_cta ? 0 : kv_tiles(p, q01);
+  const int nkv1 = cls_cta ? 0 : (cls_g == 1 ? (p.N + 127) / 128 : kv_tiles(p, q01));
   const int nkv_all = max(nkv0, nkv1);
 
   if (threadIdx.x == 0) {
@@ -277,8 +285,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + kColO + 64 * g + lane_off;
     const uint32_t tP = tmem + kColP + 64 * g + lane_off;
     int loa, hia, lob, hib;
-    row_keys(p, cls_cta, ia, loa, hia);
-    row_keys(p, cls_cta, ib, lob, hib);
+    const bool cls_tile = g == cls_g;
+    row_keys(p, cls_tile, ia, loa, hia);
+    row_keys(p, cls_tile, ib, lob, hib);
     const float c = p.scale_log2;
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.0f, l_b = 0.0f;  // l: this thread's share of the row sum
     bool ok = true;
@@ -401,8 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_16x256b_x8(tO, o);
         // rows this CTA writes: the CLS CTA only row 0; pair CTAs every
         // valid row but a separately computed CLS row
-        const bool st_a = cls_cta ? (ia == 0) : (ia < p.N && !(ia == 0 && p.cls_separate));
-        const bool st_b = cls_cta ? (ib == 0) : (ib < p.N && !(ib == 0 && p.cls_separate));
+        const bool st_a = cls_tile ? (ia == 0) : (ia < p.N && !(ia == 0 && p.cls_separate));
+        const bool st_b = cls_tile ? (ib == 0) : (ib < p.N && !(ib == 0 && p.cls_separate));
         if (st_a) {
           uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (static_cast<size_t>(b) * p.N + ia) * p.ldo + hd * 64 + 2 * kq);
 #pragma unroll
@@ -435,13 +444,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tP = tmem + kColP + 64 * g + 32 * ch + lane_off;
     int lo, hi;
     key_range(p, i, lo, hi);
-    if (i >= p.N || (cls_cta && i == 0)) {
+    const bool cls_tile = g == cls_g;
+    if (i >= p.N || cls_tile) {
       lo = 0;
       hi = p.N - 1;
     }
     // rows this CTA writes: the CLS CTA only row 0; pair CTAs every valid row
     // but a separately computed CLS row
-    const bool store_row = cls_cta ? (i == 0) : (i < p.N && !(i == 0 && p.cls_separate));
+    const bool store_row = cls_tile ? (i == 0) : (i < p.N && !(i == 0 && p.cls_separate));
     const float c = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
@@ -609,6 +619,7 @@ int attn_prepare(AttnOp* op, const __half* q, const __half* k, const __half* vt,
   p.out = out;
   p.ldo = heads * 64;
   p.cls_separate = (mask == JEPA_B200_MASK_BLOCK_CAUSAL && has_cls) ? 1 : 0;
+  p.cls_in_pair = (p.cls_separate && p.n_q_tiles % 2 == 1) ? 1 : 0;
   op->q = q;
   op->k = k;
   op->vt = vt;
@@ -629,7 +640,7 @@ static int attn_launch_impl(const AttnParams& p, const AttnOp& op, cudaStream_t 
       return JEPA_B200_ERR_CUDA;
     attr_done |= 1ull << dev;
   }
-  const int units = (p.n_q_tiles + 1) / 2 + p.cls_separate;
+  const int units = (p.n_q_tiles + 1) / 2 + (p.cls_separate && !p.cls_in_pair ? 1 : 0);
   const dim3 grid = p.mask == JEPA_B200_MASK_BLOCK_CAUSAL ? dim3(op.B * p.heads, units) : dim3(units, op.B * p.heads);
   kern<<<grid, kThreads, kAttnSmem, st>>>(op.tmQ, op.tmK, op.tmV, p);
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;

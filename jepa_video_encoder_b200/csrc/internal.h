@@ -78,7 +78,8 @@ int gemm_launch(const GemmOp& op, cudaStream_t st, DevErr* err, unsigned long lo
 
 struct AttnParams {
   int N, heads, n_q_tiles, mask, has_cls, ppf;
-  int cls_separate;  // block-causal with CLS: row 0 by the one-query kernel
+  int cls_separate;  // block-causal with CLS: row 0 computed apart from query tile 0
+  int cls_in_pair;   // ... as the second query tile of the last pair (odd tile count), else in a CTA of its own
   float scale_log2;
   __half* out;
   int ldo;

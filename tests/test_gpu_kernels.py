@@ -233,6 +233,8 @@ def _attn_case(B, heads, n_patches, ppf, has_cls, mask, seed, qscale=3.0):
     (1, 3, 256, 256, True, "bidir"),           # LeWM shape: 257 tokens
     (2, 1, 260, 4, False, "block_causal"),     # tiny slots: rows see keys in few tiles
     (1, 2, 64 * 4, 4, True, "block_causal"),   # slots of 4 with CLS
+    (2, 2, 384, 96, True, "block_causal"),     # 385 tokens: 4 query tiles, the CLS row in a CTA of its own
+    (1, 1, 127, 127, True, "block_causal"),    # 128 tokens: one query tile, paired with the CLS tile
     (1, 1, 1000, 1000, False, "bidir"),
 ])
 def test_attention(B, heads, n_patches, ppf, has_cls, mask):
