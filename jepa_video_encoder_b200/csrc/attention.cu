@@ -160,6 +160,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_sh;
+  pdl_wait();  // Q, K, V^T come from the previous kernel
+  pdl_trigger();
 
   WaitCtl w;
   w.abort = reinterpret_cast<volatile int*>(&abort_sh);
@@ -642,8 +644,9 @@ static int attn_launch_impl(const AttnParams& p, const AttnOp& op, cudaStream_t 
   }
   const int units = (p.n_q_tiles + 1) / 2 + (p.cls_separate && !p.cls_in_pair ? 1 : 0);
   const dim3 grid = p.mask == JEPA_B200_MASK_BLOCK_CAUSAL ? dim3(op.B * p.heads, units) : dim3(units, op.B * p.heads);
-  kern<<<grid, kThreads, kAttnSmem, st>>>(op.tmQ, op.tmK, op.tmV, p);
-  return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+  if (launch_pdl(kern, grid, dim3(kThreads), kAttnSmem, st, 1, op.tmQ, op.tmK, op.tmV, p) != cudaSuccess)
+    return JEPA_B200_ERR_CUDA;
+  return JEPA_B200_OK;
 }
 
 int attn_launch(const AttnOp& op, cudaStream_t st, DevErr* err, unsigned long long timeout_ns) {

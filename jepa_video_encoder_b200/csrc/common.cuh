@@ -424,6 +424,16 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int k) {
   return static_cast<uint32_t>(row * 128 + ((((k >> 3) ^ (row & 7)) & 7) << 4) + ((k & 7) << 1));
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization (launch_pdl) may start while the kernel before it in the
+// stream is still running; pdl_wait() returns once that kernel has completed
+// and its memory operations are visible, so every kernel calls it after its
+// own set-up and before it reads or writes anything another kernel touches.
+// pdl_trigger() lets the next kernel's blocks be scheduled (onto SMs this
+// grid has left).  Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

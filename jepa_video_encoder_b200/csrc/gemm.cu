@@ -569,6 +569,8 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
+  pdl_wait();  // A (and a residual output) come from the previous kernel
+  pdl_trigger();
 
   WaitCtl w;
   w.abort = reinterpret_cast<volatile int*>(&abort_sh);
@@ -799,6 +801,8 @@ __global__ void __launch_bounds__(320, 1)
   cluster_sync();  // barriers of both CTAs initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
+  pdl_wait();  // A (and a residual output) come from the previous kernel
+  pdl_trigger();
 
   WaitCtl w;
   w.abort = reinterpret_cast<volatile int*>(&abort_sh);
@@ -1073,8 +1077,10 @@ static int launch_impl(const GemmOp& op, cudaStream_t st) {
     attr_done |= 1ull << dev;
   }
   constexpr int threads = (BMODE != B_F16 || GATHER) ? 448 : 320;
-  kern<<<op.grid, threads, GemmCfg<BN>::SMEM, st>>>(op.tmA, op.tmB, op.tmC, op.tmC2, op.p);
-  return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+  if (launch_pdl(kern, dim3(op.grid), dim3(threads), GemmCfg<BN>::SMEM, st, 1, op.tmA, op.tmB, op.tmC, op.tmC2, op.p) !=
+      cudaSuccess)
+    return JEPA_B200_ERR_CUDA;
+  return JEPA_B200_OK;
 }
 
 template <int BN>
@@ -1088,19 +1094,9 @@ static int launch_pair(const GemmOp& op, cudaStream_t st) {
       return JEPA_B200_ERR_CUDA;
     attr_done |= 1ull << dev;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(op.grid);
-  cfg.blockDim = dim3(320);
-  cfg.dynamicSmemBytes = Gemm2Cfg<BN>::SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, op.tmA, op.tmB, op.tmC, op.tmC2, op.p) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+  if (launch_pdl(kern, dim3(op.grid), dim3(320), Gemm2Cfg<BN>::SMEM, st, 2, op.tmA, op.tmB, op.tmC, op.tmC2, op.p) !=
+      cudaSuccess)
+    return JEPA_B200_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 

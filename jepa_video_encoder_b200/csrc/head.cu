@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(256) gemv_kernel(const float* __restrict__ x, 
                                                   int N, const float* __restrict__ bias, int epi, const float* resid,
                                                   long long resid_stride, float* y) {
   extern __shared__ float xs[];
+  pdl_wait();
+  pdl_trigger();
   for (int i = threadIdx.x; i < M * K; i += 256) xs[i] = x[i];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -133,11 +135,14 @@ int launch_gemv(const float* x, int M, int K, const DevMatrix& W, const float* b
     const float* rr = resid ? resid + static_cast<size_t>(m0) * resid_stride : nullptr;
     float* yr = y + static_cast<size_t>(m0) * N;
     if (bm == 1)
-      gemv_kernel<B_Q8><<<grid, 256, smem, st>>>(xr, mc, K, W.data, W.scales, N, bias, epi, rr, resid_stride, yr);
+      launch_pdl(gemv_kernel<B_Q8>, grid, dim3(256), smem, st, 1, xr, mc, K, static_cast<const void*>(W.data),
+                 static_cast<const __half*>(W.scales), N, bias, epi, rr, resid_stride, yr);
     else if (bm == 2)
-      gemv_kernel<B_Q4><<<grid, 256, smem, st>>>(xr, mc, K, W.data, W.scales, N, bias, epi, rr, resid_stride, yr);
+      launch_pdl(gemv_kernel<B_Q4>, grid, dim3(256), smem, st, 1, xr, mc, K, static_cast<const void*>(W.data),
+                 static_cast<const __half*>(W.scales), N, bias, epi, rr, resid_stride, yr);
     else
-      gemv_kernel<B_F16><<<grid, 256, smem, st>>>(xr, mc, K, W.data, W.scales, N, bias, epi, rr, resid_stride, yr);
+      launch_pdl(gemv_kernel<B_F16>, grid, dim3(256), smem, st, 1, xr, mc, K, static_cast<const void*>(W.data),
+                 static_cast<const __half*>(W.scales), N, bias, epi, rr, resid_stride, yr);
   }
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
@@ -148,6 +153,8 @@ __global__ void __launch_bounds__(256) xattn_1q_kernel(const float* __restrict__
                                                        float* __restrict__ out) {
   extern __shared__ float sc[];
   __shared__ float qh[64];
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[8];
   const int bh = blockIdx.x, b = bh / heads, hd = bh % heads;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -213,7 +220,7 @@ int launch_xattn_1q(const float* q, const __half* k, const __half* vt, int B, in
       return JEPA_B200_ERR_CUDA;
     attr_done |= 1ull << dev;
   }
-  xattn_1q_kernel<<<B * heads, 256, smem, st>>>(q, k, vt, heads, ntok, npad, out);
+  launch_pdl(xattn_1q_kernel, dim3(B * heads), dim3(256), smem, st, 1, q, k, vt, heads, ntok, npad, out);
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 

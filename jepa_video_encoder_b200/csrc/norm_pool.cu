@@ -22,6 +22,8 @@ template <int MAXV, bool OUT_F16>
 __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict__ x, int rows, int D,
                                                        long long in_stride, const float* __restrict__ g,
                                                        const float* __restrict__ b, float eps, void* out) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nv = D >> 2;
   // grid-stride over rows: the grid is sized to the resident capacity
@@ -79,20 +81,22 @@ int launch_layernorm(const float* x, int rows, int D, long long in_stride, const
   const dim3 grid(std::min((rows + 7) / 8, num_sms() * 8));
   if (D <= 1024) {
     if (out_f16)
-      layernorm_kernel<8, true><<<grid, 256, 0, st>>>(x, rows, D, in_stride, g, b, eps, out);
+      launch_pdl(layernorm_kernel<8, true>, grid, dim3(256), 0, st, 1, x, rows, D, in_stride, g, b, eps, out);
     else
-      layernorm_kernel<8, false><<<grid, 256, 0, st>>>(x, rows, D, in_stride, g, b, eps, out);
+      launch_pdl(layernorm_kernel<8, false>, grid, dim3(256), 0, st, 1, x, rows, D, in_stride, g, b, eps, out);
   } else {
     if (out_f16)
-      layernorm_kernel<32, true><<<grid, 256, 0, st>>>(x, rows, D, in_stride, g, b, eps, out);
+      launch_pdl(layernorm_kernel<32, true>, grid, dim3(256), 0, st, 1, x, rows, D, in_stride, g, b, eps, out);
     else
-      layernorm_kernel<32, false><<<grid, 256, 0, st>>>(x, rows, D, in_stride, g, b, eps, out);
+      launch_pdl(layernorm_kernel<32, false>, grid, dim3(256), 0, st, 1, x, rows, D, in_stride, g, b, eps, out);
   }
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 
 // x[b, 0, :] = cls + pos[0]
 __global__ void cls_rows_kernel(float* x, int B, int ntok, int D, const float* cls, const float* pos) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.y;
   for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < D; c += gridDim.x * blockDim.x)
     x[static_cast<size_t>(b) * ntok * D + c] = cls[c] + pos[c];
@@ -100,7 +104,7 @@ __global__ void cls_rows_kernel(float* x, int B, int ntok, int D, const float* c
 
 int launch_cls_rows(float* x, int B, int ntok, int D, const float* cls, const float* pos, cudaStream_t st) {
   if (!x || !cls || !pos) return JEPA_B200_ERR_ARG;
-  cls_rows_kernel<<<dim3((D + 255) / 256, B), 256, 0, st>>>(x, B, ntok, D, cls, pos);
+  launch_pdl(cls_rows_kernel, dim3((D + 255) / 256, B), dim3(256), 0, st, 1, x, B, ntok, D, cls, pos);
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 
@@ -110,6 +114,8 @@ constexpr int kPoolSplits = 32;
 
 __global__ void mean_pool_partial_kernel(const float* __restrict__ y, int ntok, int D, int first,
                                          float* __restrict__ partial) {
+  pdl_wait();
+  pdl_trigger();
   const int col = blockIdx.x * 256 + threadIdx.x;
   const int sp = blockIdx.y, b = blockIdx.z;
   if (col >= D) return;
@@ -131,6 +137,8 @@ __global__ void mean_pool_partial_kernel(const float* __restrict__ y, int ntok, 
 
 __global__ void mean_pool_final_kernel(const float* __restrict__ partial, int B, int D, float inv_count,
                                        float* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   const int i = blockIdx.x * 256 + threadIdx.x;
   if (i >= B * D) return;
   const int b = i / D, col = i % D;
@@ -145,8 +153,10 @@ int launch_mean_pool(const float* y, int B, int ntok, int D, int first, float* p
                      cudaStream_t st) {
   if (!y || !partial || !out) return JEPA_B200_ERR_ARG;
   if (B < 1 || D < 1 || first < 0 || first >= ntok || B > 65535) return JEPA_B200_ERR_SHAPE;
-  mean_pool_partial_kernel<<<dim3((D + 255) / 256, kPoolSplits, B), 256, 0, st>>>(y, ntok, D, first, partial);
-  mean_pool_final_kernel<<<(B * D + 255) / 256, 256, 0, st>>>(partial, B, D, 1.0f / (ntok - first), out);
+  launch_pdl(mean_pool_partial_kernel, dim3((D + 255) / 256, kPoolSplits, B), dim3(256), 0, st, 1, y, ntok, D, first,
+             partial);
+  launch_pdl(mean_pool_final_kernel, dim3((B * D + 255) / 256), dim3(256), 0, st, 1, static_cast<const float*>(partial),
+             B, D, 1.0f / (ntok - first), out);
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 
@@ -154,6 +164,8 @@ int launch_mean_pool(const float* y, int B, int ntok, int D, int first, float* p
 // qs [N, K] int8 or [N, K/2] nibble bytes (block order kept) + scales [N, K/32].
 __global__ void repack_kernel(int bmode, const uint8_t* __restrict__ blocks, long long nblocks, uint8_t* qs,
                               uint16_t* scales) {
+  pdl_wait();
+  pdl_trigger();
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= nblocks) return;
   const int bsz = bmode == B_Q8 ? 34 : 18;
