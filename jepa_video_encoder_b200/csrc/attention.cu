@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   // per query tile g: S ready / S taken / P written / PV done
   __shared__ uint64_t s_full[2], s_free[2], p_full[2], pv_done[2], drain_bar[2];
+  __shared__ uint64_t stagger_bar;  // one phase: query tile 0 has computed its first P (cross-warp layout)
   // cross-warp row layout only: both halves of every row posted their partial
   __shared__ uint64_t x_bar[2];
   __shared__ float xmax[2][2][2][128];  // [tile parity][g][column half][row]: partial row maxima
@@ -149,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&drain_bar[g], 1);
       mbar_init(&x_bar[g], 256);
     }
+    mbar_init(&stagger_bar, 256);
     abort_sh = 0;
     mbar_fence_init();
   }
@@ -293,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.scale_log2;
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.0f, l_b = 0.0f;  // l: this thread's share of the row sum
     bool ok = true;
-    for (int j = 0; j < n_my; ++j) {
+    for (int j = 0; ok && j < n_my; ++j) {
       bool okw = mbar_wait(&s_full[g], j & 1, w);
       okw = __all_sync(0xffffffffu, okw);
       if (!okw) {
@@ -457,7 +459,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
-    for (int j = 0; j < n_my; ++j) {
+    // Stagger: query tile 1 starts once tile 0 has its first P, so that one
+    // tile's exponentials overlap the other's TMEM traffic and row-max
+    // exchange (these bidirectional tiles are long; the block-causal layout
+    // above is faster without it).
+    if (g == 1 && nkv0 > 0 && n_my > 0) {
+      bool okw = mbar_wait(&stagger_bar, 0, w);
+      ok = __all_sync(0xffffffffu, okw);
+    }
+    for (int j = 0; ok && j < n_my; ++j) {
       bool okw = mbar_wait(&s_full[g], j & 1, w);
       okw = __all_sync(0xffffffffu, okw);
       if (!okw) {
@@ -524,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         lsv2[e & 3] = f2_add(lsv2[e & 3], f2_pack(pa, pb));
         pk[e] = pack_half2(pa, pb);
       }
+      if (j == 0 && g == 0) mbar_arrive(&stagger_bar);
       if (j > 0) {  // P_g free and O_g stable once the PV product of tile j-1 is done
         okw = mbar_wait(&pv_done[g], (j - 1) & 1, w);
         okw = __all_sync(0xffffffffu, okw);
