@@ -15,10 +15,13 @@
 // frame's: as the second tile of the last pair when the tile count is odd
 // (that pair has no second tile of its own), else in a CTA of its own.
 //
-// One CTA per (pair of 128-query tiles, clip*head), one CTA per SM:
-//   warp 0      TMA: both Q tiles once, then K and V^T tiles through a
-//               4-stage ring shared by the two query tiles;
-//   warps 1,18  MMA, one issuer per query tile g: for each KV tile j,
+// Bidirectional: one CTA per (pair of 128-query tiles, clip*head), one CTA
+// per SM.  Block-causal: one CTA per (128-query tile, clip*head), two CTAs
+// per SM (half the TMEM and shared memory each), so that the start and the
+// drain of one CTA's short tile overlap the other CTA's work.
+//   warp 0      TMA: the Q tile(s) once, then K and V^T tiles through a
+//               ring (4 stages shared by the two query tiles, or 2);
+//   warps 1,18  MMA, one issuer per query tile g (warp 18 with two tiles): for each KV tile j,
 //               S_g = Q_g K_j^T into TMEM (M=128, N=128, both operands in
 //               shared memory) and O_g += P_g V_{j-1} into TMEM (M=128, N=64,
 //               P read from TMEM);
@@ -46,15 +49,22 @@ namespace jb {
 
 namespace {
 constexpr int kTile = 128 * 64 * 2;  // one [128 x 64] f16 tile, 16 KB
-constexpr int kStages = 4;
-constexpr int kOffQ = 0;                        // Q0, Q1
-constexpr int kOffK = kOffQ + 2 * kTile;        // K ring
-constexpr int kOffV = kOffK + kStages * kTile;  // V^T ring, each [64 dims x 128 keys] as two [64 x 64]
-constexpr int kAttnSmem = kOffV + kStages * kTile + 1024;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O when the row max grew by more than 2^8
-// TMEM columns: S_g (f32, 128 keys), O_g (f32, 64 dims), P_g (f16 pairs, 128 keys)
-constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
-constexpr int kThreads = 19 * 32;  // producer, 2 MMA issuers, 2 x 8 softmax warps
+// Query tiles per CTA: 2 (one CTA per SM, K / V shared by the two tiles) or 1
+// (two CTAs per SM, so one CTA's start and drain overlap the other's work).
+template <int TILES>
+struct AttnCfg {
+  static constexpr int kStages = TILES == 2 ? 4 : 2;
+  static constexpr int kOffQ = 0;                        // Q tiles
+  static constexpr int kOffK = kOffQ + TILES * kTile;    // K ring
+  static constexpr int kOffV = kOffK + kStages * kTile;  // V^T ring, each [64 dims x 128 keys] as two [64 x 64]
+  static constexpr int kSmem = kOffV + kStages * kTile + 1024;
+  // TMEM columns: S_g (f32, 128 keys), O_g (f32, 64 dims), P_g (f16 pairs, 128 keys)
+  static constexpr uint32_t kColS = 0, kColO = 128 * TILES, kColP = 192 * TILES;
+  static constexpr uint32_t kTmemCols = 256 * TILES;
+  // producer, one MMA issuer per tile, 8 softmax warps per tile
+  static constexpr int kThreads = (TILES == 2 ? 19 : 10) * 32;
+};
 }  // namespace
 
 __device__ __forceinline__ void key_range(const AttnParams& p, int i, int& lo, int& hi) {
@@ -94,10 +104,12 @@ __device__ __forceinline__ void row_keys(const AttnParams& p, bool cls_tile, int
   }
 }
 
-template <bool ROWS_IN_WARP>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool ROWS_IN_WARP, int TILES>
+__global__ void __launch_bounds__(AttnCfg<TILES>::kThreads, TILES == 2 ? 1 : 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using C = AttnCfg<TILES>;
+  constexpr int kStages = C::kStages;
   extern __shared__ uint8_t dsmem[];
   __shared__ uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   // per query tile g: S ready / S taken / P written / PV done
@@ -116,31 +128,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_pairs = (p.n_q_tiles + 1) / 2;
   // Grid: (unit, clip*head), or (clip*head, unit) under the block-causal mask
-  // so that the hardware starts the heaviest units of every head first.  With
-  // a separate CLS row, unit 0 computes the CLS row alone (query tile 0
-  // against every KV tile); the pair units follow, later (heavier) tiles first.
+  // so that the hardware starts the heaviest units of every head first.  A
+  // unit is a pair of query tiles (TILES == 2) or one query tile, later
+  // (heavier) tiles first.
   const int unit = p.mask == JEPA_B200_MASK_BLOCK_CAUSAL ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
   const int bh = p.mask == JEPA_B200_MASK_BLOCK_CAUSAL ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.y);
   // The CLS tile (query rows 0..127 against every key, only row 0 kept) is
-  // either the second tile of the last pair, whose own second tile does not
-  // exist when the tile count is odd, or the one tile of unit 0.
-  const int cls_unit = p.cls_separate && !p.cls_in_pair;
+  // the second tile of the last pair when the tile count is odd (that pair
+  // has no second tile of its own), else the one tile of unit 0.
+  const int cls_unit = p.cls_separate && !(TILES == 2 && p.cls_in_pair);
   const bool cls_cta = cls_unit && unit == 0;
-  const int pair = n_pairs - 1 - (unit - cls_unit);
-  const int cls_g = cls_cta ? 0 : ((p.cls_in_pair && pair == n_pairs - 1) ? 1 : -1);  // query tile g holding CLS
-  const int q00 = cls_cta ? 0 : 2 * pair * 128;  // first rows of query tiles 0 and 1
-  const int q01 = cls_g == 1 ? 0 : q00 + 128;
-  const int nkv0 = cls_cta ? (p.N + 127) / 128 : kv_tiles(p, q00);
-  const int nkv1 = cls_cta ? 0 : (cls_g == 1 ? (p.N + 127) / 128 : kv_tiles(p, q01));
+  int q00, q01 = 0, nkv0, nkv1 = 0, cls_g = cls_cta ? 0 : -1;  // cls_g: query tile g holding CLS
+  if (TILES == 2) {
+    const int pair = n_pairs - 1 - (unit - cls_unit);
+    if (!cls_cta && p.cls_in_pair && pair == n_pairs - 1) cls_g = 1;
+    q00 = cls_cta ? 0 : 2 * pair * 128;  // first rows of query tiles 0 and 1
+    q01 = cls_g == 1 ? 0 : q00 + 128;
+    nkv0 = cls_cta ? (p.N + 127) / 128 : kv_tiles(p, q00);
+    nkv1 = cls_cta ? 0 : (cls_g == 1 ? (p.N + 127) / 128 : kv_tiles(p, q01));
+  } else {
+    q00 = cls_cta ? 0 : (p.n_q_tiles - 1 - (unit - cls_unit)) * 128;
+    nkv0 = cls_cta ? (p.N + 127) / 128 : kv_tiles(p, q00);
+  }
   const int nkv_all = max(nkv0, nkv1);
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 2);
+      mbar_init(&k_empty[s], TILES);  // one release per MMA issuer
       mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 2);
+      mbar_init(&v_empty[s], TILES);
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(&s_full[g], 1);
@@ -155,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_fence_init();
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_sh, 512);
+    tmem_alloc(&tmem_sh, C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -176,8 +194,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       uint32_t karmed = 0, kpar = 0, varmed = 0, vpar = 0;
       mbar_expect_tx(&q_full, nkv1 > 0 ? 2 * kTile : kTile);
-      tma_load_3d(sm + kOffQ, &tmQ, &q_full, 0, q00, bh);
-      if (nkv1 > 0) tma_load_3d(sm + kOffQ + kTile, &tmQ, &q_full, 0, q01, bh);
+      tma_load_3d(sm + C::kOffQ, &tmQ, &q_full, 0, q00, bh);
+      if (nkv1 > 0) tma_load_3d(sm + C::kOffQ + kTile, &tmQ, &q_full, 0, q01, bh);
       for (int j = 0; j < nkv_all; ++j) {
         const int s = j % kStages;
         const uint32_t ph = (j / kStages) & 1;
@@ -186,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         mbar_expect_tx(&k_full[s], kTile);
-        tma_load_3d(sm + kOffK + s * kTile, &tmK, &k_full[s], 0, j * 128, bh);
+        tma_load_3d(sm + C::kOffK + s * kTile, &tmK, &k_full[s], 0, j * 128, bh);
         karmed |= 1u << s;
         kpar = (kpar & ~(1u << s)) | (ph << s);
         if (!mbar_wait(&v_empty[s], ph ^ 1, w)) {
@@ -194,8 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         mbar_expect_tx(&v_full[s], kTile);
-        tma_load_3d(sm + kOffV + s * kTile, &tmV, &v_full[s], j * 128, 0, bh);
-        tma_load_3d(sm + kOffV + s * kTile + kTile / 2, &tmV, &v_full[s], j * 128 + 64, 0, bh);
+        tma_load_3d(sm + C::kOffV + s * kTile, &tmV, &v_full[s], j * 128, 0, bh);
+        tma_load_3d(sm + C::kOffV + s * kTile + kTile / 2, &tmV, &v_full[s], j * 128 + 64, 0, bh);
         varmed |= 1u << s;
         vpar = (vpar & ~(1u << s)) | (ph << s);
       }
@@ -207,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1 || warp == 18) {
+  } else if (warp == 1 || (TILES == 2 && warp == 18)) {
     // one MMA issuer per query tile, so each tile's S / PV products follow
     // its own softmax without waiting on the other tile's
     if (lane == 0) {
@@ -215,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nkv_g = g == 0 ? nkv0 : nkv1;
       constexpr uint32_t idesc_s = idesc_f16_f32(128, 128);
       constexpr uint32_t idesc_o = idesc_f16_f32(128, 64);
-      const uint64_t qd = sdesc_kmajor_sw128(smem_u32(sm + kOffQ + g * kTile));
+      const uint64_t qd = sdesc_kmajor_sw128(smem_u32(sm + C::kOffQ + g * kTile));
       bool ok = mbar_wait(&q_full, 0, w);
       // Every issuer waits for each K / V tile to land and then arrives on
       // its release barrier (count 2), also for tiles it does not use: a
@@ -233,10 +251,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            const uint64_t kd = sdesc_kmajor_sw128(smem_u32(sm + kOffK + ks * kTile));
+            const uint64_t kd = sdesc_kmajor_sw128(smem_u32(sm + C::kOffK + ks * kTile));
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              tc_mma_f16_ss(tmem + kColS + 128 * g, qd + static_cast<uint64_t>(2 * k),
+              tc_mma_f16_ss(tmem + C::kColS + 128 * g, qd + static_cast<uint64_t>(2 * k),
                             kd + static_cast<uint64_t>(2 * k), idesc_s, k > 0 ? 1u : 0u);
             tc_commit(&s_full[g]);
           }
@@ -254,11 +272,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t vb = smem_u32(sm + kOffV + vs * kTile);
+            const uint32_t vb = smem_u32(sm + C::kOffV + vs * kTile);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               const uint64_t bd = sdesc_kmajor_sw128(vb + (k >> 2) * (kTile / 2)) + static_cast<uint64_t>(2 * (k & 3));
-              tc_mma_f16_ts(tmem + kColO + 64 * g, tmem + kColP + 64 * g + 8 * k, bd, idesc_o,
+              tc_mma_f16_ts(tmem + C::kColO + 64 * g, tmem + C::kColP + 64 * g + 8 * k, bd, idesc_o,
                             (j > 1 || k > 0) ? 1u : 0u);
             }
             tc_commit(&pv_done[g]);
@@ -285,9 +303,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ia = q0 + ra, ib = ia + 8;
     const int n_my = g == 0 ? nkv0 : nkv1;
     const uint32_t lane_off = static_cast<uint32_t>(lane_base) << 16;
-    const uint32_t tS = tmem + kColS + 128 * g + lane_off;
-    const uint32_t tO = tmem + kColO + 64 * g + lane_off;
-    const uint32_t tP = tmem + kColP + 64 * g + lane_off;
+    const uint32_t tS = tmem + C::kColS + 128 * g + lane_off;
+    const uint32_t tO = tmem + C::kColO + 64 * g + lane_off;
+    const uint32_t tP = tmem + C::kColP + 64 * g + lane_off;
     int loa, hia, lob, hib;
     const bool cls_tile = g == cls_g;
     row_keys(p, cls_tile, ia, loa, hia);
@@ -443,9 +461,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i = (g == 0 ? q00 : q01) + r;
     const int n_my = g == 0 ? nkv0 : nkv1;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tS = tmem + kColS + 128 * g + 64 * ch + lane_off;
-    const uint32_t tO = tmem + kColO + 64 * g + 32 * ch + lane_off;
-    const uint32_t tP = tmem + kColP + 64 * g + 32 * ch + lane_off;
+    const uint32_t tS = tmem + C::kColS + 128 * g + 64 * ch + lane_off;
+    const uint32_t tO = tmem + C::kColO + 64 * g + 32 * ch + lane_off;
+    const uint32_t tP = tmem + C::kColP + 64 * g + 32 * ch + lane_off;
     int lo, hi;
     key_range(p, i, lo, hi);
     const bool cls_tile = g == cls_g;
@@ -594,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_sh, 512);
+    tmem_dealloc(tmem_sh, C::kTmemCols);
   }
 }
 
@@ -638,27 +656,33 @@ int attn_prepare(AttnOp* op, const __half* q, const __half* k, const __half* vt,
   op->vt = vt;
   op->npad = npad;
   op->B = B;
-  op->smem = kAttnSmem;
+  op->smem = AttnCfg<2>::kSmem;
   return JEPA_B200_OK;
 }
 
-template <bool ROWS_IN_WARP>
+template <bool ROWS_IN_WARP, int TILES>
 static int attn_launch_impl(const AttnParams& p, const AttnOp& op, cudaStream_t st) {
-  auto kern = attn_fwd_kernel<ROWS_IN_WARP>;
+  using C = AttnCfg<TILES>;
+  auto kern = attn_fwd_kernel<ROWS_IN_WARP, TILES>;
   static unsigned long long attr_done = 0;  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !((attr_done >> dev) & 1ull)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) != cudaSuccess)
       return JEPA_B200_ERR_CUDA;
     attr_done |= 1ull << dev;
   }
-  const int units = (p.n_q_tiles + 1) / 2 + (p.cls_separate && !p.cls_in_pair ? 1 : 0);
+  const int units = TILES == 2 ? (p.n_q_tiles + 1) / 2 + (p.cls_separate && !p.cls_in_pair ? 1 : 0)
+                               : p.n_q_tiles + p.cls_separate;
   const dim3 grid = p.mask == JEPA_B200_MASK_BLOCK_CAUSAL ? dim3(op.B * p.heads, units) : dim3(units, op.B * p.heads);
-  if (launch_pdl(kern, grid, dim3(kThreads), kAttnSmem, st, 1, op.tmQ, op.tmK, op.tmV, p) != cudaSuccess)
+  if (launch_pdl(kern, grid, dim3(C::kThreads), C::kSmem, st, 1, op.tmQ, op.tmK, op.tmV, p) != cudaSuccess)
     return JEPA_B200_ERR_CUDA;
   return JEPA_B200_OK;
 }
+
+// Query tiles per CTA under each mask.
+constexpr int kTilesBlockCausal = 1;
+constexpr int kTilesBidir = 2;
 
 int attn_launch(const AttnOp& op, cudaStream_t st, DevErr* err, unsigned long long timeout_ns) {
   AttnParams p = op.p;
@@ -668,8 +692,8 @@ int attn_launch(const AttnOp& op, cudaStream_t st, DevErr* err, unsigned long lo
   // exchange between warps is a large share: rows kept inside one warp.
   // Bidirectional tiles are long and bound by the exponentials, where the
   // cross-warp layout issues fewer instructions.
-  if (p.mask == JEPA_B200_MASK_BLOCK_CAUSAL) return attn_launch_impl<true>(p, op, st);
-  return attn_launch_impl<false>(p, op, st);
+  if (p.mask == JEPA_B200_MASK_BLOCK_CAUSAL) return attn_launch_impl<true, kTilesBlockCausal>(p, op, st);
+  return attn_launch_impl<false, kTilesBidir>(p, op, st);
 }
 
 }  // namespace jb
