@@ -680,9 +680,11 @@ static int attn_launch_impl(const AttnParams& p, const AttnOp& op, cudaStream_t 
   return JEPA_B200_OK;
 }
 
-// Query tiles per CTA under each mask.
+// Query tiles per CTA and row layout under each mask.
 constexpr int kTilesBlockCausal = 1;
 constexpr int kTilesBidir = 2;
+constexpr bool kRowsInWarpBlockCausal = true;
+constexpr bool kRowsInWarpBidir = false;
 
 int attn_launch(const AttnOp& op, cudaStream_t st, DevErr* err, unsigned long long timeout_ns) {
   AttnParams p = op.p;
@@ -692,8 +694,8 @@ int attn_launch(const AttnOp& op, cudaStream_t st, DevErr* err, unsigned long lo
   // exchange between warps is a large share: rows kept inside one warp.
   // Bidirectional tiles are long and bound by the exponentials, where the
   // cross-warp layout issues fewer instructions.
-  if (p.mask == JEPA_B200_MASK_BLOCK_CAUSAL) return attn_launch_impl<true, kTilesBlockCausal>(p, op, st);
-  return attn_launch_impl<false, kTilesBidir>(p, op, st);
+  if (p.mask == JEPA_B200_MASK_BLOCK_CAUSAL) return attn_launch_impl<kRowsInWarpBlockCausal, kTilesBlockCausal>(p, op, st);
+  return attn_launch_impl<kRowsInWarpBidir, kTilesBidir>(p, op, st);
 }
 
 }  // namespace jb
