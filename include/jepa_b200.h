@@ -116,7 +116,11 @@ typedef struct jepa_b200_model jepa_b200_model;
  * ffn_up,ffn_down}.{weight,bias}, head.xattn.ln2.*, head.cls.{weight,bias}.
  * q8_0 / q4_0 are accepted only for the matrices that page re-types and only
  * when the input dimension is a multiple of 64.  f32 matrices are rounded to
- * f16 once here; 1-D tensors and pos_embed are kept in f32.
+ * f16 once here; 1-D tensors and pos_embed are kept in f32.  A q8_0 / q4_0
+ * matrix is kept as its blocks (unpacked in the GEMM's loader and by the
+ * head's few-row kernels) and also dequantised once, on the device, to f16
+ * (each q*d or (q-8)*d rounded once: the values the loader unpack produces),
+ * which the GEMMs with 256 or more rows use.
  * On success *out_model owns its device memory until jepa_b200_free.
  * Errors: ERR_ARG, ERR_MISSING_TENSOR, ERR_SHAPE, ERR_DTYPE, ERR_CUDA. */
 JEPA_B200_API int jepa_b200_load_weights(const jepa_b200_config *cfg, const jepa_b200_tensor *table, int n_tensors, int device,
@@ -163,7 +167,8 @@ JEPA_B200_API int jepa_b200_sync_status(jepa_b200_model *m, void *stream);
  * that encode finished.  Returns a negative value if there is none. */
 JEPA_B200_API double jepa_b200_last_ms(jepa_b200_model *m);
 
-/* Bytes of weights resident on the device after the load (repacked form). */
+/* Bytes of weights resident on the device after the load (repacked blocks
+ * plus, for quantised matrices, their f16 copies). */
 JEPA_B200_API size_t jepa_b200_model_n_bytes(const jepa_b200_model *m);
 
 /* Bound, in nanoseconds, of every device-side wait of the model's kernels
@@ -220,6 +225,15 @@ JEPA_B200_API int jepa_b200_op_layernorm(const float *x, int rows, int D, int in
  * qs = int8 [N, K] (q8_0) or nibble bytes [N, K/2] in block order (q4_0),
  * scales = fp16 [N, K/32].  Byte moves only (bit-exact).  K % 32 == 0. */
 JEPA_B200_API int jepa_b200_op_repack(int dtype, const void *blocks, int N, int K, void *qs, void *scales, void *stream);
+
+/* f16 [N, K] from repacked quants and scales (the layout jepa_b200_op_repack
+ * writes): element (n, k) = q * d (q8_0) or (q - 8) * d (q4_0), d the fp16
+ * scale of its 32-element block, the exact product rounded once to f16 --
+ * the values the GEMM's loader unpack produces, made once for GEMMs with many
+ * rows ("Quantization" page, "The rule": the dequantisation formula).
+ * K % 32 == 0; out 16-byte aligned.  Errors: ERR_ARG, ERR_DTYPE, ERR_SHAPE. */
+JEPA_B200_API int jepa_b200_op_dequant_f16(int dtype, const void *qs, const void *scales, int N, int K, void *out,
+                                           void *stream);
 
 /* Epilogues of jepa_b200_op_linear. */
 typedef enum {

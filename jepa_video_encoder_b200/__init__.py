@@ -170,6 +170,12 @@ def repack(dtype: int, blocks, N: int, K: int, qs, scales, stream=None):
                                              _stream_ptr(stream)), "repack")
 
 
+def dequant_f16(dtype: int, qs, scales, N: int, K: int, out, stream=None):
+    check(load_library().jepa_b200_op_dequant_f16(dtype, _ptr(qs), _ptr(scales), N, K, _ptr(out),
+                                                  _stream_ptr(stream)), "dequant_f16")
+    return out
+
+
 def linear(A, w, w_dtype: int, N: int, bias, epilogue: int, out, w_scales=None, stream=None):
     M, K = A.shape
     check(load_library().jepa_b200_op_linear(_ptr(A), M, K, _ptr(w), _ptr(w_scales) if w_scales is not None else None,

@@ -46,6 +46,7 @@ SIGNATURES = {
     "jepa_b200_op_layernorm": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_float, c_void_p,
                                        c_int, c_void_p]),
     "jepa_b200_op_repack": (c_int, [c_int, c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+    "jepa_b200_op_dequant_f16": (c_int, [c_int, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
     "jepa_b200_op_linear": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_int, c_void_p, c_int,
                                     c_void_p, c_int, c_void_p]),
     "jepa_b200_op_linear_qkv": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_int, c_void_p, c_int,

@@ -982,8 +982,17 @@ int num_sms() {
   return n;
 }
 
-int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& W, const float* bias, int epi,
+int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& Win, const float* bias, int epi,
                  void* out, int ldo, const QkvDst* qkv, const PatchSrc* patch) {
+  // A quantised matrix with a dequantised f16 copy runs as f16 once there
+  // are at least 256 rows: unpacking a 256 x 64 weight tile per 128 x 256 x
+  // 64 product in the loader costs more issue slots than the MMA takes.
+  DevMatrix W = Win;
+  if (W.bmode != B_F16 && W.f16 && !patch && M >= 256) {
+    W.bmode = B_F16;
+    W.data = W.f16;
+    W.scales = nullptr;
+  }
   if (!op || !out || M < 1 || K < 64 || K % 64 != 0 || W.K != K || W.N < 1 || !W.data) return JEPA_B200_ERR_SHAPE;
   if (!patch && !A) return JEPA_B200_ERR_ARG;
   const int N = W.N;

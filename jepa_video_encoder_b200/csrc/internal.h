@@ -23,6 +23,11 @@ struct DevMatrix {
   int N = 0, K = 0;   // K: row length as stored (f16: padded to 64 with zeros)
   void* data = nullptr;       // f16 [N, K] | int8 [N, K] | nibble bytes [N, K/2]
   __half* scales = nullptr;   // fp16 [N, K/32] for quantised matrices
+  // quantised matrices: the same values dequantised once to f16 [N, K] (each
+  // q * d or (q - 8) * d rounded once, as the in-loader unpack rounds them),
+  // used by GEMMs with M >= 256 rows, where the unpack in the loader cannot
+  // keep pace with the tensor cores; null where absent
+  __half* f16 = nullptr;
 };
 
 // Destination of the QKV scatter epilogue.
@@ -110,6 +115,8 @@ int launch_mean_pool(const float* y, int B, int ntok, int D, int first, float* p
                      cudaStream_t st);
 int mean_pool_partial_floats(int B, int D);
 int launch_repack(int bmode, const uint8_t* blocks, int N, int K, void* qs, __half* scales, cudaStream_t st);
+// f16 [N, K] from repacked q8_0 / q4_0 quants and scales (DevMatrix::f16).
+int launch_dequant_f16(int bmode, const void* qs, const __half* scales, int N, int K, __half* out, cudaStream_t st);
 int launch_gemv(const float* x, int M, int K, const DevMatrix& W, const float* bias, int epi, const float* resid,
                 long long resid_stride, float* y, cudaStream_t st);
 int launch_xattn_1q(const float* q, const __half* k, const __half* vt, int B, int heads, int ntok, int npad,

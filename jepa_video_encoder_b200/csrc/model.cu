@@ -253,6 +253,7 @@ struct Loader {
       M.bmode = dt == JEPA_B200_Q8_0 ? B_Q8 : (dt == JEPA_B200_Q4_0 ? B_Q4 : B_F16);
       M.data = dalloc(1);
       M.scales = quant ? static_cast<__half*>(dalloc(1)) : nullptr;
+      M.f16 = quant ? static_cast<__half*>(dalloc(1)) : nullptr;
       return M;
     }
     if (dt == JEPA_B200_F32 || dt == JEPA_B200_F16) {
@@ -292,6 +293,11 @@ struct Loader {
     M.scales = static_cast<__half*>(dalloc(sc.size() * 2));
     if (M.data) upload(M.data, qs.data(), qs.size());
     if (M.scales) upload(M.scales, sc.data(), sc.size() * 2);
+    // the dequantised f16 copy for the large-M GEMMs, made on the device
+    M.f16 = static_cast<__half*>(dalloc(static_cast<size_t>(N * K) * 2));
+    if (M.f16 && status == JEPA_B200_OK &&
+        launch_dequant_f16(M.bmode, M.data, M.scales, M.N, M.K, M.f16, nullptr) != JEPA_B200_OK)
+      status = JEPA_B200_ERR_CUDA;
     return M;
   }
   DevMatrix mat(const std::string& name, int64_t N, int64_t K) {
@@ -645,6 +651,7 @@ int jepa_b200_load_weights(const jepa_b200_config* cfg, const jepa_b200_tensor* 
   L.m = m;
   for (int i = 0; i < n_tensors; ++i) L.tab[table[i].name] = &table[i];
   load_sequence(L);
+  if (L.status == JEPA_B200_OK && cudaDeviceSynchronize() != cudaSuccess) L.status = JEPA_B200_ERR_CUDA;
   if (L.status == JEPA_B200_OK) {
     if (cudaMalloc(&m->err, sizeof(DevErr)) != cudaSuccess || cudaMemset(m->err, 0, sizeof(DevErr)) != cudaSuccess ||
         cudaEventCreate(&m->ev0) != cudaSuccess || cudaEventCreate(&m->ev1) != cudaSuccess)

@@ -185,4 +185,47 @@ int launch_repack(int bmode, const uint8_t* blocks, int N, int K, void* qs, __ha
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 
+// f16 copy of a repacked matrix: element (n, k) = q * d (q8_0) or (q - 8) * d
+// (q4_0), d the scale of its 32-element block; the product is exact in f32
+// (an 8-bit integer times an 11-bit significand) and rounded once to f16.
+// One thread writes 8 consecutive elements of one block.
+__global__ void dequant_f16_kernel(int bmode, const uint8_t* __restrict__ qs, const uint16_t* __restrict__ scales,
+                                   long long n_units, int K, __half* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
+  const long long u = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (u >= n_units) return;
+  const long long e0 = u * 8;  // first element, row-major [N, K]
+  const long long n = e0 / K;
+  const int k = static_cast<int>(e0 - n * K);
+  const float d = __half2float(__ushort_as_half(scales[n * (K / 32) + k / 32]));
+  float v[8];
+  if (bmode == B_Q8) {
+    const int8_t* q = reinterpret_cast<const int8_t*>(qs) + e0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = static_cast<float>(q[i]) * d;
+  } else {
+    const int j0 = k & 31;  // byte j of a block holds elements j (low nibble) and j + 16 (high)
+    const uint8_t* q = qs + n * (K / 2) + (k / 32) * 16 + (j0 & 15);
+    const int sh = j0 >= 16 ? 4 : 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = static_cast<float>(static_cast<int>((q[i] >> sh) & 0xF) - 8) * d;
+  }
+  uint4 w;
+  w.x = pack_half2(v[0], v[1]);
+  w.y = pack_half2(v[2], v[3]);
+  w.z = pack_half2(v[4], v[5]);
+  w.w = pack_half2(v[6], v[7]);
+  *reinterpret_cast<uint4*>(out + e0) = w;
+}
+
+int launch_dequant_f16(int bmode, const void* qs, const __half* scales, int N, int K, __half* out, cudaStream_t st) {
+  if (!qs || !scales || !out) return JEPA_B200_ERR_ARG;
+  if ((bmode != B_Q8 && bmode != B_Q4) || N < 1 || K < 32 || K % 32 != 0) return JEPA_B200_ERR_SHAPE;
+  const long long units = static_cast<long long>(N) * K / 8;
+  launch_pdl(dequant_f16_kernel, dim3(static_cast<unsigned>((units + 255) / 256)), dim3(256), 0, st, 1, bmode,
+             static_cast<const uint8_t*>(qs), reinterpret_cast<const uint16_t*>(scales), units, K, out);
+  return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+}
+
 }  // namespace jb

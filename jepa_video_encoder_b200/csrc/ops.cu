@@ -90,6 +90,14 @@ int jepa_b200_op_repack(int dtype, const void* blocks, int N, int K, void* qs, v
                        static_cast<cudaStream_t>(stream));
 }
 
+int jepa_b200_op_dequant_f16(int dtype, const void* qs, const void* scales, int N, int K, void* out, void* stream) {
+  const int bm = bmode_of(dtype);
+  if (bm != B_Q8 && bm != B_Q4) return JEPA_B200_ERR_DTYPE;
+  if (!qs || !scales || !out || !aligned16(out)) return JEPA_B200_ERR_ARG;
+  return launch_dequant_f16(bm, qs, static_cast<const __half*>(scales), N, K, static_cast<__half*>(out),
+                            static_cast<cudaStream_t>(stream));
+}
+
 int jepa_b200_op_linear(const void* A, int M, int K, const void* w, const void* w_scales, int w_dtype, int N,
                         const float* bias, int epilogue, void* out, int ldo, void* stream) {
   if (!A || !out) return JEPA_B200_ERR_ARG;

@@ -146,6 +146,20 @@ def test_quant_unpack_bit_exact(wdt):
 
 
 @pytest.mark.parametrize("wdt", ["q8_0", "q4_0"])
+def test_dequant_f16_bit_exact(wdt):
+    """The f16 copy the large-M GEMMs use holds binary16(q*d) / binary16((q-8)*d)
+    of the oracle's dequantisation, bit for bit, over all codes."""
+    need_cuda()
+    N, K = 384, 512
+    dt, blocks, deq, qs, sc = _quant_weight(wdt, N, K, 13)
+    out = torch.empty((N, K), dtype=torch.float16, device="cuda")
+    jb.dequant_f16(dt, qs, sc, N, K, out)
+    _ok()
+    want = deq.astype(np.float16)  # one rounding of the exact product (q*d is exact in float64)
+    assert np.array_equal(out.cpu().numpy().view(np.uint16), want.view(np.uint16))
+
+
+@pytest.mark.parametrize("wdt", ["q8_0", "q4_0"])
 @pytest.mark.parametrize("M,K,N", [(300, 1024, 768), (1000, 4096, 1024)])
 def test_linear_quant(wdt, M, K, N):
     need_cuda()
