@@ -171,6 +171,14 @@ JEPA_B200_API double jepa_b200_last_ms(jepa_b200_model *m);
  * plus, for quantised matrices, their f16 copies). */
 JEPA_B200_API size_t jepa_b200_model_n_bytes(const jepa_b200_model *m);
 
+/* Replay the forward as a CUDA graph (default on): when two consecutive
+ * encodes have the same (pixels, out, B, pool, wait bound), the second
+ * captures its kernel sequence on a stream of the model's own and it and
+ * later calls with those inputs launch that graph on `stream`.  Other calls,
+ * and every call while this is off or profiling is on, launch the kernels
+ * one by one.  Errors: ERR_ARG. */
+JEPA_B200_API int jepa_b200_set_graph(jepa_b200_model *m, int enable);
+
 /* Bound, in nanoseconds, of every device-side wait of the model's kernels
  * (default 4e9).  0 makes the first wait that does not succeed at once give
  * up: used to test the timeout path.  Returns OK or ERR_ARG. */

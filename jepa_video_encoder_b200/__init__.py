@@ -83,6 +83,10 @@ class Model:
     def set_timeout_ns(self, ns: int) -> None:
         check(load_library().jepa_b200_set_timeout_ns(self._h, ns), "set_timeout_ns")
 
+    def set_graph(self, enable: bool) -> None:
+        """Replay repeated forwards as a CUDA graph (default on)."""
+        check(load_library().jepa_b200_set_graph(self._h, 1 if enable else 0), "set_graph")
+
     def set_profiling(self, enable: bool) -> None:
         check(load_library().jepa_b200_set_profiling(self._h, 1 if enable else 0), "set_profiling")
 

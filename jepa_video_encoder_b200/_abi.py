@@ -38,6 +38,7 @@ SIGNATURES = {
     "jepa_b200_last_ms": (c_double, [c_void_p]),
     "jepa_b200_model_n_bytes": (c_size_t, [c_void_p]),
     "jepa_b200_set_timeout_ns": (c_int, [c_void_p, c_ulonglong]),
+    "jepa_b200_set_graph": (c_int, [c_void_p, c_int]),
     "jepa_b200_last_launch_count": (c_int, [c_void_p]),
     "jepa_b200_set_profiling": (c_int, [c_void_p, c_int]),
     "jepa_b200_profile_read": (c_int, [c_void_p, POINTER(c_double), POINTER(c_int), c_int]),

@@ -47,6 +47,17 @@ struct DeviceGuard {
   }
 };
 
+// The inputs a captured forward is bound to.
+struct EncodeKey {
+  const float* pixels = nullptr;
+  const float* out = nullptr;
+  int B = 0, pool = -1;
+  unsigned long long timeout_ns = 0;
+  bool operator==(const EncodeKey& o) const {
+    return pixels == o.pixels && out == o.out && B == o.B && pool == o.pool && timeout_ns == o.timeout_ns;
+  }
+};
+
 }  // namespace
 
 struct jepa_b200_model {
@@ -66,7 +77,8 @@ struct jepa_b200_model {
   size_t weight_bytes = 0;
 
   // workspace for the largest B seen
-  int ws_B = 0;
+  int ws_B = 0;   // clips the workspace holds
+  int ops_B = 0;  // clips the prepared ops process
   float* X = nullptr;
   __half *Y = nullptr, *Q = nullptr, *Kb = nullptr, *Vt = nullptr, *O = nullptr, *H = nullptr;
   float *Yf = nullptr, *partial = nullptr;
@@ -86,6 +98,14 @@ struct jepa_b200_model {
   bool have_timing = false;
   unsigned long long timeout_ns = kDefaultTimeoutNs;
   int launches = 0;
+
+  // CUDA graph of the last forward, replayed while its inputs (pointers, B,
+  // pool, wait bound) are unchanged; captured on a stream of the model's own
+  bool use_graph = true;
+  cudaStream_t cap_stream = nullptr;
+  cudaGraphExec_t graph = nullptr;
+  EncodeKey g_key, last_key;  // inputs of the captured graph; of the previous encode
+  int g_launches = 0;
 
   // per-kernel timing (jepa_b200_set_profiling)
   bool prof = false;
@@ -367,11 +387,37 @@ int prepare_block_ops(jepa_b200_model* m, const LayerW& L, BlockOps& ops, float*
   return JEPA_B200_OK;
 }
 
+// Workspace buffers for B clips; every launch's parameters (row counts,
+// tensor maps) for B clips.
+int alloc_workspace(jepa_b200_model* m, int B);
+int prepare_ops(jepa_b200_model* m, int B);
+
+// Workspace for at least B clips (grown, never shrunk) and the ops for
+// exactly B clips (rebuilt whenever B changes).
 int ensure_workspace(jepa_b200_model* m, int B) {
-  if (B <= m->ws_B) return JEPA_B200_OK;
-  cudaDeviceSynchronize();
-  free_list(m->ws_allocs);
-  m->ws_B = 0;
+  int s = JEPA_B200_OK;
+  if (B > m->ws_B) {
+    cudaDeviceSynchronize();
+    if (m->graph) {  // it points into the workspace about to be freed
+      cudaGraphExecDestroy(m->graph);
+      m->graph = nullptr;
+    }
+    m->g_key = EncodeKey();
+    free_list(m->ws_allocs);
+    m->ws_B = 0;
+    m->ops_B = 0;
+    if ((s = alloc_workspace(m, B))) return s;
+    m->ws_B = B;
+  }
+  if (B != m->ops_B) {
+    m->ops_B = 0;
+    if ((s = prepare_ops(m, B))) return s;
+    m->ops_B = B;
+  }
+  return JEPA_B200_OK;
+}
+
+int alloc_workspace(jepa_b200_model* m, int B) {
   const jepa_b200_config& c = m->cfg;
   const size_t R = static_cast<size_t>(B) * m->N;
   const size_t D = c.dim;
@@ -397,6 +443,13 @@ int ensure_workspace(jepa_b200_model* m, int B) {
   }
   // V^T columns past the last token stay zero: the attention multiplies them by p = 0
   if (cudaMemset(m->Vt, 0, vt_bytes) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+  return JEPA_B200_OK;
+}
+
+int prepare_ops(jepa_b200_model* m, int B) {
+  const jepa_b200_config& c = m->cfg;
+  const size_t R = static_cast<size_t>(B) * m->N;
+  int s = JEPA_B200_OK;
   const int Ri = static_cast<int>(R);
   m->enc_ops.assign(m->enc.size(), BlockOps());
   for (size_t l = 0; l < m->enc.size(); ++l)
@@ -438,7 +491,39 @@ int ensure_workspace(jepa_b200_model* m, int B) {
     if ((s = gemm_prepare(&m->kv_op, m->Y, Ri, c.dim, m->xkv, m->b_xkv, EPI_QKV, m->Kb, 2 * c.dim, &qd, nullptr)))
       return s;
   }
-  m->ws_B = B;
+  return JEPA_B200_OK;
+}
+
+// The kernel sequence of one forward on `st` (workspace and ops ready).
+int enqueue_forward(jepa_b200_model* m, const float* pixels, int B, int pool, float* out, cudaStream_t st);
+
+// Capture the forward into m->graph (replacing the previous one).
+int capture_forward(jepa_b200_model* m, const EncodeKey& key) {
+  if (m->graph) {
+    cudaGraphExecDestroy(m->graph);
+    m->graph = nullptr;
+  }
+  if (!m->cap_stream && cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess)
+    return JEPA_B200_ERR_CUDA;
+  if (cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
+    return JEPA_B200_ERR_CUDA;
+  m->launches = 0;
+  const int s = enqueue_forward(m, key.pixels, key.B, key.pool, const_cast<float*>(key.out), m->cap_stream);
+  cudaGraph_t g = nullptr;
+  const cudaError_t e = cudaStreamEndCapture(m->cap_stream, &g);
+  if (s || e != cudaSuccess) {
+    if (g) cudaGraphDestroy(g);
+    cudaGetLastError();
+    return s ? s : JEPA_B200_ERR_CUDA;
+  }
+  const cudaError_t ei = cudaGraphInstantiate(&m->graph, g, 0);
+  cudaGraphDestroy(g);
+  if (ei != cudaSuccess) {
+    m->graph = nullptr;
+    return JEPA_B200_ERR_CUDA;
+  }
+  m->g_key = key;
+  m->g_launches = m->launches;
   return JEPA_B200_OK;
 }
 
@@ -575,6 +660,30 @@ int check_encode_args(jepa_b200_model* m, const void* pixels, int B, int pool, c
   if (out_bytes < out_elems(m, B, pool) * 4) return JEPA_B200_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(pixels) & 15) || (reinterpret_cast<uintptr_t>(out) & 15)) return JEPA_B200_ERR_ARG;
   return JEPA_B200_OK;
+}
+
+int enqueue_forward(jepa_b200_model* m, const float* pixels, int B, int pool, float* out, cudaStream_t st) {
+  const jepa_b200_config& c = m->cfg;
+  const int R = B * m->N, D = c.dim;
+  int s = run_embed_and_blocks(m, pixels, B, c.depth, st);
+  if (s) return s;
+  {
+    ProfScope ps(m, JEPA_B200_KC_LAYERNORM, st);
+    if (pool == JEPA_B200_POOL_NONE)
+      s = launch_layernorm(m->X, R, D, 1, m->norm_g, m->norm_b, c.ln_eps, out, false, st);
+    else if (pool == JEPA_B200_POOL_CLS)
+      s = launch_layernorm(m->X, B, D, m->N, m->norm_g, m->norm_b, c.ln_eps, out, false, st);
+    else
+      s = launch_layernorm(m->X, R, D, 1, m->norm_g, m->norm_b, c.ln_eps, m->Yf, false, st);
+    m->launches += 1;
+  }
+  if (!s && pool == JEPA_B200_POOL_MEAN) {
+    ProfScope ps(m, JEPA_B200_KC_POOL_HEAD, st);
+    s = launch_mean_pool(m->Yf, B, m->N, D, c.has_cls ? 1 : 0, m->partial, out, st);
+    m->launches += 2;
+  }
+  if (!s && pool == JEPA_B200_POOL_ATTENTIVE) s = run_head(m, B, out, st);
+  return s;
 }
 
 }  // namespace
@@ -751,29 +860,25 @@ int jepa_b200_encode(jepa_b200_model* m, const float* pixels, int B, int pool, f
   DeviceGuard guard(m->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((s = ensure_workspace(m, B))) return s;
-  const jepa_b200_config& c = m->cfg;
-  const int R = B * m->N, D = c.dim;
-  m->launches = 0;
   m->have_timing = false;
-  if (cudaEventRecord(m->ev0, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
-  if ((s = run_embed_and_blocks(m, pixels, B, c.depth, st))) return s;
-  {
-    ProfScope ps(m, JEPA_B200_KC_LAYERNORM, st);
-    if (pool == JEPA_B200_POOL_NONE)
-      s = launch_layernorm(m->X, R, D, 1, m->norm_g, m->norm_b, c.ln_eps, out, false, st);
-    else if (pool == JEPA_B200_POOL_CLS)
-      s = launch_layernorm(m->X, B, D, m->N, m->norm_g, m->norm_b, c.ln_eps, out, false, st);
-    else
-      s = launch_layernorm(m->X, R, D, 1, m->norm_g, m->norm_b, c.ln_eps, m->Yf, false, st);
-    m->launches += 1;
+  // The graph is captured when the same inputs come twice in a row (a call
+  // with new buffers each time runs its kernels directly, capture-free), and
+  // replayed while they stay the same; per-kernel events (profiling) need
+  // the launches one by one.
+  const EncodeKey key{pixels, out, B, pool, m->timeout_ns};
+  const bool replay = m->use_graph && !m->prof && m->graph && key == m->g_key;
+  const bool capture = m->use_graph && !m->prof && !replay && key == m->last_key;
+  m->last_key = key;
+  if (!replay && !capture) {
+    m->launches = 0;
+    if (cudaEventRecord(m->ev0, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+    if ((s = enqueue_forward(m, pixels, B, pool, out, st))) return s;
+  } else {
+    if (capture && (s = capture_forward(m, key))) return s;
+    m->launches = m->g_launches;
+    if (cudaEventRecord(m->ev0, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+    if (cudaGraphLaunch(m->graph, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
   }
-  if (!s && pool == JEPA_B200_POOL_MEAN) {
-    ProfScope ps(m, JEPA_B200_KC_POOL_HEAD, st);
-    s = launch_mean_pool(m->Yf, B, m->N, D, c.has_cls ? 1 : 0, m->partial, out, st);
-    m->launches += 2;
-  }
-  if (!s && pool == JEPA_B200_POOL_ATTENTIVE) s = run_head(m, B, out, st);
-  if (s) return s;
   if (cudaEventRecord(m->ev1, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
   m->have_timing = true;
   return JEPA_B200_OK;
@@ -858,6 +963,12 @@ int jepa_b200_set_timeout_ns(jepa_b200_model* m, unsigned long long ns) {
   return JEPA_B200_OK;
 }
 
+int jepa_b200_set_graph(jepa_b200_model* m, int enable) {
+  if (!m) return JEPA_B200_ERR_ARG;
+  m->use_graph = enable != 0;
+  return JEPA_B200_OK;
+}
+
 int jepa_b200_last_launch_count(const jepa_b200_model* m) { return m ? m->launches : -1; }
 
 int jepa_b200_set_profiling(jepa_b200_model* m, int enable) {
@@ -901,6 +1012,8 @@ void jepa_b200_free(jepa_b200_model* m) {
   if (m->ev0) cudaEventDestroy(m->ev0);
   if (m->ev1) cudaEventDestroy(m->ev1);
   for (cudaEvent_t e : m->prof_events) cudaEventDestroy(e);
+  if (m->graph) cudaGraphExecDestroy(m->graph);
+  if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   delete m;
 }
 

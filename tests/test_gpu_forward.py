@@ -94,6 +94,40 @@ def test_batch_invariance_bitwise():
     m.close()
 
 
+def test_graph_replay_matches_direct_launches():
+    """The CUDA-graph replay of a forward gives the bits of the kernel-by-kernel
+    forward; a new output buffer or a smaller batch recaptures (and the ops are
+    rebuilt for the smaller batch)."""
+    need_cuda()
+    cfg = SMALL["levjepa"]
+    table = synth.make_tensor_table(cfg)
+    pix = synth.make_pixels(cfg)
+    m = jb.Model(cfg, table)
+    m.set_graph(False)
+    direct = m.encode(dev(pix), pool="none").cpu().numpy()
+    m.set_graph(True)
+    x = dev(pix)
+    out = torch.empty(m.out_shape(cfg.batch, "none"), dtype=torch.float32, device="cuda")
+    for _ in range(3):  # capture, then two replays
+        m.encode(x, pool="none", out=out)
+        assert np.array_equal(out.cpu().numpy().view(np.uint32), direct.view(np.uint32))
+    out2 = torch.empty_like(out)
+    m.encode(x, pool="none", out=out2)
+    assert np.array_equal(out2.cpu().numpy().view(np.uint32), direct.view(np.uint32))
+    one = m.encode(dev(pix[1:2]), pool="none").cpu().numpy()
+    assert np.array_equal(one[0].view(np.uint32), direct[1].view(np.uint32))
+    # a larger batch reallocates the workspace: the graph bound to the old one
+    # must not be replayed
+    pix2 = np.concatenate([pix, pix], axis=0)
+    big = m.encode(dev(pix2), pool="none").cpu().numpy()
+    assert np.array_equal(big[cfg.batch:].view(np.uint32), direct.view(np.uint32))
+    for _ in range(2):
+        m.encode(x, pool="none", out=out)
+        assert np.array_equal(out.cpu().numpy().view(np.uint32), direct.view(np.uint32))
+    assert m.sync_status() == 0
+    m.close()
+
+
 def test_block_causal_perturbation_forward_bit_identical():
     """Perturbing the pixels of frame t+1 leaves every patch token of frames
     <= t bit-identical at the encoder output (GPU path)."""
