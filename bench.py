@@ -35,6 +35,23 @@ DEFAULT_WORKLOAD = synth.LEVJEPA_VIT_L.name
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest of every rank's value (all-reduce MAX over the process
+    group); a timed region lasts as long as its slowest rank."""
+    if world <= 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step: int, world: int, steps: int, total_ms: float) -> float:
+    """Units all replicas processed per second: every rank encodes its own
+    batch each step (weak scaling), the time is the slowest rank's."""
+    return world * units_per_rank_step * steps / (total_ms / 1000.0)
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -264,14 +281,9 @@ def run_ours(args, cfg, rank, world, local_rank):
     if model.sync_status(stream) != 0:
         raise RuntimeError("device error in the timed region")
     ms_steps = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(ms_steps)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(ms_steps), world, dev)
     ms_per_step = total_ms / args.steps
-    tokens = world * cfg.batch * cfg.n_tokens * args.steps
-    value = tokens / (total_ms / 1000.0)
+    value = whole_job_rate(cfg.batch * cfg.n_tokens, world, args.steps, total_ms)
 
     # ---- per-kernel timing pass (event pairs around every launch)
     model.set_profiling(True)
@@ -298,10 +310,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         b.record(stream)
         b.synchronize()
         e2e_ms.append(a.elapsed_time(b))
-    te = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
-    e2e_value = tokens / (float(te.item()) / 1000.0)
+    e2e_value = whole_job_rate(cfg.batch * cfg.n_tokens, world, args.steps, max_over_ranks(sum(e2e_ms), world, dev))
 
     if rank != 0:
         model.close()
