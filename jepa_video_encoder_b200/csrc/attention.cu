@@ -10,10 +10,12 @@
 // so a query tile only visits KV tiles up to its largest hi (the fully masked
 // tiles past it are never loaded), and only tiles that cut an interval need
 // the per-element mask.  The CLS row, the one row that reads every key, is
-// computed apart (a "CLS tile": the query tile at row 0 against every KV
-// tile, only row 0 kept) so that query tile 0 stays as short as the first
-// frame's: as the second tile of the last pair when the tile count is odd
-// (that pair has no second tile of its own), else in a CTA of its own.
+// computed apart so that query tile 0 stays as short as the first frame's:
+// with one query tile per CTA and N % 128 != 0, its query is copied into row
+// N (the first padding row) of the last query tile, which already visits
+// every KV tile; otherwise a "CLS tile" (the query tile at row 0 against
+// every KV tile, only row 0 kept) runs as the second tile of the last pair
+// (two tiles per CTA, odd tile count) or in a CTA of its own.
 //
 // Bidirectional: one CTA per (pair of 128-query tiles, clip*head), one CTA
 // per SM.  Block-causal: one CTA per (128-query tile, clip*head), two CTAs
@@ -136,7 +138,7 @@ __global__ void __launch_bounds__(AttnCfg<TILES>::kThreads, TILES == 2 ? 1 : 2)
   // The CLS tile (query rows 0..127 against every key, only row 0 kept) is
   // the second tile of the last pair when the tile count is odd (that pair
   // has no second tile of its own), else the one tile of unit 0.
-  const int cls_unit = p.cls_separate && !(TILES == 2 && p.cls_in_pair);
+  const int cls_unit = p.cls_separate && !(TILES == 2 ? p.cls_in_pair : p.cls_tail);
   const bool cls_cta = cls_unit && unit == 0;
   int q00, q01 = 0, nkv0, nkv1 = 0, cls_g = cls_cta ? 0 : -1;  // cls_g: query tile g holding CLS
   if (TILES == 2) {
@@ -150,6 +152,9 @@ __global__ void __launch_bounds__(AttnCfg<TILES>::kThreads, TILES == 2 ? 1 : 2)
     q00 = cls_cta ? 0 : (p.n_q_tiles - 1 - (unit - cls_unit)) * 128;
     nkv0 = cls_cta ? (p.N + 127) / 128 : kv_tiles(p, q00);
   }
+  // One tile per CTA with N % 128 != 0: the CLS query rides in row N, the
+  // first padding row of the last query tile, which visits every KV tile.
+  const bool tail_cls = TILES == 1 && p.cls_tail && !cls_cta && q00 == (p.n_q_tiles - 1) * 128;
   const int nkv_all = max(nkv0, nkv1);
 
   if (threadIdx.x == 0) {
@@ -228,7 +233,20 @@ __global__ void __launch_bounds__(AttnCfg<TILES>::kThreads, TILES == 2 ? 1 : 2)
   } else if (warp == 1 || (TILES == 2 && warp == 18)) {
     // one MMA issuer per query tile, so each tile's S / PV products follow
     // its own softmax without waiting on the other tile's
-    if (lane == 0) {
+    bool okq = true;
+    if (tail_cls) {
+      // once the Q tile has landed (its rows past N zero-filled), eight lanes
+      // write Q[bh, 0, :] into row N - q00 of it in the 128-byte-swizzled
+      // layout, then make the writes visible to the tensor core
+      okq = __all_sync(0xffffffffu, mbar_wait(&q_full, 0, w));
+      if (okq && lane < 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(p.q + static_cast<size_t>(bh) * p.N * 64 + lane * 8);
+        st_shared_v4(smem_u32(sm + C::kOffQ) + sw128_offset(p.N - q00, lane * 8), v.x, v.y, v.z, v.w);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+    }
+    if (lane == 0 && okq) {
       const int g = warp == 1 ? 0 : 1;
       const int nkv_g = g == 0 ? nkv0 : nkv1;
       constexpr uint32_t idesc_s = idesc_f16_f32(128, 128);
@@ -432,16 +450,18 @@ __global__ void __launch_bounds__(AttnCfg<TILES>::kThreads, TILES == 2 ? 1 : 2)
         tmem_ld_16x256b_x8(tO, o);
         // rows this CTA writes: the CLS CTA only row 0; pair CTAs every
         // valid row but a separately computed CLS row
-        const bool st_a = cls_tile ? (ia == 0) : (ia < p.N && !(ia == 0 && p.cls_separate));
-        const bool st_b = cls_tile ? (ib == 0) : (ib < p.N && !(ib == 0 && p.cls_separate));
+        // row N of the last tile holds the CLS query (tail_cls): output row 0
+        const bool st_a = cls_tile ? (ia == 0) : ((ia < p.N && !(ia == 0 && p.cls_separate)) || (tail_cls && ia == p.N));
+        const bool st_b = cls_tile ? (ib == 0) : ((ib < p.N && !(ib == 0 && p.cls_separate)) || (tail_cls && ib == p.N));
+        const int oa = ia == p.N ? 0 : ia, ob = ib == p.N ? 0 : ib;
         if (st_a) {
-          uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (static_cast<size_t>(b) * p.N + ia) * p.ldo + hd * 64 + 2 * kq);
+          uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (static_cast<size_t>(b) * p.N + oa) * p.ldo + hd * 64 + 2 * kq);
 #pragma unroll
           for (int m = 0; m < 8; ++m)
             dst[4 * m] = pack_half2(__uint_as_float(o[4 * m]) * inv_a, __uint_as_float(o[4 * m + 1]) * inv_a);
         }
         if (st_b) {
-          uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (static_cast<size_t>(b) * p.N + ib) * p.ldo + hd * 64 + 2 * kq);
+          uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (static_cast<size_t>(b) * p.N + ob) * p.ldo + hd * 64 + 2 * kq);
 #pragma unroll
           for (int m = 0; m < 8; ++m)
             dst[4 * m] = pack_half2(__uint_as_float(o[4 * m + 2]) * inv_b, __uint_as_float(o[4 * m + 3]) * inv_b);
@@ -651,6 +671,8 @@ int attn_prepare(AttnOp* op, const __half* q, const __half* k, const __half* vt,
   p.ldo = heads * 64;
   p.cls_separate = (mask == JEPA_B200_MASK_BLOCK_CAUSAL && has_cls) ? 1 : 0;
   p.cls_in_pair = (p.cls_separate && p.n_q_tiles % 2 == 1) ? 1 : 0;
+  p.cls_tail = (p.cls_separate && ntok % 128 != 0) ? 1 : 0;
+  p.q = q;
   op->q = q;
   op->k = k;
   op->vt = vt;
@@ -673,7 +695,7 @@ static int attn_launch_impl(const AttnParams& p, const AttnOp& op, cudaStream_t 
     attr_done |= 1ull << dev;
   }
   const int units = TILES == 2 ? (p.n_q_tiles + 1) / 2 + (p.cls_separate && !p.cls_in_pair ? 1 : 0)
-                               : p.n_q_tiles + p.cls_separate;
+                               : p.n_q_tiles + (p.cls_separate && !p.cls_tail ? 1 : 0);
   const dim3 grid = p.mask == JEPA_B200_MASK_BLOCK_CAUSAL ? dim3(op.B * p.heads, units) : dim3(units, op.B * p.heads);
   if (launch_pdl(kern, grid, dim3(C::kThreads), C::kSmem, st, 1, op.tmQ, op.tmK, op.tmV, p) != cudaSuccess)
     return JEPA_B200_ERR_CUDA;

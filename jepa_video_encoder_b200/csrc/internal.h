@@ -85,6 +85,8 @@ struct AttnParams {
   int N, heads, n_q_tiles, mask, has_cls, ppf;
   int cls_separate;  // block-causal with CLS: row 0 computed apart from query tile 0
   int cls_in_pair;   // ... as the second query tile of the last pair (odd tile count), else in a CTA of its own
+  int cls_tail;      // one tile per CTA: ... as padding row N of the last query tile (N % 128 != 0)
+  const __half* q;   // Q [B*h, N, 64] (the CLS query row copied into that padding row)
   float scale_log2;
   __half* out;
   int ldo;
