@@ -71,6 +71,7 @@ class EncoderConfig:
     pix_mean: tuple = IMAGENET_MEAN
     pix_std: tuple = IMAGENET_STD
     random_ln_affine: bool = False   # tests: exercise gamma/beta instead of 1/0
+    rope: bool = False               # 3-D rotary positions in the attention instead of pos_embed (no CLS)
 
     # -- derived shapes ---------------------------------------------------
     @property
@@ -187,8 +188,10 @@ def _block_names(prefix: str, D: int, M: int) -> List[tuple]:
     ]
 
 
-def tensor_specs(cfg: EncoderConfig, with_pos: bool = True) -> List[tuple]:
-    """(name, shape, kind) in table order."""
+def tensor_specs(cfg: EncoderConfig, with_pos: Optional[bool] = None) -> List[tuple]:
+    """(name, shape, kind) in table order (no pos_embed for a rotary model)."""
+    if with_pos is None:
+        with_pos = not cfg.rope
     D, M, kt, p = cfg.dim, cfg.mlp, cfg.tubelet, cfg.patch
     s = [("enc.patch_embed.weight", (D, 3, kt, p, p), "w"),
          ("enc.patch_embed.bias", (D,), "b")]

@@ -199,14 +199,54 @@ def merge_heads(x):
     return x.transpose(0, 2, 1, 3).reshape(B, N, h * d)
 
 
+# ---------------------------------------------------------------------------
+# 3-D rotary position embedding of the V-JEPA 2 encoders (the V-JEPA 2 card
+# and the "Quantization" page's check list name an "encoder with 3-D RoPE";
+# the pages give no formula, so the plainest 3-D extension of rotary
+# embeddings is read here): the head dimensions are split into three groups
+# of g = 2*floor(d_h/6), one per axis (time slot, patch row, patch column);
+# in group a the pair of dimensions (a*g + 2i, a*g + 2i + 1) is turned by the
+# angle pos_a * 10000^(-2i/g); the last d_h - 3g dimensions are not turned.
+# ---------------------------------------------------------------------------
+ROPE_BASE = 10000.0
+
+
+def rope_positions(cfg) -> np.ndarray:
+    """[N, 3] integer (slot, patch row, patch column) of every token; the
+    rotary models have no CLS row."""
+    pw = cfg.img_w // cfg.patch
+    ppf = cfg.patches_per_slot
+    n = np.arange(cfg.n_patches)
+    return np.stack([n // ppf, (n % ppf) // pw, (n % ppf) % pw], axis=1)
+
+
+def rope(x: np.ndarray, pos: np.ndarray, base: float = ROPE_BASE) -> np.ndarray:
+    """Rotate the head vectors x [..., N, d_h] of tokens at positions pos [N, 3]."""
+    d = x.shape[-1]
+    g = 2 * (d // 6)
+    out = np.array(x, np.float64, copy=True)
+    for a in range(3):
+        for i in range(g // 2):
+            th = pos[:, a].astype(np.float64) * base ** (-2.0 * i / g)
+            c, s = np.cos(th), np.sin(th)
+            j = a * g + 2 * i
+            x0, x1 = x[..., j], x[..., j + 1]
+            out[..., j] = x0 * c - x1 * s
+            out[..., j + 1] = x0 * s + x1 * c
+    return out
+
+
 def block(x, W: Dict[str, np.ndarray], prefix: str, heads: int, eps: float,
-          allow: Optional[np.ndarray]) -> np.ndarray:
+          allow: Optional[np.ndarray], rope_pos: Optional[np.ndarray] = None) -> np.ndarray:
     """One pre-LN transformer block.  attn_qkv's output columns are
-    [q | k | v], each head-major (head hd at hd*d_h ...)."""
+    [q | k | v], each head-major (head hd at hd*d_h ...).  With rope_pos, q and
+    k are rotated (after their bias) before the attention."""
     D = x.shape[-1]
     y = layer_norm(x, W[prefix + "ln1.weight"], W[prefix + "ln1.bias"], eps)
     qkv = linear(y, W[prefix + "attn_qkv.weight"], W[prefix + "attn_qkv.bias"])
     q, k, v = (split_heads(qkv[..., i * D:(i + 1) * D], heads) for i in range(3))
+    if rope_pos is not None:
+        q, k = rope(q, rope_pos), rope(k, rope_pos)
     o = merge_heads(attention(q, k, v, allow))
     x = x + linear(o, W[prefix + "attn_out.weight"], W[prefix + "attn_out.bias"])
     y = layer_norm(x, W[prefix + "ln2.weight"], W[prefix + "ln2.bias"], eps)
@@ -215,12 +255,15 @@ def block(x, W: Dict[str, np.ndarray], prefix: str, heads: int, eps: float,
 
 
 def embed(cfg, W, pixels) -> np.ndarray:
-    """Patch-embed, prepend CLS (when the model has one), add pos_embed."""
+    """Patch-embed, prepend CLS (when the model has one), add pos_embed (the
+    rotary models have none: their positions enter the attention)."""
     x = patch_embed(pixels, W["enc.patch_embed.weight"], W["enc.patch_embed.bias"],
                     cfg.patch, cfg.tubelet)
     if cfg.has_cls:
         cls = np.broadcast_to(W["enc.cls_token"], (x.shape[0], 1, x.shape[-1]))
         x = np.concatenate([cls, x], axis=1)
+    if getattr(cfg, "rope", False):
+        return x
     return x + W["enc.pos_embed"][None]
 
 
@@ -235,10 +278,11 @@ def encoder(cfg, W, pixels, layers: Optional[int] = None,
     """Full encoder: embed, ``depth`` blocks, final LayerNorm ->
     last_hidden_state [B, N, D]."""
     allow = encoder_allow(cfg)
+    rope_pos = rope_positions(cfg) if getattr(cfg, "rope", False) else None
     x = embed(cfg, W, pixels)
     res = [x]
     for i in range(cfg.depth if layers is None else layers):
-        x = block(x, W, f"enc.blk.{i}.", cfg.heads, cfg.ln_eps, allow)
+        x = block(x, W, f"enc.blk.{i}.", cfg.heads, cfg.ln_eps, allow, rope_pos)
         res.append(x)
     y = layer_norm(x, W["enc.norm.weight"], W["enc.norm.bias"], cfg.ln_eps)
     return (y, res) if return_residuals else y
@@ -298,7 +342,8 @@ def forward(cfg, W, pixels, pool_mode: Optional[str] = None) -> np.ndarray:
 # needed (K and V still come from every row).
 # ---------------------------------------------------------------------------
 def block_rows(x_clip: np.ndarray, W, prefix: str, heads: int, eps: float,
-               allow: Optional[np.ndarray], rows: Sequence[int]) -> np.ndarray:
+               allow: Optional[np.ndarray], rows: Sequence[int],
+               rope_pos: Optional[np.ndarray] = None) -> np.ndarray:
     rows = np.asarray(rows)
     N, D = x_clip.shape
     y = layer_norm(x_clip, W[prefix + "ln1.weight"], W[prefix + "ln1.bias"], eps)
@@ -307,6 +352,8 @@ def block_rows(x_clip: np.ndarray, W, prefix: str, heads: int, eps: float,
     k = linear(y, wqkv[D:2 * D], bqkv[D:2 * D])
     v = linear(y, wqkv[2 * D:], bqkv[2 * D:])
     qh, kh, vh = (split_heads(t[None], heads)[0] for t in (q, k, v))
+    if rope_pos is not None:
+        qh, kh = rope(qh, rope_pos[rows]), rope(kh, rope_pos)
     o = merge_heads(attention(qh, kh, vh, None if allow is None else allow[rows])[None])[0]
     xr = x_clip[rows] + linear(o, W[prefix + "attn_out.weight"], W[prefix + "attn_out.bias"])
     y2 = layer_norm(xr, W[prefix + "ln2.weight"], W[prefix + "ln2.bias"], eps)

@@ -389,3 +389,61 @@ def test_metrics_definitions():
     assert np.allclose(orc.token_cosines(a, b), [1 / math.sqrt(2), -1.0])
     assert orc.rel_max(a, b) == 4.0 / 2.0
     assert math.isclose(orc.rel_fro(a, b), math.sqrt(1 + 16) / math.sqrt(6))
+
+
+# ------------------------------------------------ 3-D rotary positions (R18) --
+def _rope_cfg():
+    return synth.VJEPA2_LONG.with_(name="rope_pin", dim=128, depth=1, heads=2, mlp=256, frames=6,
+                                   img_h=48, img_w=64, patch=16, rope=True)
+
+
+def test_rope_positions_enumerate_slot_row_column():
+    cfg = _rope_cfg()
+    want = [(t, y, x) for t in range(cfg.slots) for y in range(cfg.img_h // cfg.patch)
+            for x in range(cfg.img_w // cfg.patch)]
+    assert np.array_equal(orc.rope_positions(cfg), np.array(want))
+
+
+def test_rope_identity_at_origin_and_last_dims_untouched():
+    rng = np.random.default_rng(30)
+    x = rng.standard_normal((2, 7, 64))
+    assert np.array_equal(orc.rope(x, np.zeros((7, 3), int)), x)
+    pos = rng.integers(0, 40, (7, 3))
+    y = orc.rope(x, pos)
+    assert np.array_equal(y[..., 60:], x[..., 60:])  # 64 - 3 * 20 dimensions are not turned
+    pairs = lambda t: np.hypot(t[..., 0:60:2], t[..., 1:60:2])
+    assert np.allclose(pairs(y), pairs(x), rtol=1e-13, atol=0)  # every pair keeps its length
+
+
+def test_rope_rotation_closed_forms():
+    """Pair i = 0 of each axis turns by pos radians; pair i = 5 by pos / 100
+    (10000^(-10/20) = 1/100); a unit vector on the pair's first dimension
+    goes to (cos, sin) of that angle."""
+    for a in range(3):
+        for i, scale in ((0, 1.0), (5, 0.01)):
+            j = 20 * a + 2 * i
+            e = np.zeros((1, 64))
+            e[0, j] = 1.0
+            pos = np.zeros((1, 3), int)
+            pos[0, a] = 7
+            y = orc.rope(e, pos)
+            assert y[0, j] == pytest.approx(math.cos(7 * scale), abs=1e-15)
+            assert y[0, j + 1] == pytest.approx(math.sin(7 * scale), abs=1e-15)
+            assert np.count_nonzero(np.abs(y) > 1e-15) <= 2
+
+
+def test_rope_composition_adds_positions():
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((5, 64))
+    p, q = rng.integers(0, 20, (5, 3)), rng.integers(0, 20, (5, 3))
+    assert np.allclose(orc.rope(orc.rope(x, p), q), orc.rope(x, p + q), rtol=0, atol=1e-12)
+
+
+def test_rope_scores_depend_on_position_differences_only():
+    rng = np.random.default_rng(32)
+    qv, kv = rng.standard_normal((1, 64)), rng.standard_normal((1, 64))
+    for _ in range(5):
+        p, pk, c = rng.integers(0, 30, (1, 3)), rng.integers(0, 30, (1, 3)), rng.integers(0, 30, (1, 3))
+        s1 = (orc.rope(qv, p) @ orc.rope(kv, pk).T).item()
+        s2 = (orc.rope(qv, p + c) @ orc.rope(kv, pk + c).T).item()
+        assert s1 == pytest.approx(s2, rel=1e-11, abs=1e-12)
