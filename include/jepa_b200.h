@@ -90,6 +90,12 @@ typedef struct {
   int head_sa_blocks; /* attentive head: self-attention blocks before the cross-attention (0 = no head) */
   int n_classes;      /* attentive head: logits (0 = no head) */
   float ln_eps;       /* LayerNorm epsilon */
+  int rope;           /* 1: 3-D rotary positions in the encoder's attention instead of an additive
+                       * enc.pos_embed (the V-JEPA 2 encoders); needs has_cls = 0, at most 64
+                       * slots, patch rows and patch columns.  The head dims form three groups
+                       * of 20 (slot, patch row, patch column); in group a the pair
+                       * (20a + 2i, 20a + 2i + 1) of q and k turns by pos_a * 10000^(-2i/20),
+                       * i < 10; dims 60..63 stay as they are. */
 } jepa_b200_config;
 
 /* One entry of the tensor table.  Host memory, owned by the caller; it is
@@ -110,7 +116,7 @@ typedef struct jepa_b200_model jepa_b200_model;
 
 /* Validate the table against cfg and upload it to `device`.  Names follow the
  * "Quantization" page's scheme: enc.patch_embed.{weight,bias}, enc.pos_embed
- * [N, D], enc.cls_token [D] (has_cls), enc.blk.<i>.{ln1,attn_qkv,attn_out,ln2,
+ * [N, D] (not with rope), enc.cls_token [D] (has_cls), enc.blk.<i>.{ln1,attn_qkv,attn_out,ln2,
  * ffn_up,ffn_down}.{weight,bias}, enc.norm.{weight,bias}; with a head also
  * head.blk.<i>.*, head.query [D], head.ln_kv.*, head.xattn.{q,k,v,out,
  * ffn_up,ffn_down}.{weight,bias}, head.xattn.ln2.*, head.cls.{weight,bias}.

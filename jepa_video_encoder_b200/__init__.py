@@ -32,7 +32,8 @@ def make_config(cfg: "synth.EncoderConfig") -> _abi.Config:
     return _abi.Config(dim=cfg.dim, depth=cfg.depth, heads=cfg.heads, mlp=cfg.mlp, patch=cfg.patch,
                        tubelet=cfg.tubelet, img_h=cfg.img_h, img_w=cfg.img_w, frames=cfg.frames,
                        has_cls=1 if cfg.has_cls else 0, mask=synth.MASK_IDS[cfg.mask],
-                       head_sa_blocks=cfg.head_sa_blocks, n_classes=cfg.n_classes, ln_eps=cfg.ln_eps)
+                       head_sa_blocks=cfg.head_sa_blocks, n_classes=cfg.n_classes, ln_eps=cfg.ln_eps,
+                       rope=1 if cfg.rope else 0)
 
 
 class Model:

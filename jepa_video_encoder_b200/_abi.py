@@ -19,7 +19,7 @@ class Config(ctypes.Structure):
     _fields_ = [("dim", c_int), ("depth", c_int), ("heads", c_int), ("mlp", c_int),
                 ("patch", c_int), ("tubelet", c_int), ("img_h", c_int), ("img_w", c_int),
                 ("frames", c_int), ("has_cls", c_int), ("mask", c_int),
-                ("head_sa_blocks", c_int), ("n_classes", c_int), ("ln_eps", c_float)]
+                ("head_sa_blocks", c_int), ("n_classes", c_int), ("ln_eps", c_float), ("rope", c_int)]
 
 
 class TensorEntry(ctypes.Structure):

@@ -54,8 +54,31 @@ __device__ __forceinline__ void gelu_pair(float& a, float& b) {
   }
 }
 
+// Rotary positions: turn the pair (x0, x1) at head dims (d, d + 1), d even,
+// of the token at (slot, patch row, patch column) = (pt, py, px): axis group
+// a = d / 20, pair i = (d % 20) / 2, angle pos_a * 10000^(-2i/20) read from
+// the (cos, sin) table; dims 60..63 are not turned.
+__device__ __forceinline__ void rope_pair(float& x0, float& x1, int d, int pt, int py, int px, const float2* tab) {
+  if (d >= 60) return;
+  const int a = d / 20, i = (d - 20 * a) >> 1;
+  const int pos = a == 0 ? pt : (a == 1 ? py : px);
+  const float2 cs = __ldg(tab + (a * kRopeMaxPos + pos) * 10 + i);
+  const float y0 = x0 * cs.x - x1 * cs.y;
+  x1 = x0 * cs.y + x1 * cs.x;
+  x0 = y0;
+}
+
+// The token position of tile row `row` (rows are b * ntok + t, no CLS row).
+__device__ __forceinline__ void rope_position(const QkvDst& q, int row, int& pt, int& py, int& px) {
+  const int t = row % q.ntok;
+  pt = t / q.rope_ppf;
+  const int rem = t - pt * q.rope_ppf;
+  py = rem / q.rope_pw;
+  px = rem - py * q.rope_pw;
+}
+
 // Epilogue for 32 consecutive output columns col0..col0+31 of one row.
-template <bool LOWREG>
+template <bool LOWREG, bool ROPE>
 __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int col0, const uint32_t (&r)[32]) {
   float v[32];
 #pragma unroll
@@ -107,6 +130,12 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int
       const int hd = within >> 6, d0 = within & 63;
       const int b = row / p.qkv.ntok, t = row % p.qkv.ntok;
       const size_t bh = static_cast<size_t>(b) * p.qkv.heads + hd;
+      if (ROPE && part < 2) {
+        int pt, py, px;
+        rope_position(p.qkv, row, pt, py, px);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) rope_pair(v[2 * j], v[2 * j + 1], d0 + 2 * j, pt, py, px, p.qkv.rope);
+      }
       if (part < 2) {
         __half* base = part == 0 ? p.qkv.q : p.qkv.k;
         if (base) {
@@ -129,8 +158,8 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int
                                               (static_cast<size_t>(b) * p.patch.ntok + tok) * p.ldo + col0);
       const float4* pos = reinterpret_cast<const float4*>(p.patch.pos + static_cast<size_t>(tok) * p.ldo + col0);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float4 q = __ldg(pos + j);
+      for (int j = 0; j < 8; ++j) {  // a rotary model has no positional table
+        const float4 q = p.patch.pos ? __ldg(pos + j) : make_float4(0.f, 0.f, 0.f, 0.f);
         dst[j] = make_float4(v[4 * j] + q.x, v[4 * j + 1] + q.y, v[4 * j + 2] + q.z, v[4 * j + 3] + q.w);
       }
     } break;
@@ -284,7 +313,7 @@ __device__ __forceinline__ void fill_a_patch_vec8(uint8_t* sA, const GemmParams&
 
 // Epilogue of one output tile for one thread: its row, half of the BN
 // columns (chalf), read from TMEM at tb (lane quadrant already applied).
-template <int BN, bool LOWREG>
+template <int BN, bool LOWREG, bool ROPE = false>
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tb, int row, int nb, int chalf) {
   if (p.epi == EPI_RESID_F32) {
     // residual add: the residual's loads are issued before the TMEM load
@@ -318,7 +347,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tb, 
     for (int c = chalf * (BN / 64); c < (chalf + 1) * (BN / 64); ++c) {
       uint32_t r[32];
       tmem_ld32(tb + static_cast<uint32_t>(c * 32), r);
-      if (row < p.M) epilogue_chunk<LOWREG>(p, row, nb * BN + c * 32, r);
+      if (row < p.M) epilogue_chunk<LOWREG, ROPE>(p, row, nb * BN + c * 32, r);
     }
   }
 }
@@ -445,7 +474,7 @@ __device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUt
 // TMA store at (0, t0, b*h + head) when the 32 rows lie in one clip, else
 // written row by row.  V goes to V^T [B*h, 64, Npad] column by column (one
 // coalesced 64-byte store per dimension and warp).
-template <int BN, bool LOWREG>
+template <int BN, bool LOWREG, bool ROPE = false>
 __device__ __forceinline__ void epilogue_tile_qkv(const GemmParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
                                                   uint32_t tb, int row0, int nb, int chalf, uint8_t* stage_buf,
                                                   int lane, bool& pending) {
@@ -485,6 +514,8 @@ __device__ __forceinline__ void epilogue_tile_qkv(const GemmParams& p, const CUt
       continue;
     }
     __half* base = part == 0 ? p.qkv.q : p.qkv.k;
+    int pt = 0, py = 0, px = 0;
+    if (ROPE) rope_position(p.qkv, min(row, p.M - 1), pt, py, px);
     uint32_t w[32];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -495,9 +526,14 @@ __device__ __forceinline__ void epilogue_tile_qkv(const GemmParams& p, const CUt
       if (LOWREG) load_bias32(p.bias, col0 + h * 32, bb);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        w[h * 16 + 2 * j] = pack_half2(__uint_as_float(r[4 * j]) + bb[j].x, __uint_as_float(r[4 * j + 1]) + bb[j].y);
-        w[h * 16 + 2 * j + 1] =
-            pack_half2(__uint_as_float(r[4 * j + 2]) + bb[j].z, __uint_as_float(r[4 * j + 3]) + bb[j].w);
+        float x0 = __uint_as_float(r[4 * j]) + bb[j].x, x1 = __uint_as_float(r[4 * j + 1]) + bb[j].y;
+        float x2 = __uint_as_float(r[4 * j + 2]) + bb[j].z, x3 = __uint_as_float(r[4 * j + 3]) + bb[j].w;
+        if (ROPE) {  // q and k of a rotary model
+          rope_pair(x0, x1, h * 32 + 4 * j, pt, py, px, p.qkv.rope);
+          rope_pair(x2, x3, h * 32 + 4 * j + 2, pt, py, px, p.qkv.rope);
+        }
+        w[h * 16 + 2 * j] = pack_half2(x0, x1);
+        w[h * 16 + 2 * j + 1] = pack_half2(x2, x3);
       }
     }
     if (!base) continue;
@@ -526,7 +562,7 @@ __device__ __forceinline__ void epilogue_tile_qkv(const GemmParams& p, const CUt
   }
 }
 
-template <int BN, int BMODE, bool GATHER>
+template <int BN, int BMODE, bool GATHER, bool ROPE>
 __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
@@ -679,7 +715,8 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
       bool done = false;
       if constexpr (!kLowReg) {  // the 128-register kernels keep the row-by-row QKV stores
         if (p.tma_epi && p.epi == EPI_QKV) {
-          epilogue_tile_qkv<BN, false>(p, &tmC, &tmC2, tb, mb * 128 + quad * 32, nb, chalf, stage_buf, lane, pending);
+          epilogue_tile_qkv<BN, false, ROPE>(p, &tmC, &tmC2, tb, mb * 128 + quad * 32, nb, chalf, stage_buf, lane,
+                                             pending);
           done = true;
         }
       }
@@ -687,7 +724,7 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
       } else if (p.tma_epi && p.epi != EPI_QKV)
         epilogue_tile_tma<BN, kLowReg>(p, &tmC, tb, mb * 128 + quad * 32, nb, chalf, stage_buf, lane, pending);
       else
-        epilogue_tile<BN, kLowReg>(p, tb, row, nb, chalf);
+        epilogue_tile<BN, kLowReg, ROPE>(p, tb, row, nb, chalf);
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
       if (++acc == 2) {
@@ -759,7 +796,7 @@ struct Gemm2Cfg {
   static constexpr int SMEM = STAGES * STAGE_BYTES + 8 * 4096 + 1024;  // + epilogue staging
 };
 
-template <int BN>
+template <int BN, bool ROPE>
 __global__ void __launch_bounds__(320, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
@@ -905,11 +942,11 @@ __global__ void __launch_bounds__(320, 1)
       const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quad * 32;
       const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
       if (p.tma_epi && p.epi == EPI_QKV)
-        epilogue_tile_qkv<BN, true>(p, &tmC, &tmC2, tb, row0, nb, chalf, stage_buf, lane, pending);
+        epilogue_tile_qkv<BN, true, ROPE>(p, &tmC, &tmC2, tb, row0, nb, chalf, stage_buf, lane, pending);
       else if (p.tma_epi)
         epilogue_tile_tma<BN, false>(p, &tmC, tb, row0, nb, chalf, stage_buf, lane, pending);
       else
-        epilogue_tile<BN, false>(p, tb, row0 + lane, nb, chalf);
+        epilogue_tile<BN, false, ROPE>(p, tb, row0 + lane, nb, chalf);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tempty0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
@@ -1074,9 +1111,9 @@ int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& Win
   return JEPA_B200_OK;
 }
 
-template <int BN, int BMODE, bool GATHER>
+template <int BN, int BMODE, bool GATHER, bool ROPE = false>
 static int launch_impl(const GemmOp& op, cudaStream_t st) {
-  auto kern = gemm_tc_kernel<BN, BMODE, GATHER>;
+  auto kern = gemm_tc_kernel<BN, BMODE, GATHER, ROPE>;
   static unsigned long long attr_done = 0;  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1092,9 +1129,9 @@ static int launch_impl(const GemmOp& op, cudaStream_t st) {
   return JEPA_B200_OK;
 }
 
-template <int BN>
+template <int BN, bool ROPE = false>
 static int launch_pair(const GemmOp& op, cudaStream_t st) {
-  auto kern = gemm_pair_kernel<BN>;
+  auto kern = gemm_pair_kernel<BN, ROPE>;
   static unsigned long long attr_done = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1113,11 +1150,14 @@ int gemm_launch(const GemmOp& op_in, cudaStream_t st, DevErr* err, unsigned long
   GemmOp op = op_in;
   op.p.err = err;
   op.p.timeout_ns = timeout_ns;
+  // rotary q / k only in the QKV GEMMs of a rotary model: their own instances,
+  // so that the others carry no rotation code
+  const bool rope = op.p.epi == EPI_QKV && op.p.qkv.rope;
   if (op.pair) {
     switch (op.bn) {
-      case 256: return launch_pair<256>(op, st);
-      case 192: return launch_pair<192>(op, st);
-      default: return launch_pair<128>(op, st);
+      case 256: return rope ? launch_pair<256, true>(op, st) : launch_pair<256>(op, st);
+      case 192: return rope ? launch_pair<192, true>(op, st) : launch_pair<192>(op, st);
+      default: return rope ? launch_pair<128, true>(op, st) : launch_pair<128>(op, st);
     }
   }
   if (op.gather) {
@@ -1127,12 +1167,12 @@ int gemm_launch(const GemmOp& op_in, cudaStream_t st, DevErr* err, unsigned long
       default: return launch_impl<128, B_F16, true>(op, st);
     }
   }
-#define JB_GEMM_CASE(BNV)                                      \
-  case BNV:                                                    \
-    switch (op.bmode) {                                        \
-      case B_Q8: return launch_impl<BNV, B_Q8, false>(op, st); \
-      case B_Q4: return launch_impl<BNV, B_Q4, false>(op, st); \
-      default: return launch_impl<BNV, B_F16, false>(op, st);  \
+#define JB_GEMM_CASE(BNV)                                                                                      \
+  case BNV:                                                                                                    \
+    switch (op.bmode) {                                                                                        \
+      case B_Q8: return rope ? launch_impl<BNV, B_Q8, false, true>(op, st) : launch_impl<BNV, B_Q8, false>(op, st); \
+      case B_Q4: return rope ? launch_impl<BNV, B_Q4, false, true>(op, st) : launch_impl<BNV, B_Q4, false>(op, st); \
+      default: return rope ? launch_impl<BNV, B_F16, false, true>(op, st) : launch_impl<BNV, B_F16, false>(op, st); \
     }
   switch (op.bn) {
     JB_GEMM_CASE(256)

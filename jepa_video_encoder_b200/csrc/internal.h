@@ -36,7 +36,13 @@ struct QkvDst {
   __half* k = nullptr;
   __half* vt = nullptr;
   int ntok = 0, heads = 0, npad = 0, first_part = 0, dim = 0;
+  // 3-D rotary positions of q and k (null: none): (cos, sin) [3 axes][kRopeMaxPos][10]
+  const float2* rope = nullptr;
+  int rope_ppf = 0, rope_pw = 0;  // patches per slot, per patch row
 };
+
+// Positions per axis the rotary table holds (slots, patch rows, patch columns).
+constexpr int kRopeMaxPos = 64;
 
 // Source geometry of the implicit-GEMM patch-embed.
 struct PatchSrc {

@@ -66,6 +66,7 @@ struct jepa_b200_model {
   int N = 0, Np = 0, ppf = 0, Kpe = 0, Kpe_pad = 0, npad = 0;
   DevMatrix pe;
   float *b_pe = nullptr, *pos = nullptr, *cls = nullptr;
+  float2* rope = nullptr;  // rotary (cos, sin) table [3][kRopeMaxPos][10] (cfg.rope)
   std::vector<LayerW> enc, head;
   float *norm_g = nullptr, *norm_b = nullptr;
   bool has_head = false;
@@ -358,6 +359,10 @@ int validate_config(const jepa_b200_config* c) {
   if (c->dim > 4096 || c->mlp > 16384) return JEPA_B200_ERR_SHAPE;
   if (c->n_classes < 0 || c->head_sa_blocks < 0) return JEPA_B200_ERR_ARG;
   if (!(c->ln_eps > 0.0f)) return JEPA_B200_ERR_ARG;
+  if (c->rope != 0 && c->rope != 1) return JEPA_B200_ERR_ARG;
+  if (c->rope && (c->has_cls || c->frames / c->tubelet > kRopeMaxPos || c->img_h / c->patch > kRopeMaxPos ||
+                  c->img_w / c->patch > kRopeMaxPos))
+    return JEPA_B200_ERR_SHAPE;
   return JEPA_B200_OK;
 }
 
@@ -367,9 +372,14 @@ int alloc_ws(jepa_b200_model* m, void** p, size_t bytes) {
   return JEPA_B200_OK;
 }
 
-int prepare_block_ops(jepa_b200_model* m, const LayerW& L, BlockOps& ops, float* Xres, int R) {
+int prepare_block_ops(jepa_b200_model* m, const LayerW& L, BlockOps& ops, float* Xres, int R, bool rope) {
   const int D = m->cfg.dim, Mh = m->cfg.mlp;
   QkvDst qd;
+  if (rope) {  // the encoder blocks of a rotary model
+    qd.rope = m->rope;
+    qd.rope_ppf = (m->cfg.img_h / m->cfg.patch) * (m->cfg.img_w / m->cfg.patch);
+    qd.rope_pw = m->cfg.img_w / m->cfg.patch;
+  }
   qd.q = m->Q;
   qd.k = m->Kb;
   qd.vt = m->Vt;
@@ -453,10 +463,10 @@ int prepare_ops(jepa_b200_model* m, int B) {
   const int Ri = static_cast<int>(R);
   m->enc_ops.assign(m->enc.size(), BlockOps());
   for (size_t l = 0; l < m->enc.size(); ++l)
-    if ((s = prepare_block_ops(m, m->enc[l], m->enc_ops[l], m->X, Ri))) return s;
+    if ((s = prepare_block_ops(m, m->enc[l], m->enc_ops[l], m->X, Ri, m->cfg.rope != 0))) return s;
   m->head_ops.assign(m->head.size(), BlockOps());
   for (size_t l = 0; l < m->head.size(); ++l)
-    if ((s = prepare_block_ops(m, m->head[l], m->head_ops[l], m->Yf, Ri))) return s;
+    if ((s = prepare_block_ops(m, m->head[l], m->head_ops[l], m->Yf, Ri, false))) return s;
   PatchSrc ps;
   ps.pixels = nullptr;
   ps.T = c.frames;
@@ -786,7 +796,22 @@ static void load_sequence(Loader& L) {
     if (t && L.status == JEPA_B200_OK) m->pe = L.matrix({t}, m->Kpe, m->Kpe_pad);
   }
   m->b_pe = L.vec("enc.patch_embed.bias", D);
-  m->pos = L.table2d("enc.pos_embed", m->N, D);
+  if (c.rope) {
+    // (cos, sin) of pos * 10000^(-2i/20) for every axis position and pair i,
+    // in double precision, rounded once to f32
+    std::vector<float2> tab(static_cast<size_t>(3) * kRopeMaxPos * 10);
+    for (int a = 0; a < 3; ++a)
+      for (int pos = 0; pos < kRopeMaxPos; ++pos)
+        for (int i = 0; i < 10; ++i) {
+          const double th = pos * std::pow(10000.0, -2.0 * i / 20.0);
+          tab[(static_cast<size_t>(a) * kRopeMaxPos + pos) * 10 + i] =
+              make_float2(static_cast<float>(std::cos(th)), static_cast<float>(std::sin(th)));
+        }
+    m->rope = static_cast<float2*>(L.dalloc(tab.size() * sizeof(float2)));
+    if (m->rope) L.upload(m->rope, tab.data(), tab.size() * sizeof(float2));
+  } else {
+    m->pos = L.table2d("enc.pos_embed", m->N, D);
+  }
   if (c.has_cls) m->cls = L.vec("enc.cls_token", D);
   m->enc.resize(c.depth);
   for (int l = 0; l < c.depth; ++l) L.block(m->enc[l], "enc.blk." + std::to_string(l) + ".", D, Mh);

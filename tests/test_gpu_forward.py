@@ -28,6 +28,10 @@ SMALL = {
     "vjepa2_ssv2": _small(synth.VJEPA2_SSV2, frames=8, batch=3, head_sa_blocks=1),   # q8_0 + head
     "levjepa_q4": _small(synth.LEVJEPA_VIT_L_Q4, frames=8, batch=2),
     "vjepa2_long": _small(synth.VJEPA2_LONG, frames=16, batch=2),                    # 128 tokens, bidir
+    # 3-D rotary positions: 128 tokens x 2 clips (CTA-pair GEMMs, TMA QKV epilogue) and,
+    # with q8_0 and the head, 64 tokens x 3 clips (row-by-row QKV epilogue)
+    "vjepa2_rope": _small(synth.VJEPA2_LONG, frames=16, batch=2, rope=True),
+    "vjepa2_ssv2_rope": _small(synth.VJEPA2_SSV2, frames=8, batch=3, head_sa_blocks=1, rope=True),
 }
 
 
@@ -216,13 +220,14 @@ def _full_size_layers(cfg, layers, clips, rows_fn):
     for b in clips:
         assert_tokens_close(x0[b], emb[b], COS_F16, REL_MAX_F16, what=f"{cfg.name} embed clip {b}")
     allow = orc.encoder_allow(cfg)
+    rope_pos = orc.rope_positions(cfg) if cfg.rope else None
     for l in layers:
         xin = host(m.debug_stage(pd, l))
         xout = host(m.debug_stage(pd, l + 1))
         assert m.sync_status() == 0
         for b in clips:
             rows = rows_fn(cfg)
-            ref = orc.block_rows(xin[b], W, f"enc.blk.{l}.", cfg.heads, cfg.ln_eps, allow, rows)
+            ref = orc.block_rows(xin[b], W, f"enc.blk.{l}.", cfg.heads, cfg.ln_eps, allow, rows, rope_pos)
             _increment_check(xin[b], xout[b], ref, rows, cos_min, f"{cfg.name} block {l} clip {b}")
     return m, table, pix, W
 
@@ -292,4 +297,14 @@ def test_vjepa2_long_full_size_sampled():
     assert m.sync_status() == 0
     ref = orc.layer_norm(x24, W["enc.norm.weight"], W["enc.norm.bias"], cfg.ln_eps)
     assert_tokens_close(out, ref, what="long final norm")
+    m.close()
+
+
+def test_vjepa2_long_rope_full_size_sampled():
+    """The 64-frame, 8192-token V-JEPA 2 clip with 3-D rotary positions in
+    every encoder block (slots up to 31, patch rows and columns up to 15):
+    blocks 0 and 23 on sampled rows."""
+    need_cuda()
+    cfg = synth.VJEPA2_LONG.with_(name="vjepa2_vit_l16_64f256_rope_b2", rope=True)
+    m, table, pix, W = _full_size_layers(cfg, [0, 23], [0, 1], _rows)
     m.close()
