@@ -132,9 +132,14 @@ VJEPA2_LONG = EncoderConfig(
     patch=16, tubelet=2, img_h=256, img_w=256, frames=64, has_cls=False,
     mask="bidir", weights="f16", batch=2, pool="none", seed=4)
 
+# The V-JEPA 2 workloads with the 3-D rotary positions of the real encoders
+# (instead of an additive table).
+VJEPA2_LONG_ROPE = VJEPA2_LONG.with_(name="vjepa2_vit_l16_64f256_rope_b2", rope=True)
+VJEPA2_SSV2_ROPE = VJEPA2_SSV2.with_(name="vjepa2_vit_l16_16f256_ssv2_q8_rope_b8", rope=True)
+
 WORKLOADS: Dict[str, EncoderConfig] = {
     c.name: c for c in (LEWM_VIT_TI, LEVJEPA_VIT_L, VJEPA2_SSV2,
-                        LEVJEPA_VIT_L_Q4, VJEPA2_LONG)}
+                        LEVJEPA_VIT_L_Q4, VJEPA2_LONG, VJEPA2_LONG_ROPE, VJEPA2_SSV2_ROPE)}
 
 
 def small_config(base: EncoderConfig, **kw) -> EncoderConfig:
