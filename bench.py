@@ -23,6 +23,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -259,8 +260,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         return 0 if st == 0 else 1
 
     # ---- timed region: K steps, each between CUDA events, L2 flushed between steps
-    clock_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv") if os.path.isdir(
-        os.path.join(ROOT, "gpurun_out")) else f"/tmp/jepa_clocks_rank{rank}.csv"
+    clock_path = (args.clock_log.replace("{rank}", str(rank)) if args.clock_log else
+                  os.path.join(tempfile.gettempdir(), f"jepa_clocks_rank{rank}.csv"))
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     if world > 1:
         torch.distributed.barrier()
@@ -377,6 +378,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
+    ap.add_argument("--clock-log", default=None,
+                    help="CSV of the nvidia-smi clock samples taken during the timed region ({rank} is replaced)")
     ap.add_argument("--forward-only", action="store_true",
                     help="run warm-up + --steps forwards and exit (no timing, no JSON): for ncu launch lists")
     args = ap.parse_args()
