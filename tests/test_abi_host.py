@@ -132,6 +132,29 @@ def test_bad_config(lib):
     assert lib.jepa_b200_load_weights(ctypes.byref(c), None, 0, 0, ctypes.byref(h)) == _abi.ERR_ARG
 
 
+def test_rotary_config_validation(lib):
+    """Rotary positions take one (slot, row, column) index per patch token:
+    no CLS token, and at most 64 positions on each axis."""
+    cfg = _tiny_cfg(has_cls=False, rope=True, pool="mean")
+    table = synth.make_tensor_table(cfg)
+    assert "enc.pos_embed" not in [t.name for t in table]
+    assert _load(lib, cfg, table) == (0 if _has_gpu() else _abi.ERR_CUDA)
+    assert _load(lib, cfg.with_(has_cls=True, pool="cls"), synth.make_tensor_table(cfg.with_(has_cls=True))) \
+        == _abi.ERR_SHAPE
+    edge = cfg.with_(frames=64, img_w=8 * 64)                              # 64 slots, 64 patch columns
+    assert _load(lib, edge, synth.make_tensor_table(edge)) == (0 if _has_gpu() else _abi.ERR_CUDA)
+    assert _load(lib, cfg.with_(frames=65), table) == _abi.ERR_SHAPE       # 65 slots
+    assert _load(lib, cfg.with_(frames=130, tubelet=2), table) == _abi.ERR_SHAPE   # 65 slots of two frames
+    assert _load(lib, cfg.with_(img_h=8 * 65), table) == _abi.ERR_SHAPE    # 65 patch rows
+    assert _load(lib, cfg.with_(img_w=8 * 65), table) == _abi.ERR_SHAPE    # 65 patch columns
+    c = make_config(cfg)
+    c.rope = 2
+    h = ctypes.c_void_p()
+    assert lib.jepa_b200_load_weights(ctypes.byref(c), None, 0, 0, ctypes.byref(h)) == _abi.ERR_ARG
+    # without rotary positions the additive table is required again
+    assert _load(lib, cfg.with_(rope=False), table) == _abi.ERR_MISSING_TENSOR
+
+
 def test_null_arguments(lib):
     shp = (ctypes.c_int64 * 3)()
     assert lib.jepa_b200_out_shape(None, 1, 0, shp) == _abi.ERR_ARG
