@@ -214,43 +214,13 @@ __device__ __forceinline__ void fill_b_quant(uint8_t* sB, const GemmParams& p, i
   }
 }
 
-// Gather a [128 x 64] slice of the unfolded patch matrix: row m = patch
-// (clip b, slot t', patch row, patch col); column k = (c, dt, kh, kw) in the
+// The patch-embed's A operand is gathered straight from the pixels: a
+// [128 x 64] slice of the unfolded patch matrix per K block, row m = patch
+// (clip b, slot t', patch row, patch col), column k = (c, dt, kh, kw) in the
 // row-major order of a conv weight [D, 3, kt, p, p].  Columns >= 3*kt*p*p
-// and rows >= M are zero.
-__device__ __forceinline__ void fill_a_patch(uint8_t* sA, const GemmParams& p, int m0, int kb, int ct) {
-  const PatchSrc& s = p.patch;
-  const int wp = s.W / s.patch;
-  const int ppf = (s.H / s.patch) * wp;
-  const int pp = s.patch * s.patch;
-  const int ktpp = s.tubelet * pp;
-  const uint32_t sbase = smem_u32(sA);
-  for (int idx = ct; idx < 128 * 8; idx += 128) {
-    const int r = idx >> 3, u = idx & 7;
-    const int m = m0 + r;
-    float f[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) f[e] = 0.0f;
-    if (m < p.M) {
-      const int b = m / s.n_patches, i = m % s.n_patches;
-      const int tp = i / ppf, rem = i % ppf;
-      const int hp = rem / wp, wq = rem % wp;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int k = kb * 64 + u * 8 + e;
-        if (k < s.k_real) {
-          const int c = k / ktpp, rk = k % ktpp;
-          const int dt = rk / pp, rk2 = rk % pp;
-          const int kh = rk2 / s.patch, kw = rk2 % s.patch;
-          const size_t plane = (static_cast<size_t>(b) * s.T + tp * s.tubelet + dt) * 3 + c;
-          f[e] = __ldg(s.pixels + (plane * s.H + hp * s.patch + kh) * s.W + wq * s.patch + kw);
-        }
-      }
-    }
-    st_shared_v4(sbase + sw128_offset(r, u * 8), pack_half2(f[0], f[1]), pack_half2(f[2], f[3]),
-                 pack_half2(f[4], f[5]), pack_half2(f[6], f[7]));
-  }
-}
+// and rows >= M are zero.  Pixel offset = rowbase(m) + koff(k), with
+//   rowbase = ((b*T + t'*kt) * 3) * H*W + (patch row * p) * W + patch col * p
+//   koff    = (dt*3 + c) * H*W + kh * W + kw.
 
 // Fast gather for patches whose rows are multiples of 8 pixels on 16-byte
 // aligned image rows: a converter thread always fills the same 8-column unit
@@ -308,6 +278,39 @@ __device__ __forceinline__ void fill_a_patch_vec8(uint8_t* sA, const GemmParams&
       w3 = pack_half2(b.z, b.w);
     }
     st_shared_v4(sbase + sw128_offset(r, u * 8), w0, w1, w2, w3);
+  }
+}
+
+// General gather (any patch size, pixels 4-byte aligned): the ownership of
+// the fast path above, with the 8 column offsets of the thread's unit taken
+// once per K block and 4-byte loads, all 64 of a K block independent.
+__device__ __forceinline__ void fill_a_patch_rows(uint8_t* sA, const GemmParams& p, int kb, int ct,
+                                                  const long long (&rowbase)[8]) {
+  const PatchSrc& s = p.patch;
+  const int u = ct & 7;
+  const int pp = s.patch * s.patch, ktpp = s.tubelet * pp;
+  long long koff[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int k = kb * 64 + u * 8 + e;
+    koff[e] = -1;
+    if (k < s.k_real) {
+      const int c = k / ktpp, rk = k % ktpp;
+      const int dt = rk / pp, rk2 = rk % pp;
+      const int kh = rk2 / s.patch, kw = rk2 % s.patch;
+      koff[e] = static_cast<long long>(dt * 3 + c) * s.H * s.W + static_cast<long long>(kh) * s.W + kw;
+    }
+  }
+  const uint32_t sbase = smem_u32(sA);
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int r = (ct >> 3) + 16 * it;
+    float f[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      f[e] = (rowbase[it] >= 0 && koff[e] >= 0) ? __ldg(s.pixels + rowbase[it] + koff[e]) : 0.0f;
+    st_shared_v4(sbase + sw128_offset(r, u * 8), pack_half2(f[0], f[1]), pack_half2(f[2], f[3]),
+                 pack_half2(f[4], f[5]), pack_half2(f[6], f[7]));
   }
 }
 
@@ -742,7 +745,7 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       const int nb = t % p.n_tiles, mb = t / p.n_tiles;
-      if (vec8) patch_rowbases(p, mb * 128, ct, rowbase);
+      if (GATHER) patch_rowbases(p, mb * 128, ct, rowbase);
       for (int kb = 0; kb < kblocks; ++kb) {
         bool okw = mbar_wait(&empty_bar[stage], phase ^ 1, w);
         okw = __all_sync(0xffffffffu, okw);
@@ -755,7 +758,7 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
         if (GATHER && vec8)
           fill_a_patch_vec8(sA, p, kb, ct, rowbase);
         else if (GATHER)
-          fill_a_patch(sA, p, mb * 128, kb, ct);
+          fill_a_patch_rows(sA, p, kb, ct, rowbase);
         else
           fill_b_quant<BMODE, BN>(sB, p, nb * BN, kb, ct);
         fence_proxy_async_smem();

@@ -127,6 +127,9 @@ VJEPA2_SSV2 = EncoderConfig(
 LEVJEPA_VIT_L_Q4 = LEVJEPA_VIT_L.with_(
     name="levjepa_vit_l16_16f224_q4_b8", weights="q4_0", batch=8, pool="mean",
     seed=3)
+# the same q4_0 model at one clip (where the weight stream is visible) and at 32
+LEVJEPA_VIT_L_Q4_B1 = LEVJEPA_VIT_L_Q4.with_(name="levjepa_vit_l16_16f224_q4_b1", batch=1)
+LEVJEPA_VIT_L_Q4_B32 = LEVJEPA_VIT_L_Q4.with_(name="levjepa_vit_l16_16f224_q4_b32", batch=32)
 VJEPA2_LONG = EncoderConfig(
     name="vjepa2_vit_l16_64f256_b2", dim=1024, depth=24, heads=16, mlp=4096,
     patch=16, tubelet=2, img_h=256, img_w=256, frames=64, has_cls=False,
@@ -138,8 +141,9 @@ VJEPA2_LONG_ROPE = VJEPA2_LONG.with_(name="vjepa2_vit_l16_64f256_rope_b2", rope=
 VJEPA2_SSV2_ROPE = VJEPA2_SSV2.with_(name="vjepa2_vit_l16_16f256_ssv2_q8_rope_b8", rope=True)
 
 WORKLOADS: Dict[str, EncoderConfig] = {
-    c.name: c for c in (LEWM_VIT_TI, LEVJEPA_VIT_L, VJEPA2_SSV2,
-                        LEVJEPA_VIT_L_Q4, VJEPA2_LONG, VJEPA2_LONG_ROPE, VJEPA2_SSV2_ROPE)}
+    c.name: c for c in (LEWM_VIT_TI, LEVJEPA_VIT_L, VJEPA2_SSV2, LEVJEPA_VIT_L_Q4,
+                        LEVJEPA_VIT_L_Q4_B1, LEVJEPA_VIT_L_Q4_B32, VJEPA2_LONG,
+                        VJEPA2_LONG_ROPE, VJEPA2_SSV2_ROPE)}
 
 
 def small_config(base: EncoderConfig, **kw) -> EncoderConfig:

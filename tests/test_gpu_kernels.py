@@ -316,6 +316,11 @@ def test_attention_block_causal_perturbation_bit_identical():
     (2, 4, 64, 48, 16, 2, 256, False),
     (1, 1, 224, 224, 14, 1, 192, True),        # LeWM: K = 588, padded to 640
     (3, 3, 32, 32, 16, 1, 128, True),
+    # the general gather (patch rows not a multiple of 8 pixels): tubelet 2,
+    # ragged K blocks, a ragged row tile, several row tiles
+    (2, 4, 36, 60, 12, 2, 128, False),
+    (3, 2, 42, 28, 14, 2, 192, True),
+    (2, 2, 112, 98, 14, 1, 128, True),
 ])
 def test_patch_embed(B, T, H, W, p, kt, D, has_cls):
     need_cuda()
