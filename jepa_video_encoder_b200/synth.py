@@ -115,6 +115,9 @@ LEWM_VIT_TI = EncoderConfig(
     tubelet=1, img_h=224, img_w=224, frames=1, has_cls=True, mask="bidir",
     weights="f32", batch=1, pool="cls", seed=0, pix_mean=(0.5, 0.5, 0.5),
     pix_std=(0.5, 0.5, 0.5))
+# the same model at the batch sizes the pages also time it at
+LEWM_VIT_TI_B8 = LEWM_VIT_TI.with_(name="lewm_vit_ti14_224_b8", batch=8)
+LEWM_VIT_TI_B32 = LEWM_VIT_TI.with_(name="lewm_vit_ti14_224_b32", batch=32)
 LEVJEPA_VIT_L = EncoderConfig(
     name="levjepa_vit_l16_16f224_b4", dim=1024, depth=24, heads=16, mlp=4096,
     patch=16, tubelet=1, img_h=224, img_w=224, frames=16, has_cls=True,
@@ -141,9 +144,9 @@ VJEPA2_LONG_ROPE = VJEPA2_LONG.with_(name="vjepa2_vit_l16_64f256_rope_b2", rope=
 VJEPA2_SSV2_ROPE = VJEPA2_SSV2.with_(name="vjepa2_vit_l16_16f256_ssv2_q8_rope_b8", rope=True)
 
 WORKLOADS: Dict[str, EncoderConfig] = {
-    c.name: c for c in (LEWM_VIT_TI, LEVJEPA_VIT_L, VJEPA2_SSV2, LEVJEPA_VIT_L_Q4,
-                        LEVJEPA_VIT_L_Q4_B1, LEVJEPA_VIT_L_Q4_B32, VJEPA2_LONG,
-                        VJEPA2_LONG_ROPE, VJEPA2_SSV2_ROPE)}
+    c.name: c for c in (LEWM_VIT_TI, LEWM_VIT_TI_B8, LEWM_VIT_TI_B32, LEVJEPA_VIT_L,
+                        VJEPA2_SSV2, LEVJEPA_VIT_L_Q4, LEVJEPA_VIT_L_Q4_B1,
+                        LEVJEPA_VIT_L_Q4_B32, VJEPA2_LONG, VJEPA2_LONG_ROPE, VJEPA2_SSV2_ROPE)}
 
 
 def small_config(base: EncoderConfig, **kw) -> EncoderConfig:

@@ -70,11 +70,12 @@ def test_small_workload_last_hidden_state(name):
     m.close()
 
 
-def test_lewm_full_size():
+@pytest.mark.parametrize("name", ["lewm_vit_ti14_224_b1", "lewm_vit_ti14_224_b8"])
+def test_lewm_full_size(name):
     """LeWM ViT-Ti/14, 224^2, 257 tokens, f32 weights, CLS output: the whole
-    forward in the oracle."""
+    forward in the oracle, one clip and a batch of 8 (2056 rows)."""
     need_cuda()
-    cfg = synth.LEWM_VIT_TI
+    cfg = synth.WORKLOADS[name]
     m, table, pix, got = _run(cfg, "none")
     ref = orc.encoder(cfg, orc.weights_f64(table), pix.astype(np.float64))
     assert_tokens_close(got, ref, what="lewm full")
