@@ -80,8 +80,10 @@ typedef enum {
 } jepa_b200_mask;
 
 /* Model shape.  N = (frames/tubelet) * (img_h/patch) * (img_w/patch) + has_cls.
- * Requirements: dim = 64 * heads; dim and mlp multiples of 64; img_h, img_w
- * multiples of patch; frames a multiple of tubelet. */
+ * Requirements (JEPA_B200_ERR_SHAPE otherwise): dim = 64 * heads, at most
+ * 4096; dim and mlp multiples of 64, mlp at most 16384; img_h, img_w
+ * multiples of patch; frames a multiple of tubelet; N at most 524288 (one
+ * clip within a call's row limit); 3 * tubelet * patch^2 at most 32768. */
 typedef struct {
   int dim, depth, heads, mlp;
   int patch, tubelet, img_h, img_w, frames;

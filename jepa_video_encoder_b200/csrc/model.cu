@@ -357,6 +357,12 @@ int validate_config(const jepa_b200_config* c) {
     return JEPA_B200_ERR_SHAPE;
   if (c->mask != JEPA_B200_MASK_BIDIR && c->mask != JEPA_B200_MASK_BLOCK_CAUSAL) return JEPA_B200_ERR_ARG;
   if (c->dim > 4096 || c->mlp > 16384) return JEPA_B200_ERR_SHAPE;
+  // one clip must fit the row limit of a call (B * N * 4096 < 2^31), and the
+  // patch vector 3 * kt * p * p the patch-embed's K
+  const long long tokens = static_cast<long long>(c->frames / c->tubelet) * (c->img_h / c->patch) *
+                           (c->img_w / c->patch) + (c->has_cls ? 1 : 0);
+  if (tokens > (1ll << 31) / 4096) return JEPA_B200_ERR_SHAPE;
+  if (3ll * c->tubelet * c->patch * c->patch > 32768) return JEPA_B200_ERR_SHAPE;
   if (c->n_classes < 0 || c->head_sa_blocks < 0) return JEPA_B200_ERR_ARG;
   if (!(c->ln_eps > 0.0f)) return JEPA_B200_ERR_ARG;
   if (c->rope != 0 && c->rope != 1) return JEPA_B200_ERR_ARG;

@@ -126,6 +126,11 @@ def test_bad_config(lib):
     table = synth.make_tensor_table(cfg)
     assert _load(lib, cfg.with_(heads=3), table) == _abi.ERR_SHAPE       # dim != 64 * heads
     assert _load(lib, cfg.with_(img_h=20), table) == _abi.ERR_SHAPE      # not a multiple of the patch
+    # shapes whose sizes would overflow 32-bit indexing are refused up front
+    assert _load(lib, cfg.with_(patch=1, img_h=1 << 16, img_w=1 << 16), table) == _abi.ERR_SHAPE
+    assert _load(lib, cfg.with_(patch=1, img_h=512, img_w=1024, frames=1), table) == _abi.ERR_SHAPE
+    assert _load(lib, cfg.with_(patch=1 << 16, img_h=1 << 16, img_w=1 << 16), table) == _abi.ERR_SHAPE
+    assert _load(lib, cfg.with_(patch=128, tubelet=1, img_h=128, img_w=128), table) == _abi.ERR_SHAPE
     c = make_config(cfg)
     c.mask = 7
     h = ctypes.c_void_p()
