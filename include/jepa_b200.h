@@ -287,7 +287,9 @@ JEPA_B200_API int jepa_b200_op_attention(const void *q, const void *k, const voi
 /* Tubelet patch-embed as an implicit GEMM, plus pos_embed and the CLS row.
  * pixels f32 [B, T, 3, H, W]; w_pe f16 [D, kpad] (kpad = 3*kt*p*p rounded up
  * to 64, zero padded); bias f32 [D]; pos f32 [ntok, D]; cls f32 [D] (has_cls);
- * x out f32 [B, ntok, D] with ntok = has_cls + (T/kt)(H/p)(W/p). */
+ * x out f32 [B, ntok, D] with ntok = has_cls + (T/kt)(H/p)(W/p).  The shape
+ * limits are the model's: D <= 4096, 3*kt*p*p <= 32768, B * ntok <= 524288
+ * (JEPA_B200_ERR_SHAPE otherwise). */
 JEPA_B200_API int jepa_b200_op_patch_embed(const float *pixels, int B, int T, int H, int W, int patch, int tubelet,
                              const void *w_pe, int D, const float *bias, const float *pos, const float *cls,
                              int has_cls, float *x, void *stream);

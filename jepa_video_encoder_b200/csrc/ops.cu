@@ -166,6 +166,11 @@ int jepa_b200_op_patch_embed(const float* pixels, int B, int T, int H, int W, in
       W < patch || D < 64 || D % 32 != 0)
     return JEPA_B200_ERR_SHAPE;
   if (!aligned16(x) || !aligned16(pos) || (bias && !aligned16(bias))) return JEPA_B200_ERR_ARG;
+  // the limits of the model loader: K = 3 * kt * p^2 <= 32768, B * ntok * 4096 < 2^31
+  if (D > 4096 || 3ll * tubelet * patch * patch > 32768 ||
+      static_cast<long long>(B) * ((static_cast<long long>(T / tubelet) * (H / patch) * (W / patch)) + 1) >
+          (1ll << 31) / 4096)
+    return JEPA_B200_ERR_SHAPE;
   const int k_real = 3 * tubelet * patch * patch;
   const int kpad = (k_real + 63) / 64 * 64;
   const int n_patches = (T / tubelet) * (H / patch) * (W / patch);

@@ -160,6 +160,23 @@ def test_rotary_config_validation(lib):
     assert _load(lib, cfg.with_(rope=False), table) == _abi.ERR_MISSING_TENSOR
 
 
+def test_patch_embed_op_shape_limits(lib):
+    """The single-kernel patch-embed refuses shapes beyond the model's limits
+    before touching the device (the pointers are never dereferenced)."""
+    buf = (ctypes.c_float * 64)()
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    p = ctypes.c_void_p((p.value + 15) // 16 * 16) if p.value % 16 else p
+
+    def call(B, T, H, W, patch, kt, D):
+        return lib.jepa_b200_op_patch_embed(p, B, T, H, W, patch, kt, p, D, None, p, None, 0, p, None)
+
+    assert call(1, 1, 128, 128, 128, 1, 128) == _abi.ERR_SHAPE           # K = 49152
+    assert call(1, 1, 1 << 16, 1 << 16, 1, 1, 128) == _abi.ERR_SHAPE      # 2^32 patches
+    assert call(3, 1, 512, 512, 1, 1, 128) == _abi.ERR_SHAPE              # 3 * 262144 rows
+    assert call(1, 1, 64, 64, 16, 1, 8192) == _abi.ERR_SHAPE              # D > 4096
+    assert call(1, 1, 20, 64, 16, 1, 128) == _abi.ERR_SHAPE               # H not a multiple of the patch
+
+
 def test_null_arguments(lib):
     shp = (ctypes.c_int64 * 3)()
     assert lib.jepa_b200_out_shape(None, 1, 0, shp) == _abi.ERR_ARG
