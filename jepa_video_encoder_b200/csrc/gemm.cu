@@ -21,6 +21,10 @@
 //   warps 10-13 (quantised weights or patch-embed only) converters: unpack
 //               q8_0 (q*d) or q4_0 ((q-8)*d) blocks, or gather pixels, into
 //               the swizzled operand tile in shared memory.
+// That single-CTA kernel serves the patch-embed and GEMMs of fewer than 256
+// rows.  The encoder's GEMMs (256 rows or more, f16 weights or the f16 copy
+// of dequantised ones) run the CTA-pair variant further down: two SMs share
+// a 256 x BN tile through tcgen05.mma.cta_group::2.
 #include <cudaTypedefs.h>
 #include <string.h>
 
