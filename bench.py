@@ -183,6 +183,7 @@ def cpu_oracle_sample(cfg, target_s: float = 12.0):
     x = orc.embed(cfg, W, pix)
     t_embed = time.perf_counter() - t0
     allow = orc.encoder_allow(cfg)
+    rope_pos = orc.rope_positions(cfg) if cfg.rope else None
     blocks, t_blocks = 0, 0.0
     while blocks < cfg.depth and t_blocks < target_s:
         pre = f"enc.blk.{blocks}."
@@ -190,7 +191,7 @@ def cpu_oracle_sample(cfg, target_s: float = 12.0):
             if n.startswith(pre):
                 W[n] = orc.tensor_f64(table[n])
         t1 = time.perf_counter()
-        x = orc.block(x, W, pre, cfg.heads, cfg.ln_eps, allow)
+        x = orc.block(x, W, pre, cfg.heads, cfg.ln_eps, allow, rope_pos)
         t_blocks += time.perf_counter() - t1
         blocks += 1
     t2 = time.perf_counter()
@@ -363,7 +364,7 @@ def run_ours(args, cfg, rank, world, local_rank):
                 "h2d_bytes_per_step": int(pix_host.numel() * 4), "d2h_bytes_per_step": int(out_host.numel() * 4)},
         "gpu_launches": launches,
         "clocks": clocks,
-        "when": datetime.datetime.utcnow().isoformat() + "Z",
+        "when": datetime.datetime.now(datetime.timezone.utc).strftime("%Y-%m-%dT%H:%M:%S.%fZ"),
     }
     print(json.dumps(line), flush=True)
     model.close()

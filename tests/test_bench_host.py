@@ -1,0 +1,68 @@
+"""bench.py's host-side pieces, on the CPU: the algorithmic FLOP count the
+roofline divides by, the oracle's timed sample, and the reference arm's line."""
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from jepa_video_encoder_b200 import synth  # noqa: E402
+from oracle import jepa_oracle as orc  # noqa: E402
+
+
+def test_block_causal_pair_count_closed_form():
+    """LeVJEPA, 16 slots of 196 patches plus the CLS sink: a patch of slot s
+    reads the (s+1)*196 patches of slots <= s; the CLS row reads all N keys."""
+    cfg = synth.LEVJEPA_VIT_L
+    pf, slots, N = 196, 16, 3137
+    pairs = pf * pf * sum(s + 1 for s in range(slots)) + N
+    assert pairs == 5_227_713
+    fl = bench._flops(cfg)
+    assert fl["attention"] == 4.0 * pairs * cfg.dim * cfg.depth
+    # against the oracle's own mask table on the same shape
+    allow = orc.allowed_keys(cfg.n_patches, cfg.patches_per_slot, cfg.has_cls, cfg.mask)
+    assert int(allow.sum()) == pairs
+    # bidirectional models count every pair
+    v = synth.VJEPA2_LONG
+    assert bench._flops(v)["attention"] == 4.0 * v.n_tokens ** 2 * v.dim * v.depth
+
+
+def test_gemm_flops_per_clip():
+    cfg = synth.LEVJEPA_VIT_L
+    fl = bench._flops(cfg)
+    N, D, M, L = 3137, 1024, 4096, 24
+    assert fl["gemm_qkv"] + fl["gemm_out"] + fl["gemm_up"] + fl["gemm_down"] == 2.0 * N * L * (3 * D * D + D * D + 2 * D * M)
+    assert fl["patch_embed"] == 2.0 * 3136 * 768 * D
+
+
+def test_cpu_sample_runs_the_rotary_blocks(monkeypatch):
+    calls = []
+    real = orc.rope
+
+    def counting(x, pos, *a, **k):
+        calls.append(x.shape)
+        return real(x, pos, *a, **k)
+
+    monkeypatch.setattr(orc, "rope", counting)
+    cfg = synth.small_config(synth.VJEPA2_LONG_ROPE)
+    s = bench.cpu_oracle_sample(cfg, target_s=0.5)
+    assert s["value"] > 0 and s["kind"] == "oracle" and s["cores"] >= 1
+    assert calls and len(calls) % 2 == 0          # q and k of every block timed
+
+
+def test_reference_arm_line(capsys):
+    class Args:
+        steps, warmup = 2, 1
+    cfg = synth.small_config(synth.LEVJEPA_VIT_L, frames=2, batch=1)
+    assert bench.run_reference(Args(), cfg, rank=0, world=1) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "tokens/s" and line["higher_is_better"] is True and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert line["ms_per_step"] == pytest.approx(1000.0 * cfg.n_tokens * cfg.batch / line["value"])
