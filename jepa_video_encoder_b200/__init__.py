@@ -24,8 +24,46 @@ def _stream_ptr(stream) -> Optional[int]:
     return stream.cuda_stream
 
 
-def _ptr(t) -> int:
+def _dptr(t) -> int:
+    """Device address of a CUDA tensor on the current device.  The library
+    takes raw pointers; a host tensor or another device's memory handed to a
+    kernel would be read as device memory, so both are refused here."""
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("expected a CUDA tensor, got " + (str(t.device) if isinstance(t, torch.Tensor) else
+                                                           type(t).__name__))
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensor on {t.device}, but the current device is cuda:{torch.cuda.current_device()}")
     return t.data_ptr()
+
+
+def check_pixels(cfg: "synth.EncoderConfig", pixels, on_cuda: bool, device: Optional[int] = None) -> int:
+    """Validate a pixel batch for encode / encode_host: float32, contiguous,
+    [B, frames, 3, img_h, img_w] with B >= 1, on a CUDA device (``device``)
+    or on the host.  Returns B."""
+    import torch
+    if not isinstance(pixels, torch.Tensor):
+        raise TypeError("pixels must be a torch.Tensor")
+    want = (cfg.frames, 3, cfg.img_h, cfg.img_w)
+    if pixels.dim() != 5 or tuple(pixels.shape[1:]) != want or pixels.shape[0] < 1:
+        raise ValueError(f"pixels must be [B, {', '.join(map(str, want))}], got {list(pixels.shape)}")
+    if pixels.dtype != torch.float32:
+        raise ValueError(f"pixels must be float32, got {pixels.dtype}")
+    if not pixels.is_contiguous():
+        raise ValueError("pixels must be contiguous")
+    if pixels.is_cuda != on_cuda or (on_cuda and device is not None and pixels.device.index != device):
+        raise ValueError(f"pixels on {pixels.device}; expected " + (f"cuda:{device}" if on_cuda else "the host"))
+    return int(pixels.shape[0])
+
+
+def check_out(out, on_cuda: bool, device: Optional[int] = None) -> None:
+    """A caller-supplied output: float32, contiguous, on the same side as the
+    pixels (its size is checked by the library against the pool mode)."""
+    import torch
+    if not isinstance(out, torch.Tensor) or out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous float32 tensor")
+    if out.is_cuda != on_cuda or (on_cuda and device is not None and out.device.index != device):
+        raise ValueError(f"out on {out.device}; expected " + (f"cuda:{device}" if on_cuda else "the host"))
 
 
 def make_config(cfg: "synth.EncoderConfig") -> _abi.Config:
@@ -108,10 +146,11 @@ class Model:
         output tensor (allocated if ``out`` is None).  Asynchronous."""
         import torch
         pool = self.cfg.pool if pool is None else pool
-        B = pixels.shape[0]
+        B = check_pixels(self.cfg, pixels, True, self.device)
         if out is None:
             out = torch.empty(self.out_shape(B, pool), dtype=torch.float32, device=pixels.device)
-        check(load_library().jepa_b200_encode(self._h, _ptr(pixels), B, POOLS[pool], _ptr(out),
+        check_out(out, True, self.device)
+        check(load_library().jepa_b200_encode(self._h, pixels.data_ptr(), B, POOLS[pool], out.data_ptr(),
                                               out.numel() * 4, _stream_ptr(stream)), "encode")
         return out
 
@@ -120,20 +159,22 @@ class Model:
         asynchronous copies) -> result in a CPU tensor.  Synchronous."""
         import torch
         pool = self.cfg.pool if pool is None else pool
-        B = pixels.shape[0]
+        B = check_pixels(self.cfg, pixels, False)
         if out is None:
             out = torch.empty(self.out_shape(B, pool), dtype=torch.float32, pin_memory=True)
-        check(load_library().jepa_b200_encode_host(self._h, _ptr(pixels), B, POOLS[pool], _ptr(out),
+        check_out(out, False)
+        check(load_library().jepa_b200_encode_host(self._h, pixels.data_ptr(), B, POOLS[pool], out.data_ptr(),
                                                    out.numel() * 4, _stream_ptr(stream)), "encode_host")
         return out
 
     def debug_stage(self, pixels, layer: int, out=None, stream=None):
         """Residual stream f32 [B, N, D] after patch-embed and ``layer`` blocks."""
         import torch
-        B = pixels.shape[0]
+        B = check_pixels(self.cfg, pixels, True, self.device)
         if out is None:
             out = torch.empty((B, self.cfg.n_tokens, self.cfg.dim), dtype=torch.float32, device=pixels.device)
-        check(load_library().jepa_b200_debug_stage(self._h, _ptr(pixels), B, layer, 0, _ptr(out),
+        check_out(out, True, self.device)
+        check(load_library().jepa_b200_debug_stage(self._h, pixels.data_ptr(), B, layer, 0, out.data_ptr(),
                                                    out.numel() * 4, _stream_ptr(stream)), "debug_stage")
         return out
 
@@ -165,51 +206,51 @@ def layernorm(x, gamma, beta, eps: float, out, in_row_stride: int = 1, rows: Opt
     D = x.shape[-1]
     rows = out.numel() // D if rows is None else rows
     dt = synth.DT_F16 if out.dtype == torch.float16 else synth.DT_F32
-    check(load_library().jepa_b200_op_layernorm(_ptr(x), rows, D, in_row_stride, _ptr(gamma), _ptr(beta), eps,
-                                                _ptr(out), dt, _stream_ptr(stream)), "layernorm")
+    check(load_library().jepa_b200_op_layernorm(_dptr(x), rows, D, in_row_stride, _dptr(gamma), _dptr(beta), eps,
+                                                _dptr(out), dt, _stream_ptr(stream)), "layernorm")
     return out
 
 
 def repack(dtype: int, blocks, N: int, K: int, qs, scales, stream=None):
-    check(load_library().jepa_b200_op_repack(dtype, _ptr(blocks), N, K, _ptr(qs), _ptr(scales),
+    check(load_library().jepa_b200_op_repack(dtype, _dptr(blocks), N, K, _dptr(qs), _dptr(scales),
                                              _stream_ptr(stream)), "repack")
 
 
 def dequant_f16(dtype: int, qs, scales, N: int, K: int, out, stream=None):
-    check(load_library().jepa_b200_op_dequant_f16(dtype, _ptr(qs), _ptr(scales), N, K, _ptr(out),
+    check(load_library().jepa_b200_op_dequant_f16(dtype, _dptr(qs), _dptr(scales), N, K, _dptr(out),
                                                   _stream_ptr(stream)), "dequant_f16")
     return out
 
 
 def linear(A, w, w_dtype: int, N: int, bias, epilogue: int, out, w_scales=None, stream=None):
     M, K = A.shape
-    check(load_library().jepa_b200_op_linear(_ptr(A), M, K, _ptr(w), _ptr(w_scales) if w_scales is not None else None,
-                                             w_dtype, N, _ptr(bias) if bias is not None else None, epilogue,
-                                             _ptr(out), out.shape[-1], _stream_ptr(stream)), "linear")
+    check(load_library().jepa_b200_op_linear(_dptr(A), M, K, _dptr(w), _dptr(w_scales) if w_scales is not None else None,
+                                             w_dtype, N, _dptr(bias) if bias is not None else None, epilogue,
+                                             _dptr(out), out.shape[-1], _stream_ptr(stream)), "linear")
     return out
 
 
 def linear_qkv(A, w, w_dtype: int, N: int, bias, ntok: int, heads: int, npad: int, first_part: int, q, k, vt,
                w_scales=None, stream=None):
     M, K = A.shape
-    f = lambda t: _ptr(t) if t is not None else None
-    check(load_library().jepa_b200_op_linear_qkv(_ptr(A), M, K, _ptr(w), f(w_scales), w_dtype, N, f(bias), ntok,
+    f = lambda t: _dptr(t) if t is not None else None
+    check(load_library().jepa_b200_op_linear_qkv(_dptr(A), M, K, _dptr(w), f(w_scales), w_dtype, N, f(bias), ntok,
                                                  heads, npad, first_part, f(q), f(k), f(vt), _stream_ptr(stream)),
           "linear_qkv")
 
 
 def attention(q, k, vt, B: int, heads: int, ntok: int, npad: int, mask: int, has_cls: int, ppf: int, out,
               stream=None):
-    check(load_library().jepa_b200_op_attention(_ptr(q), _ptr(k), _ptr(vt), B, heads, ntok, npad, mask, has_cls,
-                                                ppf, _ptr(out), _stream_ptr(stream)), "attention")
+    check(load_library().jepa_b200_op_attention(_dptr(q), _dptr(k), _dptr(vt), B, heads, ntok, npad, mask, has_cls,
+                                                ppf, _dptr(out), _stream_ptr(stream)), "attention")
     return out
 
 
 def patch_embed(pixels, patch: int, tubelet: int, w_pe, D: int, bias, pos, cls, has_cls: int, x, stream=None):
     B, T, _, H, W = pixels.shape
-    check(load_library().jepa_b200_op_patch_embed(_ptr(pixels), B, T, H, W, patch, tubelet, _ptr(w_pe), D,
-                                                  _ptr(bias) if bias is not None else None, _ptr(pos),
-                                                  _ptr(cls) if cls is not None else None, has_cls, _ptr(x),
+    check(load_library().jepa_b200_op_patch_embed(_dptr(pixels), B, T, H, W, patch, tubelet, _dptr(w_pe), D,
+                                                  _dptr(bias) if bias is not None else None, _dptr(pos),
+                                                  _dptr(cls) if cls is not None else None, has_cls, _dptr(x),
                                                   _stream_ptr(stream)), "patch_embed")
     return x
 
@@ -217,19 +258,19 @@ def patch_embed(pixels, patch: int, tubelet: int, w_pe, D: int, bias, pos, cls, 
 def gemv(x, w, w_dtype: int, N: int, bias, epi: int, y, resid=None, resid_row_stride: int = 0, w_scales=None,
          stream=None):
     M, K = x.shape
-    f = lambda t: _ptr(t) if t is not None else None
-    check(load_library().jepa_b200_op_gemv(_ptr(x), M, K, _ptr(w), f(w_scales), w_dtype, N, f(bias), epi, f(resid),
-                                           resid_row_stride, _ptr(y), _stream_ptr(stream)), "gemv")
+    f = lambda t: _dptr(t) if t is not None else None
+    check(load_library().jepa_b200_op_gemv(_dptr(x), M, K, _dptr(w), f(w_scales), w_dtype, N, f(bias), epi, f(resid),
+                                           resid_row_stride, _dptr(y), _stream_ptr(stream)), "gemv")
     return y
 
 
 def xattn_1q(q, k, vt, B: int, heads: int, ntok: int, npad: int, out, stream=None):
-    check(load_library().jepa_b200_op_xattn_1q(_ptr(q), _ptr(k), _ptr(vt), B, heads, ntok, npad, _ptr(out),
+    check(load_library().jepa_b200_op_xattn_1q(_dptr(q), _dptr(k), _dptr(vt), B, heads, ntok, npad, _dptr(out),
                                                _stream_ptr(stream)), "xattn_1q")
     return out
 
 
 def mean_pool(y, B: int, ntok: int, D: int, first: int, out, stream=None):
-    check(load_library().jepa_b200_op_mean_pool(_ptr(y), B, ntok, D, first, _ptr(out), _stream_ptr(stream)),
+    check(load_library().jepa_b200_op_mean_pool(_dptr(y), B, ntok, D, first, _dptr(out), _stream_ptr(stream)),
           "mean_pool")
     return out
