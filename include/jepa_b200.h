@@ -141,8 +141,10 @@ JEPA_B200_API int jepa_b200_load_weights(const jepa_b200_config *cfg, const jepa
  * Enqueued on `stream`; the model's workspace grows to the largest B seen
  * (that growth allocates and synchronises the device).  A model must not be
  * used by two calls that overlap in time.
- * Errors: ERR_ARG (null, B < 1, bad pool), ERR_SHAPE (out_bytes too small),
- * ERR_MISSING_TENSOR (ATTENTIVE without a head), ERR_CUDA. */
+ * Errors: ERR_ARG (null, B < 1, bad pool, CLS pool on a model without CLS,
+ * pixels or out not 16-byte aligned), ERR_SHAPE (out_bytes too small, or
+ * B * N above 524288 rows), ERR_MISSING_TENSOR (ATTENTIVE without a head),
+ * ERR_CUDA. */
 JEPA_B200_API int jepa_b200_encode(jepa_b200_model *m, const float *pixels, int B, int pool, float *out, size_t out_bytes,
                      void *stream);
 
