@@ -20,6 +20,7 @@ import hashlib
 import glob
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -137,17 +138,36 @@ _CLASS_SOURCES = {
 _GEMM_SOURCES = ("gemm.cu", "common.cuh", "internal.h")
 
 
+_C_TOKENS = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'', re.S)
+
+
+def code_text(src: str) -> str:
+    """C / C++ / CUDA source without its comments, each line stripped of
+    leading and trailing blanks, blank lines dropped: what a comment edit
+    leaves unchanged.  String and character literals are kept as they are."""
+    out = _C_TOKENS.sub(lambda m: " " if m.group(0)[0] == "/" else m.group(0), src)
+    return "\n".join(ln.strip() for ln in out.splitlines() if ln.strip())
+
+
+def hash_sources(texts) -> str:
+    h = hashlib.sha256()
+    for t in texts:
+        h.update(code_text(t).encode())
+        h.update(b"\0")
+    return h.hexdigest()[:16]
+
+
 def _src_hash(kernel_class=None):
     names = _CLASS_SOURCES.get(kernel_class, _GEMM_SOURCES if kernel_class and (
         kernel_class.startswith("gemm_") or kernel_class == "patch_embed") else None)
     csrc = os.path.join(ROOT, "jepa_video_encoder_b200", "csrc")
     paths = [os.path.join(csrc, n) for n in names] if names else sorted(glob.glob(os.path.join(csrc, "*")))
     paths.append(os.path.join(ROOT, "include", "jepa_b200.h"))
-    h = hashlib.sha256()
+    texts = []
     for path in paths:
-        with open(path, "rb") as f:
-            h.update(f.read())
-    return h.hexdigest()[:16]
+        with open(path, encoding="utf-8") as f:
+            texts.append(f.read())
+    return hash_sources(texts)
 
 
 def _traffic(kernel_class, cfg_name):

@@ -66,3 +66,18 @@ def test_reference_arm_line(capsys):
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert line["ms_per_step"] == pytest.approx(1000.0 * cfg.n_tokens * cfg.batch / line["value"])
+
+
+def test_source_hash_ignores_comments_not_code():
+    """A traffic figure stays tied to the kernel's code: comment and blank-line
+    edits keep the hash, any change of code or of a string literal (inline
+    PTX lives in string literals) changes it."""
+    src = ('// header\n#include "x.h"\n/* a\n   b */\n__global__ void k(int* p) {\n'
+           '  asm volatile("add.s32 %0, %0, 1; // x" : "+r"(*p));  // bump\n}\n')
+    h = bench.hash_sources([src])
+    assert bench.hash_sources([src.replace("// bump", "// incremented by one\n\n")]) == h
+    assert bench.hash_sources([src.replace("/* a\n   b */", "")]) == h
+    assert bench.hash_sources([src.replace("1;", "2;")]) != h                    # PTX in a literal
+    assert bench.hash_sources([src.replace("int* p", "long* p")]) != h
+    assert bench.hash_sources([src, ""]) != h                                    # file boundaries count
+    assert "//" in bench.code_text(src) and "bump" not in bench.code_text(src)  # '//' inside the literal kept
