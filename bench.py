@@ -218,8 +218,12 @@ def cpu_oracle_sample(cfg, target_s: float = 12.0):
     orc.layer_norm(x, W["enc.norm.weight"], W["enc.norm.bias"], cfg.ln_eps)
     t_norm = time.perf_counter() - t2
     t_clip = t_embed + cfg.depth * (t_blocks / blocks) + t_norm
+    try:
+        load1 = os.getloadavg()[0]
+    except OSError:
+        load1 = None
     return {"value": cfg.n_tokens / t_clip, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "clips_per_s": 1.0 / t_clip,
+            "clips_per_s": 1.0 / t_clip, "host_cpus": os.cpu_count(), "load_avg_1m": load1,
             "sample": f"1 clip: patch-embed + {blocks} of {cfg.depth} blocks + final norm in float64 numpy, "
                       f"block time extrapolated to {cfg.depth} blocks ({t_embed + t_blocks + t_norm:.1f} s of CPU work)"}
 
@@ -369,7 +373,9 @@ def run_ours(args, cfg, rank, world, local_rank):
     peak_dense = float(peaks.get("bf16_tflops"))
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
+        "ms_per_step_min": min(ms_steps), "ms_per_step_sd": statistics.pstdev(ms_steps),
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": {"workload": cfg.name, "batch_per_gpu": B, "global_batch": B * world,
                    "tokens_per_clip": cfg.n_tokens, "weights": cfg.weights, "mask": cfg.mask, "pool": cfg.pool,

@@ -155,6 +155,8 @@ def small_config(base: EncoderConfig, **kw) -> EncoderConfig:
              frames=min(base.frames, 4), batch=2, random_ln_affine=True)
     if base.tubelet == 2:
         d["frames"] = 4
+    if 64 % base.patch:   # keep the image a whole number of patches (LeWM's 14)
+        d["img_h"] = d["img_w"] = base.patch * (64 // base.patch)
     d.update(kw)
     return base.with_(name=base.name + "_small", **d)
 

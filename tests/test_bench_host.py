@@ -81,3 +81,10 @@ def test_source_hash_ignores_comments_not_code():
     assert bench.hash_sources([src.replace("int* p", "long* p")]) != h
     assert bench.hash_sources([src, ""]) != h                                    # file boundaries count
     assert "//" in bench.code_text(src) and "bump" not in bench.code_text(src)  # '//' inside the literal kept
+
+
+def test_small_configs_are_whole_patches():
+    for base in synth.WORKLOADS.values():
+        c = synth.small_config(base)
+        assert c.img_h % c.patch == 0 and c.img_w % c.patch == 0 and c.frames % c.tubelet == 0
+        assert c.n_patches == (c.frames // c.tubelet) * (c.img_h // c.patch) * (c.img_w // c.patch) > 0
