@@ -67,7 +67,8 @@ def _f16_bits_to_f64(lo: np.ndarray, hi: np.ndarray) -> np.ndarray:
 
 def dequant_q8_0(blocks: np.ndarray, n: int) -> np.ndarray:
     """q8_0: each 34-byte block = fp16 scale d, then 32 signed bytes q;
-    element value q*d."""
+    element value q*d ("Quantization" page, "File sizes": 8.5 bits per weight;
+    the dequant formula of the encoder pass)."""
     b = np.asarray(blocks, np.uint8).reshape(-1, 34)
     d = _f16_bits_to_f64(b[:, 0], b[:, 1])
     q = b[:, 2:].view(np.int8).astype(np.float64)
@@ -77,7 +78,8 @@ def dequant_q8_0(blocks: np.ndarray, n: int) -> np.ndarray:
 
 
 def dequant_q4_0(blocks: np.ndarray, n: int) -> np.ndarray:
-    """q4_0: each 18-byte block = fp16 scale d, then 16 bytes; byte j carries
+    """q4_0 ("Quantization" page, "File sizes": 4.5 bits per weight; value
+    (q-8)*d): each 18-byte block = fp16 scale d, then 16 bytes; byte j carries
     element j (low nibble) and element j+16 (high nibble); value (q-8)*d."""
     b = np.asarray(blocks, np.uint8).reshape(-1, 18)
     d = _f16_bits_to_f64(b[:, 0], b[:, 1])
@@ -126,7 +128,9 @@ def patchify(pixels: np.ndarray, patch: int, tubelet: int) -> np.ndarray:
 
 
 def patch_embed(pixels, w_pe, b_pe, patch, tubelet) -> np.ndarray:
-    """Conv3d with stride = kernel = (kt, p, p) written as unfold + matmul."""
+    """Conv3d with stride = kernel = (kt, p, p) written as unfold + matmul
+    (the cards' patch 16 / tubelet 1 or 2 embedding; the benchmarks page,
+    "What the milliseconds are", unfolds patches before the graph)."""
     cols = patchify(pixels, patch, tubelet)
     D = w_pe.shape[0]
     return cols @ w_pe.reshape(D, -1).T + b_pe
@@ -134,7 +138,8 @@ def patch_embed(pixels, w_pe, b_pe, patch, tubelet) -> np.ndarray:
 
 def layer_norm(x: np.ndarray, gamma, beta, eps: float) -> np.ndarray:
     """(x - mean) / sqrt(var + eps) * gamma + beta over the last axis, with
-    the biased variance."""
+    the biased variance: the ln1 / ln2 / norm tensors of the "Quantization"
+    page, "The rule" (eps is a reading: the pages give none)."""
     x = np.asarray(x, np.float64)
     mu = x.mean(axis=-1, keepdims=True)
     var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
@@ -142,7 +147,9 @@ def layer_norm(x: np.ndarray, gamma, beta, eps: float) -> np.ndarray:
 
 
 def gelu(x: np.ndarray) -> np.ndarray:
-    """Exact GELU: x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2))."""
+    """Exact GELU: x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2)), the activation
+    between ffn_up and ffn_down (the pages name no variant; the erf form is
+    the reading taken)."""
     return 0.5 * x * (1.0 + _erf(x / math.sqrt(2.0)))
 
 
@@ -159,7 +166,8 @@ def allowed_keys(n_patches: int, patches_per_slot: int, has_cls: bool,
     bidir: every pair.  block_causal (LeVJEPA): a patch of time slot s reads
     the patches of slots <= s (bidirectional inside a slot, causal across
     slots); the CLS row, when present, reads every token including itself and
-    no patch reads CLS (the read-only sink)."""
+    no patch reads CLS (the read-only sink) -- "LeVJEPA ViT-L/16 (VideoMix)"
+    card, intro."""
     c = 1 if has_cls else 0
     N = n_patches + c
     if mask == "bidir":
@@ -221,7 +229,8 @@ def rope_positions(cfg) -> np.ndarray:
 
 
 def rope(x: np.ndarray, pos: np.ndarray, base: float = ROPE_BASE) -> np.ndarray:
-    """Rotate the head vectors x [..., N, d_h] of tokens at positions pos [N, 3]."""
+    """Rotate the head vectors x [..., N, d_h] of tokens at positions pos [N, 3]
+    (the 3-D rotary scheme read above for the V-JEPA 2 encoders)."""
     d = x.shape[-1]
     g = 2 * (d // 6)
     out = np.array(x, np.float64, copy=True)
@@ -238,7 +247,8 @@ def rope(x: np.ndarray, pos: np.ndarray, base: float = ROPE_BASE) -> np.ndarray:
 
 def block(x, W: Dict[str, np.ndarray], prefix: str, heads: int, eps: float,
           allow: Optional[np.ndarray], rope_pos: Optional[np.ndarray] = None) -> np.ndarray:
-    """One pre-LN transformer block.  attn_qkv's output columns are
+    """One pre-LN transformer block ("Quantization" page, "The rule": ln1,
+    attn_qkv, attn_out, ln2, ffn_up, ffn_down).  attn_qkv's output columns are
     [q | k | v], each head-major (head hd at hd*d_h ...).  With rope_pos, q and
     k are rotated (after their bias) before the attention."""
     D = x.shape[-1]
@@ -256,7 +266,9 @@ def block(x, W: Dict[str, np.ndarray], prefix: str, heads: int, eps: float,
 
 def embed(cfg, W, pixels) -> np.ndarray:
     """Patch-embed, prepend CLS (when the model has one), add pos_embed (the
-    rotary models have none: their positions enter the attention)."""
+    rotary models have none: their positions enter the attention); the
+    enc.cls_token / enc.pos_embed tensors of the "Quantization" page, "The
+    rule"."""
     x = patch_embed(pixels, W["enc.patch_embed.weight"], W["enc.patch_embed.bias"],
                     cfg.patch, cfg.tubelet)
     if cfg.has_cls:
@@ -276,7 +288,8 @@ def encoder_allow(cfg) -> Optional[np.ndarray]:
 def encoder(cfg, W, pixels, layers: Optional[int] = None,
             return_residuals: bool = False):
     """Full encoder: embed, ``depth`` blocks, final LayerNorm ->
-    last_hidden_state [B, N, D]."""
+    last_hidden_state [B, N, D] (the final ``norm``: "Quantization" page,
+    "Reading the numbers")."""
     allow = encoder_allow(cfg)
     rope_pos = rope_positions(cfg) if getattr(cfg, "rope", False) else None
     x = embed(cfg, W, pixels)
@@ -290,7 +303,8 @@ def encoder(cfg, W, pixels, layers: Optional[int] = None,
 
 def pool(cfg, y: np.ndarray, mode: str) -> np.ndarray:
     """cls: the CLS row; mean: mean over the patch tokens (CLS excluded);
-    none: the full token map."""
+    none: the full token map ("LeVJEPA" card, "Run it": --pool; which tokens
+    the mean covers is a reading)."""
     if mode == "none":
         return y
     if mode == "cls":
@@ -307,7 +321,11 @@ def attentive_head(cfg, W, tokens: np.ndarray) -> np.ndarray:
     blocks over the tokens, then one cross-attention block whose single query
     is the learned ``head.query`` (not normalised): q = W_q query + b_q;
     k, v = W_{k,v} LN_kv(tokens) + b; z = query + W_out attn + b_out;
-    z += MLP(LN2(z)); logits = W_cls z + b_cls."""
+    z += MLP(LN2(z)); logits = W_cls z + b_cls ("jepa.cpp — measured
+    benchmarks", "Attentive-pool head": three self-attention blocks, one
+    cross-attention query, MLP, linear; the tensors, head.query, ln_kv,
+    head.xattn.{q,k,v,ffn_up,ffn_down} and head.cls, from the "Quantization"
+    page, "The rule"; the cross-attention out-projection is a reading)."""
     x = tokens
     for i in range(cfg.head_sa_blocks):
         x = block(x, W, f"head.blk.{i}.", cfg.heads, cfg.ln_eps, None)
