@@ -28,8 +28,8 @@ matmul as the only primitive), in the order the pages describe the model:
   cross-attention query, MLP, linear ("jepa.cpp — measured benchmarks",
   "Attentive-pool head");
 * q8_0 / q4_0 dequantisation: value = q*d and (q-8)*d per 32-element block
-  with one fp16 scale ("Quantization" page, "File sizes": 8.5 / 4.5 bits per
-  weight).
+  with one fp16 scale (ggml's published block formats; the "Quantization"
+  page, "File sizes", gives their 8.5 / 4.5 bits per weight).
 
 Readings where the pages are silent (LayerNorm eps, exact-erf GELU, 1/sqrt(d_h)
 scale, qkv column order, mean pooling over patch tokens only, the head's
@@ -67,8 +67,9 @@ def _f16_bits_to_f64(lo: np.ndarray, hi: np.ndarray) -> np.ndarray:
 
 def dequant_q8_0(blocks: np.ndarray, n: int) -> np.ndarray:
     """q8_0: each 34-byte block = fp16 scale d, then 32 signed bytes q;
-    element value q*d ("Quantization" page, "File sizes": 8.5 bits per weight;
-    the dequant formula of the encoder pass)."""
+    element value q*d (ggml's published q8_0 block format; its 34 bytes per
+    32 weights are the 8.5 bits per weight of the "Quantization" page, "File
+    sizes")."""
     b = np.asarray(blocks, np.uint8).reshape(-1, 34)
     d = _f16_bits_to_f64(b[:, 0], b[:, 1])
     q = b[:, 2:].view(np.int8).astype(np.float64)
@@ -78,8 +79,9 @@ def dequant_q8_0(blocks: np.ndarray, n: int) -> np.ndarray:
 
 
 def dequant_q4_0(blocks: np.ndarray, n: int) -> np.ndarray:
-    """q4_0 ("Quantization" page, "File sizes": 4.5 bits per weight; value
-    (q-8)*d): each 18-byte block = fp16 scale d, then 16 bytes; byte j carries
+    """q4_0 (ggml's published block format, value (q-8)*d; 18 bytes per 32
+    weights = the 4.5 bits per weight of the "Quantization" page, "File
+    sizes"): each 18-byte block = fp16 scale d, then 16 bytes; byte j carries
     element j (low nibble) and element j+16 (high nibble); value (q-8)*d."""
     b = np.asarray(blocks, np.uint8).reshape(-1, 18)
     d = _f16_bits_to_f64(b[:, 0], b[:, 1])
