@@ -58,7 +58,8 @@ typedef enum {
   JEPA_B200_ERR_UNSUPPORTED = -7     /* valid request this build does not implement */
 } jepa_b200_status;
 
-/* Tensor dtypes use ggml's type ids ("Quantization" page, "The rule"). */
+/* Tensor dtypes use ggml's type ids (0 f32, 1 f16, 2 q4_0, 8 q8_0), the
+ * numbering of the GGUF files the pages describe. */
 typedef enum {
   JEPA_B200_F32 = 0,
   JEPA_B200_F16 = 1,
@@ -248,7 +249,8 @@ JEPA_B200_API int jepa_b200_op_repack(int dtype, const void *blocks, int N, int 
  * writes): element (n, k) = q * d (q8_0) or (q - 8) * d (q4_0), d the fp16
  * scale of its 32-element block, the exact product rounded once to f16 --
  * the values the GEMM's loader unpack produces, made once for GEMMs with many
- * rows ("Quantization" page, "The rule": the dequantisation formula).
+ * rows (ggml's q8_0 / q4_0 block formats; which matrices carry them:
+ * "Quantization" page, "The rule").
  * K % 32 == 0; out 16-byte aligned.  Errors: ERR_ARG, ERR_DTYPE, ERR_SHAPE. */
 JEPA_B200_API int jepa_b200_op_dequant_f16(int dtype, const void *qs, const void *scales, int N, int K, void *out,
                                            void *stream);
