@@ -210,8 +210,9 @@ def merge_heads(x):
 
 
 # ---------------------------------------------------------------------------
-# 3-D rotary position embedding of the V-JEPA 2 encoders (the V-JEPA 2 card
-# and the "Quantization" page's check list name an "encoder with 3-D RoPE";
+# 3-D rotary position embedding of the V-JEPA 2 encoders (the "Quantization"
+# page, "How the accuracy was measured", says that reference graph's encoder
+# uses 3-D rotary embeddings;
 # the pages give no formula, so the plainest 3-D extension of rotary
 # embeddings is read here): the head dimensions are split into three groups
 # of g = 2*floor(d_h/6), one per axis (time slot, patch row, patch column);
