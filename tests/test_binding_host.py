@@ -69,3 +69,12 @@ def test_op_wrappers_refuse_host_tensors():
     with pytest.raises(ValueError):
         jb.linear(torch.zeros(4, 64, dtype=torch.float16), torch.zeros(128, 64, dtype=torch.float16),
                   synth.DT_F16, 128, None, 0, torch.zeros(4, 128))
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without the built library nothing computes: loading it raises with the
+    build command instead of falling back to anything."""
+    from jepa_video_encoder_b200 import _abi
+    monkeypatch.setattr(_abi, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        _abi.load_library(str(tmp_path / "libjepa_b200.so"))
