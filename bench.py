@@ -186,9 +186,11 @@ def _traffic(kernel_class, cfg_name):
     return None
 
 
-def cpu_oracle_sample(cfg, target_s: float = 12.0):
+def cpu_oracle_sample(cfg, target_s: float = 12.0, table=None):
     """Time the float64 oracle on a bounded sample of one clip: patch-embed
-    and as many blocks as fit in ~target_s, extrapolated to the full depth."""
+    and as many blocks as fit in ~target_s, extrapolated to the full depth.
+    ``table`` (a table_dict of the workload) saves regenerating the inputs
+    when the sample is repeated; generating them is not timed either way."""
     import numpy as np
     from oracle import jepa_oracle as orc
     try:
@@ -196,7 +198,8 @@ def cpu_oracle_sample(cfg, target_s: float = 12.0):
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
         cores = os.cpu_count() or 1
-    table = synth.table_dict(synth.make_tensor_table(cfg))
+    if table is None:
+        table = synth.table_dict(synth.make_tensor_table(cfg))
     pix = synth.make_pixels(cfg, batch=1).astype(np.float64)
     names = [n for n in table if not n.startswith("enc.blk.") and not n.startswith("head.")]
     W = {n: orc.tensor_f64(table[n]) for n in names}
@@ -234,8 +237,9 @@ def run_reference(args, cfg, rank, world):
         return 0
     steps = []
     sample = None
+    table = synth.table_dict(synth.make_tensor_table(cfg))   # the inputs, generated once
     for _ in range(max(1, args.steps)):
-        sample = cpu_oracle_sample(cfg, target_s=max(2.0, 60.0 / max(1, args.steps)))
+        sample = cpu_oracle_sample(cfg, target_s=max(2.0, 60.0 / max(1, args.steps)), table=table)
         steps.append(sample["value"])
     v = statistics.median(steps)
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
