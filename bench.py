@@ -232,6 +232,13 @@ def cpu_oracle_sample(cfg, target_s: float = 12.0, table=None):
                       f"block time extrapolated to {cfg.depth} blocks ({t_embed + t_blocks + t_norm:.1f} s of CPU work)"}
 
 
+def run_config(cfg, world: int, l2: str) -> dict:
+    """The workload a line measures; both arms report the same keys."""
+    return {"workload": cfg.name, "batch_per_gpu": cfg.batch, "global_batch": cfg.batch * world,
+            "tokens_per_clip": cfg.n_tokens, "weights": cfg.weights, "mask": cfg.mask, "pool": cfg.pool,
+            "parallelism": f"replicas x{world}", "l2": l2}
+
+
 def run_reference(args, cfg, rank, world):
     if rank != 0:
         return 0
@@ -245,7 +252,7 @@ def run_reference(args, cfg, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * cfg.n_tokens * cfg.batch / v,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg.name, "batch": cfg.batch, "tokens_per_clip": cfg.n_tokens},
+            "config": run_config(cfg, world, l2="not applicable (host CPU run)"),
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": sample["cores"], "kind": "oracle",
                              "sample": sample["sample"]},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -382,9 +389,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         "ms_per_step_min": min(ms_steps), "ms_per_step_sd": statistics.pstdev(ms_steps),
         "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {"workload": cfg.name, "batch_per_gpu": B, "global_batch": B * world,
-                   "tokens_per_clip": cfg.n_tokens, "weights": cfg.weights, "mask": cfg.mask, "pool": cfg.pool,
-                   "parallelism": f"replicas x{world}", "l2": "flushed between steps (256 MiB write)"},
+        "config": run_config(cfg, world, l2="flushed between steps (256 MiB write)"),
         "clips_per_s": world * B * args.steps / (total_ms / 1000.0),
         "tflops": tflops, "tc_peak_frac": tflops / peak_dense,
         "tc_peak": {"value": peak_dense, "source": f"{peak_src} bf16 burst"},

@@ -88,3 +88,12 @@ def test_small_configs_are_whole_patches():
         c = synth.small_config(base)
         assert c.img_h % c.patch == 0 and c.img_w % c.patch == 0 and c.frames % c.tubelet == 0
         assert c.n_patches == (c.frames // c.tubelet) * (c.img_h // c.patch) * (c.img_w // c.patch) > 0
+
+
+def test_both_arms_report_the_same_config_keys():
+    cfg = synth.LEVJEPA_VIT_L
+    a = bench.run_config(cfg, 1, l2="flushed")
+    b = bench.run_config(cfg, 1, l2="not applicable")
+    assert set(a) == set(b) and {k: v for k, v in a.items() if k != "l2"} == {k: v for k, v in b.items() if k != "l2"}
+    assert a["workload"] == cfg.name and a["global_batch"] == cfg.batch
+    assert bench.run_config(cfg, 4, l2="x")["global_batch"] == 4 * cfg.batch
