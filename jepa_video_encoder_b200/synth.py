@@ -107,8 +107,9 @@ class EncoderConfig:
 
 
 # ---------------------------------------------------------------------------
-# The five workloads (model cards: LeWorldModel Push-T, LeVJEPA ViT-L/16,
-# V-JEPA 2 ViT-L/16 SSv2 classifier; benchmarks page: 64-frame long clip).
+# The five model configurations (model cards: LeWorldModel Push-T, LeVJEPA
+# ViT-L/16, V-JEPA 2 ViT-L/16 SSv2 classifier; benchmarks page: 64-frame long
+# clip), then the batch sweeps and rotary variants built from them.
 # ---------------------------------------------------------------------------
 LEWM_VIT_TI = EncoderConfig(
     name="lewm_vit_ti14_224_b1", dim=192, depth=12, heads=3, mlp=768, patch=14,
