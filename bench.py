@@ -88,19 +88,53 @@ def _flops(cfg) -> dict:
     return f
 
 
+_CLOCK_FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
 def _clock_sampler_start(path):
-    q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     try:
         f = open(path, "w")
-        return subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200"],
-                                stdout=f, stderr=subprocess.DEVNULL), f
+        return subprocess.Popen(["nvidia-smi", f"--query-gpu={_CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                                 "-lms", "50"], stdout=f, stderr=subprocess.DEVNULL), f
     except Exception:
         return None, None
 
 
-def _clock_sampler_stop(proc, fh, path, gpu_index):
+def parse_clock_log(path, gpu_index, t0=None, t1=None):
+    """Median SM clock, max clock and the throttle reasons seen in an nvidia-smi
+    log of _CLOCK_FIELDS.  With t0 / t1 (host epoch seconds) only the samples
+    taken inside [t0, t1] count; if none falls inside, all of them do and
+    ``in_region`` says so."""
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    rows = []
+    for line in open(path):
+        parts = [q.strip() for q in line.split(",")]
+        if len(parts) < 10 or parts[1] != str(gpu_index):
+            continue
+        try:
+            sm, mx = float(parts[2]), float(parts[3])
+        except ValueError:
+            continue
+        ts = None  # a sample whose time cannot be read still counts in the fallback
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                ts = datetime.datetime.strptime(parts[0], fmt).timestamp()
+                break
+            except ValueError:
+                pass
+        rows.append((ts, sm, mx, [n for n, v in zip(names, parts[6:10]) if v.lower() == "active"]))
+    if not rows:
+        return None
+    inside = [r for r in rows if t0 is not None and t1 is not None and r[0] is not None and t0 <= r[0] <= t1]
+    use = inside or rows
+    return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+            "reasons": sorted({n for r in use for n in r[3]}), "samples": len(use),
+            "in_region": bool(inside)}
+
+
+def _clock_sampler_stop(proc, fh, path, gpu_index, t0=None, t1=None):
     if proc is None:
         return None
     proc.terminate()
@@ -109,24 +143,7 @@ def _clock_sampler_stop(proc, fh, path, gpu_index):
     except Exception:
         proc.kill()
     fh.close()
-    sm, mx, reasons = [], [], set()
-    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-    for line in open(path):
-        parts = [p.strip() for p in line.split(",")]
-        if len(parts) < 9 or parts[0] != str(gpu_index):
-            continue
-        try:
-            sm.append(float(parts[1]))
-            mx.append(float(parts[2]))
-        except ValueError:
-            continue
-        for n, v in zip(names, parts[5:9]):
-            if v.lower() == "active":
-                reasons.add(n)
-    if not sm:
-        return None
-    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-            "samples": len(sm)}
+    return parse_clock_log(path, gpu_index, t0, t1)
 
 
 # The sources each kernel class is compiled from: a traffic figure stays valid
@@ -306,6 +323,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     proc, fh = _clock_sampler_start(clock_path)
     time.sleep(0.3)
     launches = 0
+    t_region0 = time.time()
     for k in range(args.steps):
         flush.zero_()
         ev[k][0].record(stream)
@@ -313,7 +331,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         ev[k][1].record(stream)
         launches += model.last_launch_count()
     torch.cuda.synchronize(dev)
-    clocks = _clock_sampler_stop(proc, fh, clock_path, local_rank)
+    t_region1 = time.time()
+    clocks = _clock_sampler_stop(proc, fh, clock_path, local_rank, t_region0, t_region1)
     if world > 1:
         torch.distributed.barrier()
     if model.sync_status(stream) != 0:

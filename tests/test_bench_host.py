@@ -97,3 +97,28 @@ def test_both_arms_report_the_same_config_keys():
     assert set(a) == set(b) and {k: v for k, v in a.items() if k != "l2"} == {k: v for k, v in b.items() if k != "l2"}
     assert a["workload"] == cfg.name and a["global_batch"] == cfg.batch
     assert bench.run_config(cfg, 4, l2="x")["global_batch"] == 4 * cfg.batch
+
+
+def test_clock_log_keeps_the_timed_region(tmp_path):
+    """Only samples taken inside the timed region count; throttle reasons are
+    read per sample; other GPUs' lines are ignored; without any sample inside,
+    all of them count and the record says so."""
+    import datetime as dt
+    base = dt.datetime(2026, 12, 2, 22, 0, 0)
+    def line(sec, gpu, sm, reasons=("Not Active",) * 4):
+        ts = (base + dt.timedelta(seconds=sec)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return f"{ts}, {gpu}, {sm}, 1965, 700.5, 0x0, " + ", ".join(reasons) + "\n"
+    log = tmp_path / "clocks.csv"
+    log.write_text(line(0.0, 0, 345) + line(0.5, 0, 1900) + line(0.55, 1, 100) +
+                   line(0.6, 0, 1950, ("Not Active", "Not Active", "Not Active", "Active")) +
+                   line(0.7, 0, 1965) + line(1.5, 0, 400))
+    t0 = (base + dt.timedelta(seconds=0.45)).timestamp()
+    t1 = (base + dt.timedelta(seconds=0.75)).timestamp()
+    c = bench.parse_clock_log(str(log), 0, t0, t1)
+    assert c == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3,
+                 "in_region": True}
+    c = bench.parse_clock_log(str(log), 0, t1 + 10, t1 + 20)
+    assert c["samples"] == 5 and c["in_region"] is False
+    log.write_text("garbled, 0, 1800, 1965, 1, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+    c = bench.parse_clock_log(str(log), 0, t0, t1)
+    assert c["samples"] == 1 and c["sm_mhz"] == 1800.0 and c["in_region"] is False
