@@ -130,6 +130,8 @@ typedef struct jepa_b200_model jepa_b200_model;
  * head's few-row kernels) and also dequantised once, on the device, to f16
  * (each q*d or (q-8)*d rounded once: the values the loader unpack produces),
  * which the GEMMs with 256 or more rows use.
+ * Names the model does not use (a predictor's, say) are ignored; a name given
+ * twice is ERR_ARG.
  * On success *out_model owns its device memory until jepa_b200_free.
  * Errors: ERR_ARG, ERR_MISSING_TENSOR, ERR_SHAPE, ERR_DTYPE, ERR_CUDA. */
 JEPA_B200_API int jepa_b200_load_weights(const jepa_b200_config *cfg, const jepa_b200_tensor *table, int n_tensors, int device,

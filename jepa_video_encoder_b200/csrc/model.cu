@@ -759,7 +759,11 @@ int jepa_b200_load_weights(const jepa_b200_config* cfg, const jepa_b200_tensor* 
     Loader V;
     V.m = &probe;
     V.dry = true;
-    for (int i = 0; i < n_tensors; ++i) V.tab[table[i].name] = &table[i];
+    for (int i = 0; i < n_tensors; ++i)
+      if (!V.tab.emplace(table[i].name, &table[i]).second) {  // a name given twice
+        delete m;
+        return JEPA_B200_ERR_ARG;
+      }
     load_sequence(V);
     if (V.status != JEPA_B200_OK) {
       delete m;

@@ -109,6 +109,17 @@ def test_table_validation(lib):
     assert _load(lib, cfg, bad) == _abi.ERR_SHAPE
 
 
+def test_duplicate_and_extra_names(lib):
+    cfg = _tiny_cfg()
+    table = synth.make_tensor_table(cfg)
+    ok = 0 if _has_gpu() else _abi.ERR_CUDA
+    dup = list(table) + [table[3]]
+    assert _load(lib, cfg, dup) == _abi.ERR_ARG                      # a name given twice
+    extra = list(table) + [synth.Tensor("pred.blk.0.ln1.weight", synth.DT_F32, (cfg.dim,),
+                                        np.ones(cfg.dim, np.float32))]
+    assert _load(lib, cfg, extra) == ok                               # unused names are ignored
+
+
 def test_quantised_table_validation(lib):
     cfg = _tiny_cfg(weights="q8_0")
     table = synth.make_tensor_table(cfg)
