@@ -318,8 +318,8 @@ JEPA_B200_API int jepa_b200_op_xattn_1q(const float *q, const void *k, const voi
 JEPA_B200_API int jepa_b200_op_mean_pool(const float *y, int B, int ntok, int D, int first, float *out, void *stream);
 
 /* Mean pooling that allocates nothing, for callers that cannot call
- * cudaMalloc (work recorded into a CUDA graph, serving loops under a fixed
- * device-memory budget or that must not synchronise the device, hosts whose
+ * cudaMalloc (serving loops under a fixed device-memory budget, code that
+ * must not stall the device, which cudaMalloc may synchronise, hosts whose
  * allocator belongs to another framework).  There is no counterpart on the
  * pages: it is jepa_b200_op_mean_pool with its partial sums kept in a fixed
  * file-scope device array (4 MiB on every GPU that loads the library, held

@@ -686,14 +686,8 @@ template <bool ROWS_IN_WARP, int TILES>
 static int attn_launch_impl(const AttnParams& p, const AttnOp& op, cudaStream_t st) {
   using C = AttnCfg<TILES>;
   auto kern = attn_fwd_kernel<ROWS_IN_WARP, TILES>;
-  static unsigned long long attr_done = 0;  // one bit per device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !((attr_done >> dev) & 1ull)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) != cudaSuccess)
-      return JEPA_B200_ERR_CUDA;
-    attr_done |= 1ull << dev;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  if (!smem_attr_once(attr_done, kern, C::kSmem)) return JEPA_B200_ERR_CUDA;
   const int units = TILES == 2 ? (p.n_q_tiles + 1) / 2 + (p.cls_separate && !p.cls_in_pair ? 1 : 0)
                                : p.n_q_tiles + (p.cls_separate && !p.cls_tail ? 1 : 0);
   const dim3 grid = p.mask == JEPA_B200_MASK_BLOCK_CAUSAL ? dim3(op.B * p.heads, units) : dim3(units, op.B * p.heads);

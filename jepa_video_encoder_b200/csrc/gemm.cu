@@ -975,14 +975,15 @@ __global__ void __launch_bounds__(320, 1)
 
 // ------------------------------------------------------------------ host --
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  // resolved once (a function-local static is initialised by one thread)
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void* f = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -1018,11 +1019,11 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, int esize, uint64_t cols, ui
 int num_sms() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
-  static int cache[64] = {0};
-  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  static std::atomic<int> cache[64] = {};
+  if (dev >= 0 && dev < 64 && (n = cache[dev].load(std::memory_order_relaxed)) > 0) return n;
   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   if (n <= 0) n = 148;
-  if (dev >= 0 && dev < 64) cache[dev] = n;
+  if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -1121,14 +1122,8 @@ int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& Win
 template <int BN, int BMODE, bool GATHER, bool ROPE = false>
 static int launch_impl(const GemmOp& op, cudaStream_t st) {
   auto kern = gemm_tc_kernel<BN, BMODE, GATHER, ROPE>;
-  static unsigned long long attr_done = 0;  // one bit per device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !((attr_done >> dev) & 1ull)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<BN>::SMEM) != cudaSuccess)
-      return JEPA_B200_ERR_CUDA;
-    attr_done |= 1ull << dev;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  if (!smem_attr_once(attr_done, kern, GemmCfg<BN>::SMEM)) return JEPA_B200_ERR_CUDA;
   constexpr int threads = (BMODE != B_F16 || GATHER) ? 448 : 320;
   if (launch_pdl(kern, dim3(op.grid), dim3(threads), GemmCfg<BN>::SMEM, st, 1, op.tmA, op.tmB, op.tmC, op.tmC2, op.p) !=
       cudaSuccess)
@@ -1139,14 +1134,8 @@ static int launch_impl(const GemmOp& op, cudaStream_t st) {
 template <int BN, bool ROPE = false>
 static int launch_pair(const GemmOp& op, cudaStream_t st) {
   auto kern = gemm_pair_kernel<BN, ROPE>;
-  static unsigned long long attr_done = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !((attr_done >> dev) & 1ull)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Gemm2Cfg<BN>::SMEM) != cudaSuccess)
-      return JEPA_B200_ERR_CUDA;
-    attr_done |= 1ull << dev;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  if (!smem_attr_once(attr_done, kern, Gemm2Cfg<BN>::SMEM)) return JEPA_B200_ERR_CUDA;
   if (launch_pdl(kern, dim3(op.grid), dim3(320), Gemm2Cfg<BN>::SMEM, st, 2, op.tmA, op.tmB, op.tmC, op.tmC2, op.p) !=
       cudaSuccess)
     return JEPA_B200_ERR_CUDA;

@@ -115,17 +115,12 @@ int launch_gemv(const float* x, int M, int K, const DevMatrix& W, const float* b
   while (rows_per > 1 && static_cast<size_t>(rows_per) * K * 4 > 200 * 1024) rows_per >>= 1;
   if (static_cast<size_t>(K) * 4 > 200 * 1024) return JEPA_B200_ERR_SHAPE;
   const int smem_max = rows_per * K * 4;
-  static unsigned long long attr_done[3] = {0, 0, 0};
-  int dev = 0;
-  cudaGetDevice(&dev);
+  static std::atomic<unsigned long long> attr_done[3] = {};
   const int bm = W.bmode == B_Q8 ? 1 : (W.bmode == B_Q4 ? 2 : 0);
-  if (dev < 64 && !((attr_done[bm] >> dev) & 1ull)) {
-    cudaError_t e = bm == 1 ? cudaFuncSetAttribute(gemv_kernel<B_Q8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024)
-                  : bm == 2 ? cudaFuncSetAttribute(gemv_kernel<B_Q4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024)
-                            : cudaFuncSetAttribute(gemv_kernel<B_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    if (e != cudaSuccess) return JEPA_B200_ERR_CUDA;
-    attr_done[bm] |= 1ull << dev;
-  }
+  const bool attr_ok = bm == 1   ? smem_attr_once(attr_done[1], gemv_kernel<B_Q8>, 200 * 1024)
+                       : bm == 2 ? smem_attr_once(attr_done[2], gemv_kernel<B_Q4>, 200 * 1024)
+                                 : smem_attr_once(attr_done[0], gemv_kernel<B_F16>, 200 * 1024);
+  if (!attr_ok) return JEPA_B200_ERR_CUDA;
   (void)smem_max;
   for (int m0 = 0; m0 < M; m0 += rows_per) {
     const int mc = std::min(rows_per, M - m0);
@@ -212,14 +207,8 @@ int launch_xattn_1q(const float* q, const __half* k, const __half* vt, int B, in
   if (!q || !k || !vt || !out) return JEPA_B200_ERR_ARG;
   if (B < 1 || heads < 1 || ntok < 1 || ntok > 16384 || npad < ntok) return JEPA_B200_ERR_SHAPE;
   const size_t smem = static_cast<size_t>(ntok) * 4;
-  static unsigned long long attr_done = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !((attr_done >> dev) & 1ull)) {
-    if (cudaFuncSetAttribute(xattn_1q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 16384 * 4) != cudaSuccess)
-      return JEPA_B200_ERR_CUDA;
-    attr_done |= 1ull << dev;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  if (!smem_attr_once(attr_done, xattn_1q_kernel, 16384 * 4)) return JEPA_B200_ERR_CUDA;
   launch_pdl(xattn_1q_kernel, dim3(B * heads), dim3(256), smem, st, 1, q, k, vt, heads, ntok, npad, out);
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/jepa_b200.h"
 #include "common.cuh"
 
@@ -138,6 +140,21 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, int esize, uint64_t cols, ui
                   uint32_t box_cols, uint32_t box_rows);
 
 int num_sms();
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` once per device.
+// `done` holds one bit per device (0..63); the entry points may be called
+// from several host threads, so the bit is read and set atomically (two
+// threads that race both set the attribute, which is harmless).
+template <typename Kern>
+inline bool smem_attr_once(std::atomic<unsigned long long>& done, Kern kern, int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const unsigned long long bit = dev >= 0 && dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  if (bit) done.fetch_or(bit, std::memory_order_release);
+  return true;
+}
 
 // Launch with programmatic stream serialization (and, cluster_x > 1, thread
 // block clusters of cluster_x CTAs): the kernel calls pdl_wait() before

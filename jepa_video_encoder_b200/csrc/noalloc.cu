@@ -2,9 +2,8 @@
 //
 // jepa_b200_op_mean_pool needs a scratch buffer for its partial column sums
 // and grows one with cudaMalloc on demand.  Some callers cannot do that:
-// code that records work into a CUDA graph (cudaMalloc is not a stream
-// operation and synchronises the device), serving loops that run under a
-// fixed device-memory budget or must never stall the device, and hosts whose
+// serving loops that run under a fixed device-memory budget, code that must
+// never stall the device (cudaMalloc may synchronise it), and hosts whose
 // device allocator belongs to another framework.  For them this file keeps
 // the scratch in a fixed file-scope __device__ array that every GPU loading
 // the library holds until the process exits, and exposes

@@ -31,10 +31,12 @@ matmul as the only primitive), in the order the pages describe the model:
   with one fp16 scale (ggml's published block formats; the "Quantization"
   page, "File sizes", gives their 8.5 / 4.5 bits per weight).
 
-Readings where the pages are silent (LayerNorm eps, exact-erf GELU, 1/sqrt(d_h)
-scale, qkv column order, mean pooling over patch tokens only, the head's
-cross-attention out-projection) are listed in the design notes and are passed
-in through the config.
+Where the pages are silent this module takes the plainest reading: LayerNorm
+eps from the config (1e-6 on every workload), GELU in its exact erf form, the
+attention scale 1/sqrt(d_h), attn_qkv's output columns ordered [q | k | v]
+with head h at columns h*d_h .. h*d_h + d_h - 1 of each, the mean pool over
+the patch tokens only (CLS excluded), and an out-projection plus an ln2 in the
+head's cross-attention block.
 """
 from __future__ import annotations
 
@@ -187,15 +189,28 @@ def allowed_keys(n_patches: int, patches_per_slot: int, has_cls: bool,
 def attention(q, k, v, allow: Optional[np.ndarray]) -> np.ndarray:
     """softmax(q k^T / sqrt(d) + mask) v for q [.., Nq, d], k/v [.., Nk, d];
     ``allow`` [Nq, Nk] boolean (None = every pair).  The row max is
-    subtracted before exp (exact in the softmax's definition)."""
+    subtracted before exp (exact in the softmax's definition).
+
+    Evaluated one (clip, head) slice at a time in one reused [Nq, Nk] buffer,
+    so that a long clip (8192 tokens: 512 MB per score matrix) holds a single
+    score matrix; every element goes through the same operations in the same
+    order as the vectorised definition."""
+    q, k, v = (np.asarray(t, np.float64) for t in (q, k, v))
     d = q.shape[-1]
-    s = (q @ np.swapaxes(k, -1, -2)) / math.sqrt(d)
-    if allow is not None:
-        s = np.where(allow, s, -np.inf)
-    s = s - s.max(axis=-1, keepdims=True)
-    e = np.exp(s)
-    p = e / e.sum(axis=-1, keepdims=True)
-    return p @ v
+    lead = q.shape[:-2]
+    out = np.empty(lead + (q.shape[-2], v.shape[-1]))
+    blocked = None if allow is None else ~np.asarray(allow, bool)
+    s = np.empty((q.shape[-2], k.shape[-2]))
+    for idx in np.ndindex(*lead):
+        np.matmul(q[idx], np.swapaxes(k[idx], -1, -2), out=s)
+        s /= math.sqrt(d)
+        if blocked is not None:
+            np.copyto(s, -np.inf, where=blocked)
+        s -= s.max(axis=-1, keepdims=True)
+        np.exp(s, out=s)
+        s /= s.sum(axis=-1, keepdims=True)
+        out[idx] = s @ v[idx]
+    return out
 
 
 def split_heads(x, heads):

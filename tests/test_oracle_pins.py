@@ -247,6 +247,23 @@ def _tiny(mask="block_causal", has_cls=True, frames=3, **kw):
     return base.with_(**kw)
 
 
+def _torch_rotary(t, cfg):
+    """3-D rotary positions on head vectors t [B, h, N, 64] (q or k), written
+    as complex multiplication: the tokens' (slot, patch row, patch column)
+    come from nested loops in token order; in axis group a (head dims
+    20a .. 20a + 19) the complex number t[20a + 2i] + i t[20a + 2i + 1] is
+    multiplied by exp(i pos_a / 10000^(i / 10)); dims 60..63 pass through."""
+    pos = torch.tensor([(s, r, c) for s in range(cfg.slots) for r in range(cfg.img_h // cfg.patch)
+                        for c in range(cfg.img_w // cfg.patch)], dtype=torch.float64)   # [N, 3]
+    freq = 10000.0 ** (-torch.arange(10, dtype=torch.float64) / 10.0)                     # [10]
+    ang = pos[:, :, None] * freq[None, None, :]                                           # [N, 3, 10]
+    rot = torch.polar(torch.ones_like(ang), ang)                                          # e^{i ang}
+    B, h, N, d = t.shape
+    z = torch.view_as_complex(t[..., :60].reshape(B, h, N, 3, 10, 2).contiguous())
+    turned = torch.view_as_real(z * rot).reshape(B, h, N, 60)
+    return torch.cat([turned, t[..., 60:]], dim=-1)
+
+
 def _torch_forward(cfg, W, pix):
     """An independent float64 forward from torch.nn.functional routines."""
     T = {k: torch.from_numpy(np.ascontiguousarray(v)) for k, v in W.items()}
@@ -255,7 +272,8 @@ def _torch_forward(cfg, W, pix):
                  stride=(cfg.tubelet, cfg.patch, cfg.patch)).flatten(2).transpose(1, 2)
     if cfg.has_cls:
         x = torch.cat([T["enc.cls_token"].expand(x.shape[0], 1, -1), x], 1)
-    x = x + T["enc.pos_embed"]
+    if not cfg.rope:   # a rotary model's positions enter through q and k instead
+        x = x + T["enc.pos_embed"]
     B, N, D = x.shape
     h = cfg.heads
     mask = None
@@ -271,7 +289,8 @@ def _torch_forward(cfg, W, pix):
         y = F.layer_norm(x, (D,), T[p + "ln1.weight"], T[p + "ln1.bias"], cfg.ln_eps)
         qkv = F.linear(y, T[p + "attn_qkv.weight"], T[p + "attn_qkv.bias"])
         qkv = qkv.reshape(B, -1, 3, h, D // h).permute(2, 0, 3, 1, 4)
-        o = F.scaled_dot_product_attention(qkv[0], qkv[1], qkv[2], attn_mask=mask)
+        q, k = (_torch_rotary(qkv[0], cfg), _torch_rotary(qkv[1], cfg)) if cfg.rope else (qkv[0], qkv[1])
+        o = F.scaled_dot_product_attention(q, k, qkv[2], attn_mask=mask)
         x = x + F.linear(o.transpose(1, 2).reshape(B, -1, D), T[p + "attn_out.weight"], T[p + "attn_out.bias"])
         y = F.layer_norm(x, (D,), T[p + "ln2.weight"], T[p + "ln2.bias"], cfg.ln_eps)
         y = F.gelu(F.linear(y, T[p + "ffn_up.weight"], T[p + "ffn_up.bias"]))
@@ -345,12 +364,10 @@ def test_block_rows_matches_full_block():
     assert np.allclose(got, full[1, rows], rtol=1e-12, atol=1e-13)
 
 
-def test_attentive_head_vs_torch_float64():
-    cfg = _tiny(mask="bidir", has_cls=False, head_sa_blocks=2, n_classes=5, pool="attentive")
-    W = orc.weights_f64(synth.make_tensor_table(cfg))
-    rng = np.random.default_rng(9)
-    tok = rng.standard_normal((2, cfg.n_tokens, cfg.dim))
-    got = orc.attentive_head(cfg, W, tok)
+def _torch_head(cfg, W, tok):
+    """The attentive-pool classifier from torch routines: pre-LN
+    self-attention blocks (no positions), then nn.MultiheadAttention with the
+    learned query, MLP and the linear classifier."""
     T = {k: torch.from_numpy(np.ascontiguousarray(v)) for k, v in W.items()}
     x = torch.from_numpy(tok)
     B, N, D = x.shape
@@ -379,8 +396,16 @@ def test_attentive_head_vs_torch_float64():
         y = F.layer_norm(z, (D,), T["head.xattn.ln2.weight"], T["head.xattn.ln2.bias"], cfg.ln_eps)
         z = z + F.linear(F.gelu(F.linear(y, T["head.xattn.ffn_up.weight"], T["head.xattn.ffn_up.bias"])),
                          T["head.xattn.ffn_down.weight"], T["head.xattn.ffn_down.bias"])
-        ref = F.linear(z[:, 0], T["head.cls.weight"], T["head.cls.bias"]).numpy()
-    assert np.allclose(got, ref, rtol=1e-10, atol=1e-12)
+        return F.linear(z[:, 0], T["head.cls.weight"], T["head.cls.bias"]).numpy()
+
+
+def test_attentive_head_vs_torch_float64():
+    cfg = _tiny(mask="bidir", has_cls=False, head_sa_blocks=2, n_classes=5, pool="attentive")
+    W = orc.weights_f64(synth.make_tensor_table(cfg))
+    rng = np.random.default_rng(9)
+    tok = rng.standard_normal((2, cfg.n_tokens, cfg.dim))
+    got = orc.attentive_head(cfg, W, tok)
+    assert np.allclose(got, _torch_head(cfg, W, tok), rtol=1e-10, atol=1e-12)
 
 
 def test_metrics_definitions():
@@ -447,3 +472,33 @@ def test_rope_scores_depend_on_position_differences_only():
         s1 = (orc.rope(qv, p) @ orc.rope(kv, pk).T).item()
         s2 = (orc.rope(qv, p + c) @ orc.rope(kv, pk + c).T).item()
         assert s1 == pytest.approx(s2, rel=1e-11, abs=1e-12)
+
+
+@pytest.mark.parametrize("mask", ["bidir", "block_causal"])
+def test_rotary_encoder_vs_torch_float64(mask):
+    """The whole rotary encoder (no positional table, q and k turned after
+    their bias in every block, v untouched) against the torch forward whose
+    rotation is a complex multiplication over enumerated positions."""
+    cfg = _rope_cfg().with_(depth=2, mask=mask, random_ln_affine=True, batch=2)
+    table = synth.make_tensor_table(cfg)
+    assert "enc.pos_embed" not in synth.table_dict(table)
+    W = orc.weights_f64(table)
+    pix = synth.make_pixels(cfg).astype(np.float64)
+    got = orc.encoder(cfg, W, pix)
+    ref = _torch_forward(cfg, W, pix)
+    assert np.allclose(got, ref, rtol=1e-10, atol=1e-11)
+    # the rotation matters: the same weights without it give another result
+    assert not np.allclose(got, _torch_forward(cfg.with_(rope=False), dict(W, **{
+        "enc.pos_embed": np.zeros((cfg.n_tokens, cfg.dim))}), pix), rtol=1e-6, atol=1e-8)
+
+
+def test_rotary_model_head_has_no_positions():
+    """A rotary encoder with the attentive head: the head's self-attention
+    blocks and its cross-attention take no rotation."""
+    cfg = _rope_cfg().with_(depth=1, head_sa_blocks=1, n_classes=5, pool="attentive",
+                            random_ln_affine=True, batch=2)
+    W = orc.weights_f64(synth.make_tensor_table(cfg))
+    pix = synth.make_pixels(cfg).astype(np.float64)
+    got = orc.forward(cfg, W, pix)
+    ref = _torch_head(cfg, W, _torch_forward(cfg, W, pix))
+    assert np.allclose(got, ref, rtol=1e-10, atol=1e-12)

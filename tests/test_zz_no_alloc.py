@@ -1,8 +1,8 @@
 """The allocation-free mean pooling entry point.
 
-Some callers cannot call cudaMalloc: work being recorded into a CUDA graph,
-serving loops that run under a fixed device-memory budget or must never
-synchronise the device, and hosts whose device allocator belongs to another
+Some callers cannot call cudaMalloc: serving loops that run under a fixed
+device-memory budget, code that must never stall the device (cudaMalloc may
+synchronise it), and hosts whose device allocator belongs to another
 framework.  jepa_b200_op_mean_pool_noalloc serves them with a fixed device
 array instead of a grown buffer.  These tests check it against the
 allocating entry point (jepa_b200_op_mean_pool) on two calls in a row, with
