@@ -41,10 +41,14 @@ head's cross-attention block.
 from __future__ import annotations
 
 import math
+import os
+import queue
+from concurrent.futures import ThreadPoolExecutor
 from typing import Dict, Iterable, Optional, Sequence
 
 import numpy as np
 from scipy.special import erf as _erf
+from threadpoolctl import threadpool_limits
 
 # ggml dtype ids (the tensor table's own numbering)
 DT_F32, DT_F16, DT_Q4_0, DT_Q8_0 = 0, 1, 2, 8
@@ -186,30 +190,53 @@ def allowed_keys(n_patches: int, patches_per_slot: int, has_cls: bool,
     return allow
 
 
+def _attention_slice(q, k, v, blocked, s):
+    """One (clip, head) slice of the attention below, scores in buffer s."""
+    np.matmul(q, np.swapaxes(k, -1, -2), out=s)
+    s /= math.sqrt(q.shape[-1])
+    if blocked is not None:
+        np.copyto(s, -np.inf, where=blocked)
+    s -= s.max(axis=-1, keepdims=True)
+    np.exp(s, out=s)
+    s /= s.sum(axis=-1, keepdims=True)
+    return s @ v
+
+
 def attention(q, k, v, allow: Optional[np.ndarray]) -> np.ndarray:
     """softmax(q k^T / sqrt(d) + mask) v for q [.., Nq, d], k/v [.., Nk, d];
     ``allow`` [Nq, Nk] boolean (None = every pair).  The row max is
     subtracted before exp (exact in the softmax's definition).
 
-    Evaluated one (clip, head) slice at a time in one reused [Nq, Nk] buffer,
-    so that a long clip (8192 tokens: 512 MB per score matrix) holds a single
-    score matrix; every element goes through the same operations in the same
-    order as the vectorised definition."""
+    Evaluated one (clip, head) slice at a time, each in a score buffer of its
+    own thread, so that a long clip (8192 tokens: 512 MB per score matrix)
+    holds only a few score matrices; the slices are independent, and every
+    element goes through the same operations in the same order as the
+    vectorised definition."""
     q, k, v = (np.asarray(t, np.float64) for t in (q, k, v))
-    d = q.shape[-1]
     lead = q.shape[:-2]
     out = np.empty(lead + (q.shape[-2], v.shape[-1]))
     blocked = None if allow is None else ~np.asarray(allow, bool)
-    s = np.empty((q.shape[-2], k.shape[-2]))
-    for idx in np.ndindex(*lead):
-        np.matmul(q[idx], np.swapaxes(k[idx], -1, -2), out=s)
-        s /= math.sqrt(d)
-        if blocked is not None:
-            np.copyto(s, -np.inf, where=blocked)
-        s -= s.max(axis=-1, keepdims=True)
-        np.exp(s, out=s)
-        s /= s.sum(axis=-1, keepdims=True)
-        out[idx] = s @ v[idx]
+    idx = list(np.ndindex(*lead))
+    nq, nk = q.shape[-2], k.shape[-2]
+    workers = max(1, min(len(idx), os.cpu_count() or 1, (8 << 30) // max(1, 8 * nq * nk)))
+    if workers == 1 or nq * nk < (1 << 20):
+        s = np.empty((nq, nk))
+        for i in idx:
+            out[i] = _attention_slice(q[i], k[i], v[i], blocked, s)
+        return out
+    bufs = queue.SimpleQueue()
+    for _ in range(workers):
+        bufs.put(np.empty((nq, nk)))
+
+    def one(i):
+        s = bufs.get()
+        out[i] = _attention_slice(q[i], k[i], v[i], blocked, s)
+        bufs.put(s)
+
+    # each slice's matrix products on one BLAS thread; the slices in parallel
+    with threadpool_limits(limits=1, user_api="blas"):
+        with ThreadPoolExecutor(max_workers=workers) as ex:
+            list(ex.map(one, idx))
     return out
 
 

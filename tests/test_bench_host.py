@@ -39,7 +39,8 @@ def test_gemm_flops_per_clip():
     assert fl["patch_embed"] == 2.0 * 3136 * 768 * D
 
 
-def test_cpu_sample_runs_the_rotary_blocks(monkeypatch):
+def test_cpu_clip_runs_every_rotary_block(monkeypatch):
+    """The cpu_baseline times one whole clip: every block's q and k turned."""
     calls = []
     real = orc.rope
 
@@ -49,14 +50,18 @@ def test_cpu_sample_runs_the_rotary_blocks(monkeypatch):
 
     monkeypatch.setattr(orc, "rope", counting)
     cfg = synth.small_config(synth.VJEPA2_LONG_ROPE)
-    s = bench.cpu_oracle_sample(cfg, target_s=0.5)
+    s = bench.cpu_oracle_clip(cfg)
     assert s["value"] > 0 and s["kind"] == "oracle" and s["cores"] >= 1
-    assert calls and len(calls) % 2 == 0          # q and k of every block timed
+    assert len(calls) == 2 * cfg.depth          # q and k of every block, timed whole
+    assert f"all {cfg.depth} blocks" in s["sample"]
 
 
 def test_reference_arm_line(capsys):
+    """A reference step is one block of one clip: ms_per_step is that step's
+    measured time (so steps x ms_per_step is the run's length), the rate is
+    one clip over its whole forward built from the measured parts."""
     class Args:
-        steps, warmup = 2, 1
+        steps, warmup = 3, 1
     cfg = synth.small_config(synth.LEVJEPA_VIT_L, frames=2, batch=1)
     assert bench.run_reference(Args(), cfg, rank=0, world=1) == 0
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
@@ -65,7 +70,10 @@ def test_reference_arm_line(capsys):
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
-    assert line["ms_per_step"] == pytest.approx(1000.0 * cfg.n_tokens * cfg.batch / line["value"])
+    # the clip's forward is longer than depth block steps, never shorter
+    assert 1000.0 * cfg.n_tokens / line["value"] >= cfg.depth * line["ms_per_step"]
+    assert bench.run_reference(Args(), cfg, rank=1, world=2) == 0     # other ranks do no work
+    assert capsys.readouterr().out == ""
 
 
 def test_source_hash_ignores_comments_not_code():
