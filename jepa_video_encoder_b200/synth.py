@@ -150,6 +150,102 @@ WORKLOADS: Dict[str, EncoderConfig] = {
                         LEVJEPA_VIT_L_Q4_B32, VJEPA2_LONG, VJEPA2_LONG_ROPE, VJEPA2_SSV2_ROPE)}
 
 
+@dataclass(frozen=True)
+class PredictorConfig:
+    """The masked predictor of a V-JEPA 2 encoder ("jepa.cpp — measured
+    benchmarks", "Masked predictor": a 12-layer, 384-wide predictor; head dim
+    32): context tokens of the encoder output are projected to the
+    predictor's width (pred.embed), one learned mask token stands at every
+    target position, both get the predictor's positional table
+    (pred.pos_embed), the sequence [context | targets] runs through pre-LN
+    blocks with bidirectional attention, and the targets leave through the
+    final norm and pred.proj back to the encoder's width.  ``ctx`` / ``tgt``
+    select token indices of the encoder's N tokens (the same for every clip);
+    "all" is every token, the pages' worst case (context = target = every
+    token)."""
+    name: str
+    enc: EncoderConfig
+    dim: int = 384
+    depth: int = 12
+    heads: int = 12
+    mlp: int = 1536
+    ctx: str = "all"          # "all" | "even" | "first_half"
+    tgt: str = "all"          # "all" | "odd" | "second_half"
+    weights: str = "f16"
+    batch: int = 1
+    seed: int = 7
+    ln_eps: float = 1e-6
+    random_ln_affine: bool = False
+
+    @property
+    def head_dim(self) -> int:
+        return self.dim // self.heads
+
+    @property
+    def n_tokens(self) -> int:
+        return self.enc.n_tokens
+
+    def _sel(self, rule: str) -> np.ndarray:
+        n = np.arange(self.n_tokens)
+        return {"all": n, "even": n[0::2], "odd": n[1::2], "first_half": n[: self.n_tokens // 2],
+                "second_half": n[self.n_tokens // 2:]}[rule]
+
+    @property
+    def ctx_idx(self) -> np.ndarray:
+        return self._sel(self.ctx)
+
+    @property
+    def tgt_idx(self) -> np.ndarray:
+        return self._sel(self.tgt)
+
+    def with_(self, **kw) -> "PredictorConfig":
+        return dataclasses.replace(self, **kw)
+
+
+def predictor_specs(pc: PredictorConfig) -> List[tuple]:
+    """(name, shape, kind) of the predictor's tensors in table order."""
+    De, D, M = pc.enc.dim, pc.dim, pc.mlp
+    s = [("pred.embed.weight", (D, De), "w"), ("pred.embed.bias", (D,), "b"),
+         ("pred.mask_tokens", (1, D), "w"), ("pred.pos_embed", (pc.n_tokens, D), "w")]
+    for i in range(pc.depth):
+        s += _block_names(f"pred.blk.{i}.", D, M)
+    s += [("pred.norm.weight", (D,), "ln_g"), ("pred.norm.bias", (D,), "ln_b"),
+          ("pred.proj.weight", (De, D), "w"), ("pred.proj.bias", (De,), "b")]
+    return s
+
+
+def make_predictor_table(pc: PredictorConfig, std: float = 0.02) -> List["Tensor"]:
+    """Seeded predictor tensors, drawn like make_tensor_table's."""
+    rng = np.random.default_rng(pc.seed)
+    table = []
+    for name, shape, kind in predictor_specs(pc):
+        if kind == "ln_g":
+            v = (np.float32(1.0) + np.float32(0.1) * rng.standard_normal(shape, dtype=np.float32)
+                 if pc.random_ln_affine else np.ones(shape, np.float32))
+        elif kind == "ln_b":
+            v = (np.float32(std) * rng.standard_normal(shape, dtype=np.float32)
+                 if pc.random_ln_affine else np.zeros(shape, np.float32))
+        else:
+            v = np.float32(std) * rng.standard_normal(shape, dtype=np.float32)
+        table.append(_store(name, shape, v, pc.weights))
+    return table
+
+
+def make_predictor_tokens(pc: PredictorConfig, batch: Optional[int] = None) -> np.ndarray:
+    """Seeded encoder-output-like tokens [B, N, D_enc]: LayerNorm outputs
+    (unit variance per token) stand in for the encoder's last_hidden_state."""
+    B = pc.batch if batch is None else batch
+    rng = np.random.default_rng(pc.seed + 2000)
+    return rng.standard_normal((B, pc.n_tokens, pc.enc.dim), dtype=np.float32)
+
+
+# The masked predictor of the V-JEPA 2 ViT-L encoder on the 16-frame 256^2
+# clip (2048 tokens), context = target = every token: a 4096-row sequence,
+# the pages' worst case ("Masked predictor").
+VJEPA2_PREDICTOR = PredictorConfig(name="vjepa2_predictor_l16_16f256_all_b8", enc=VJEPA2_SSV2.with_(weights="f16"),
+                                   batch=8)
+PREDICTORS: Dict[str, "PredictorConfig"] = {VJEPA2_PREDICTOR.name: VJEPA2_PREDICTOR}
+
 def small_config(base: EncoderConfig, **kw) -> EncoderConfig:
     """A shrunk copy of a workload that the oracle runs in seconds."""
     d = dict(dim=256, depth=2, heads=4, mlp=1024, img_h=64, img_w=64,
@@ -184,7 +280,8 @@ class Tensor:
 _RETYPED_SUFFIXES = ("attn_qkv.weight", "attn_out.weight", "ffn_up.weight",
                      "ffn_down.weight", "head.xattn.q.weight",
                      "head.xattn.k.weight", "head.xattn.v.weight",
-                     "head.xattn.out.weight", "head.cls.weight")
+                     "head.xattn.out.weight", "head.cls.weight",
+                     "pred.embed.weight", "pred.proj.weight")
 
 
 def is_retyped(name: str) -> bool:

@@ -400,6 +400,35 @@ def forward(cfg, W, pixels, pool_mode: Optional[str] = None) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# Masked predictor of the V-JEPA 2 encoders ("jepa.cpp — measured
+# benchmarks", "Masked predictor": a 12-layer, 384-wide predictor that reads
+# context tokens and predicts target tokens, head dim 32; the "Quantization"
+# page, "The rule", names its tensors: pred.embed (the context projection),
+# pred.mask_tokens, pred.pos_embed, predictor blocks with the encoder
+# block's tensor set, pred.proj).  Readings where the pages are silent: the
+# sequence is [context rows | target rows]; a context row is
+# pred.embed(token) plus the positional row of its token index; a target row
+# is the mask token plus the positional row of its token index; attention is
+# bidirectional over the whole sequence; the final norm (pred.norm) and
+# pred.proj map the target rows back to the encoder's width.
+# ---------------------------------------------------------------------------
+def predictor(pc, W, tokens: np.ndarray, ctx_idx: Sequence[int], tgt_idx: Sequence[int]) -> np.ndarray:
+    """tokens [B, N, D_enc] (the encoder's output) -> predictions [B, N_tgt,
+    D_enc] for the target indices."""
+    ctx_idx, tgt_idx = np.asarray(ctx_idx), np.asarray(tgt_idx)
+    tokens = np.asarray(tokens, np.float64)
+    B = tokens.shape[0]
+    pos = W["pred.pos_embed"]
+    ctx = linear(tokens[:, ctx_idx], W["pred.embed.weight"], W["pred.embed.bias"]) + pos[ctx_idx][None]
+    tgt = np.broadcast_to(W["pred.mask_tokens"][0] + pos[tgt_idx], (B, len(tgt_idx), pos.shape[1]))
+    x = np.concatenate([ctx, tgt], axis=1)
+    for i in range(pc.depth):
+        x = block(x, W, f"pred.blk.{i}.", pc.heads, pc.ln_eps, None)
+    y = layer_norm(x[:, len(ctx_idx):], W["pred.norm.weight"], W["pred.norm.bias"], pc.ln_eps)
+    return linear(y, W["pred.proj.weight"], W["pred.proj.bias"])
+
+
+# ---------------------------------------------------------------------------
 # Sampled rows of one block: the block's output for chosen query rows of one
 # clip, given that clip's block input.  Same definitions, evaluated only where
 # needed (K and V still come from every row).

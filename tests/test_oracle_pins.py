@@ -502,3 +502,91 @@ def test_rotary_model_head_has_no_positions():
     got = orc.forward(cfg, W, pix)
     ref = _torch_head(cfg, W, _torch_forward(cfg, W, pix))
     assert np.allclose(got, ref, rtol=1e-10, atol=1e-12)
+
+
+# ------------------------------------------------------- masked predictor --
+def _pred_cfg(**kw):
+    enc = synth.small_config(synth.VJEPA2_SSV2, frames=4, img_h=32, img_w=48, dim=128, heads=2, mlp=256)
+    base = synth.PredictorConfig(name="pred_pin", enc=enc, dim=64, depth=2, heads=2, mlp=128, ctx="even",
+                                 tgt="odd", weights="f32", batch=2, random_ln_affine=True)
+    return base.with_(**kw)
+
+
+def _torch_predictor(pc, W, tokens, ctx_idx, tgt_idx):
+    """The predictor from torch routines: rows assembled with index_select /
+    cat, blocks with scaled_dot_product_attention (head dim 32 here)."""
+    T = {k: torch.from_numpy(np.ascontiguousarray(v)) for k, v in W.items()}
+    tok = torch.from_numpy(tokens)
+    ci, ti = torch.from_numpy(np.asarray(ctx_idx)), torch.from_numpy(np.asarray(tgt_idx))
+    D, h = pc.dim, pc.heads
+    ctx = F.linear(tok.index_select(1, ci), T["pred.embed.weight"], T["pred.embed.bias"]) + \
+        T["pred.pos_embed"].index_select(0, ci)
+    tgt = (T["pred.mask_tokens"] + T["pred.pos_embed"].index_select(0, ti)).expand(tok.shape[0], -1, -1)
+    x = torch.cat([ctx, tgt], 1)
+    B, L, _ = x.shape
+    for i in range(pc.depth):
+        p = f"pred.blk.{i}."
+        y = F.layer_norm(x, (D,), T[p + "ln1.weight"], T[p + "ln1.bias"], pc.ln_eps)
+        qkv = F.linear(y, T[p + "attn_qkv.weight"], T[p + "attn_qkv.bias"]).reshape(B, L, 3, h, D // h)
+        qkv = qkv.permute(2, 0, 3, 1, 4)
+        o = F.scaled_dot_product_attention(qkv[0], qkv[1], qkv[2]).transpose(1, 2).reshape(B, L, D)
+        x = x + F.linear(o, T[p + "attn_out.weight"], T[p + "attn_out.bias"])
+        y = F.layer_norm(x, (D,), T[p + "ln2.weight"], T[p + "ln2.bias"], pc.ln_eps)
+        x = x + F.linear(F.gelu(F.linear(y, T[p + "ffn_up.weight"], T[p + "ffn_up.bias"])),
+                         T[p + "ffn_down.weight"], T[p + "ffn_down.bias"])
+    y = F.layer_norm(x[:, len(ctx_idx):], (D,), T["pred.norm.weight"], T["pred.norm.bias"], pc.ln_eps)
+    return F.linear(y, T["pred.proj.weight"], T["pred.proj.bias"]).numpy()
+
+
+@pytest.mark.parametrize("ctx,tgt", [("even", "odd"), ("all", "all"), ("first_half", "second_half")])
+def test_predictor_vs_torch_float64(ctx, tgt):
+    pc = _pred_cfg(ctx=ctx, tgt=tgt)
+    assert pc.head_dim == 32
+    W = orc.weights_f64(synth.make_predictor_table(pc))
+    tok = synth.make_predictor_tokens(pc).astype(np.float64)
+    got = orc.predictor(pc, W, tok, pc.ctx_idx, pc.tgt_idx)
+    assert got.shape == (pc.batch, len(pc.tgt_idx), pc.enc.dim)
+    assert np.allclose(got, _torch_predictor(pc, W, tok, pc.ctx_idx, pc.tgt_idx), rtol=1e-10, atol=1e-12)
+
+
+def test_predictor_permutation_properties():
+    """Attention reads the rows as a set and every row carries its own
+    position: shuffling the context list leaves the predictions unchanged,
+    shuffling the target list shuffles them the same way."""
+    pc = _pred_cfg()
+    W = orc.weights_f64(synth.make_predictor_table(pc))
+    tok = synth.make_predictor_tokens(pc).astype(np.float64)
+    ctx, tgt = pc.ctx_idx, pc.tgt_idx
+    base = orc.predictor(pc, W, tok, ctx, tgt)
+    rng = np.random.default_rng(40)
+    assert np.allclose(orc.predictor(pc, W, tok, rng.permutation(ctx), tgt), base, rtol=1e-11, atol=1e-13)
+    perm = rng.permutation(len(tgt))
+    assert np.allclose(orc.predictor(pc, W, tok, ctx, tgt[perm]), base[:, perm], rtol=1e-11, atol=1e-13)
+    # a target's prediction depends on its own position row, not only on the mask token
+    W2 = dict(W)
+    W2["pred.pos_embed"] = W["pred.pos_embed"].copy()
+    W2["pred.pos_embed"][tgt[0]] += 0.5 * rng.standard_normal(pc.dim)   # (a constant shift LayerNorm removes)
+    moved = orc.predictor(pc, W2, tok, ctx, tgt)
+    assert not np.allclose(moved[:, 0], base[:, 0])
+    assert np.abs(moved[:, 1:] - base[:, 1:]).max() > 1e-9      # the other rows read that row
+
+
+def test_predictor_with_zero_blocks_is_norm_and_projection():
+    """With every block's projection weights and biases zero the blocks are
+    the identity (each residual branch adds 0): a target's prediction is
+    pred.proj(pred.norm(mask token + its position row)), whatever the
+    context."""
+    pc = _pred_cfg()
+    W = orc.weights_f64(synth.make_predictor_table(pc))
+    for n in list(W):
+        if n.startswith("pred.blk.") and (n.endswith("attn_out.weight") or n.endswith("attn_out.bias") or
+                                          n.endswith("ffn_down.weight") or n.endswith("ffn_down.bias")):
+            W[n] = np.zeros_like(W[n])
+    tok = synth.make_predictor_tokens(pc).astype(np.float64)
+    got = orc.predictor(pc, W, tok, pc.ctx_idx, pc.tgt_idx)
+    z = W["pred.mask_tokens"][0] + W["pred.pos_embed"][pc.tgt_idx]
+    mu = z.mean(-1, keepdims=True)
+    sd = np.sqrt(((z - mu) ** 2).mean(-1, keepdims=True) + pc.ln_eps)
+    want = ((z - mu) / sd * W["pred.norm.weight"] + W["pred.norm.bias"]) @ W["pred.proj.weight"].T + \
+        W["pred.proj.bias"]
+    assert np.allclose(got, np.broadcast_to(want, got.shape), rtol=1e-12, atol=1e-13)
