@@ -255,7 +255,8 @@ def cpu_oracle_block_step(cfg, W, x, blk, allow, rope_pos):
 def run_config(cfg, world: int, l2: str) -> dict:
     """The workload a line measures; both arms report the same keys."""
     return {"workload": cfg.name, "batch_per_gpu": cfg.batch, "global_batch": cfg.batch * world,
-            "tokens_per_clip": cfg.n_tokens, "weights": cfg.weights, "mask": cfg.mask, "pool": cfg.pool,
+            "tokens_per_clip": cfg.n_tokens, "weights": cfg.weights,
+            "activations": "bf16" if cfg.act_bf16 else "f16", "mask": cfg.mask, "pool": cfg.pool,
             "parallelism": f"replicas x{world}", "l2": l2}
 
 
@@ -320,7 +321,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     table = synth.make_tensor_table(cfg)
     pix_np = synth.make_pixels(cfg)
-    model = jb.Model(cfg, table, device=local_rank)
+    model = jb.Model(cfg, table, device=local_rank, quant_f16_copy=args.quant_f16_copy)
     pixels = torch.from_numpy(pix_np).to(dev)
     out = torch.empty(model.out_shape(cfg.batch, cfg.pool), dtype=torch.float32, device=dev)
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MiB > L2
@@ -453,8 +454,10 @@ def run_ours(args, cfg, rank, world, local_rank):
         "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
         "ms_per_step_min": min(ms_steps), "ms_per_step_sd": statistics.pstdev(ms_steps),
         "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": run_config(cfg, world, l2="flushed between steps (256 MiB write)"),
+        "vs_baseline": None, "dtype": "bf16" if cfg.act_bf16 else "f16", "data": "synthetic",
+        "config": dict(run_config(cfg, world, l2="flushed between steps (256 MiB write)"),
+                       **({"quant_f16_copy": bool(args.quant_f16_copy)} if cfg.weights in ("q8_0", "q4_0") else {})),
+        "weight_bytes": model.n_bytes,
         "clips_per_s": world * B * args.steps / (total_ms / 1000.0),
         "tflops": tflops, "tc_peak_frac": tflops / peak_dense,
         "tc_peak": {"value": peak_dense, "source": f"{peak_src} bf16 burst"},
@@ -474,23 +477,131 @@ def run_ours(args, cfg, rank, world, local_rank):
     return 0
 
 
+def _pred_flops(pc) -> dict:
+    """Algorithmic FLOPs per clip of the masked predictor by kernel class
+    (attention at the predictor's head dim, every (query, key) pair)."""
+    nc, nt = len(pc.ctx_idx), len(pc.tgt_idx)
+    L, D, M, De, d = nc + nt, pc.dim, pc.mlp, pc.enc.dim, pc.depth
+    return {"patch_embed": 2.0 * nc * De * D, "gemm_qkv": 2.0 * L * D * 3 * D * d, "attention": 4.0 * L * L * D * d,
+            "gemm_out": 2.0 * L * D * D * d, "gemm_up": 2.0 * L * D * M * d, "gemm_down": 2.0 * L * M * D * d,
+            "pool_head": 2.0 * nt * D * De}
+
+
+def run_predictor(args, pc, rank, world, local_rank):
+    """The masked predictor alone on seeded encoder-output tokens resident in
+    HBM: one step = one jepa_b200_predict of the batch; the rate counts the
+    predicted target tokens."""
+    import torch
+    import numpy as np
+    import jepa_video_encoder_b200 as jb
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    table = synth.make_tensor_table(pc.enc) + synth.make_predictor_table(pc)
+    model = jb.Model(pc.enc, table, device=local_rank, predictor=pc)
+    tok_np = synth.make_predictor_tokens(pc)
+    tokens = torch.from_numpy(tok_np).to(dev)
+    ci, ti = pc.ctx_idx, pc.tgt_idx
+    out = torch.empty((pc.batch, len(ti), pc.enc.dim), dtype=torch.float32, device=dev)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, args.warmup)):
+        model.predict(tokens, ci, ti, out=out, stream=stream)
+    torch.cuda.synchronize(dev)
+    if model.sync_status(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    clock_path = os.path.join(tempfile.gettempdir(), f"jepa_clocks_rank{rank}.csv")
+    proc, fh = _clock_sampler_start(clock_path)
+    time.sleep(0.3)
+    launches = 0
+    t0 = time.time()
+    for k in range(args.steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        model.predict(tokens, ci, ti, out=out, stream=stream)
+        ev[k][1].record(stream)
+        launches += model.last_launch_count()
+    torch.cuda.synchronize(dev)
+    clocks = _clock_sampler_stop(proc, fh, clock_path, local_rank, t0, time.time())
+    if model.sync_status(stream) != 0:
+        raise RuntimeError("device error in the timed region")
+    ms_steps = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(sum(ms_steps), world, dev)
+    units = pc.batch * len(ti)
+    value = whole_job_rate(units, world, args.steps, total_ms)
+    model.set_profiling(True)
+    prof = {k: [0.0, 0] for k in jb._abi.KERNEL_CLASSES}
+    for k in range(args.steps):
+        flush.zero_()
+        model.predict(tokens, ci, ti, out=out, stream=stream)
+        for kc, (ms, n) in model.profile_read().items():
+            prof[kc][0] += ms
+            prof[kc][1] += n
+    model.set_profiling(False)
+    if rank != 0:
+        model.close()
+        return 0
+    peaks, peak_src = _peaks()
+    fl = _pred_flops(pc)
+    B = pc.batch
+    kernels = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
+               for k, v in prof.items() if v[1] > 0}
+    for k in kernels:
+        if k in fl and kernels[k]["ms_per_step"] > 0:
+            kernels[k]["tflops"] = B * fl[k] / (kernels[k]["ms_per_step"] / 1000.0) / 1e12
+    ms_per_step = total_ms / args.steps
+    tflops = B * sum(fl.values()) / (ms_per_step / 1000.0) / 1e12
+    cpu = None
+    if world == 1 and not args.no_cpu:
+        from oracle import jepa_oracle as orc
+        W = orc.weights_f64([t for t in table if t.name.startswith("pred.")])
+        tc = time.perf_counter()
+        orc.predictor(pc, W, tok_np[:1].astype(np.float64), ci, ti)
+        t_clip = time.perf_counter() - tc
+        cpu = {"value": len(ti) / t_clip, "unit": "target tokens/s", "cores": _oracle_threads(), "kind": "oracle",
+               "sample": f"1 clip: the whole predictor in float64 numpy, timed whole ({t_clip:.1f} s)"}
+    line = {"metric": "masked-predictor target tokens/s on 1 B200", "value": value, "unit": "target tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
+            "ms_per_step_min": min(ms_steps), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16", "data": "synthetic",
+            "config": {"workload": pc.name, "batch_per_gpu": B, "n_ctx": len(ci), "n_tgt": len(ti),
+                       "pred_dim": pc.dim, "pred_depth": pc.depth, "pred_heads": pc.heads, "weights": pc.weights,
+                       "l2": "flushed between steps (256 MiB write)"},
+            "tflops": tflops, "tc_peak_frac": tflops / peak_dense_of(peaks), "kernels": kernels,
+            "cpu_baseline": cpu, "gpu_launches": launches, "clocks": clocks,
+            "when": datetime.datetime.now(datetime.timezone.utc).strftime("%Y-%m-%dT%H:%M:%S.%fZ")}
+    print(json.dumps(line), flush=True)
+    model.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS) + sorted(synth.PREDICTORS))
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
     ap.add_argument("--clock-log", default=None,
                     help="CSV of the nvidia-smi clock samples taken during the timed region ({rank} is replaced)")
+    ap.add_argument("--quant-f16-copy", action="store_true",
+                    help="q8_0 / q4_0 workloads: also keep an f16 copy of the matrices for the large GEMMs")
     ap.add_argument("--forward-only", action="store_true",
                     help="run warm-up + --steps forwards and exit (no timing, no JSON): for ncu launch lists")
     args = ap.parse_args()
-    cfg = synth.WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.workload in synth.PREDICTORS:
+        if args.impl == "reference" or world > 1:
+            print(json.dumps({"impl": args.impl, "unavailable": "the predictor workload runs on one GPU, ours only"}))
+            return 0
+        return run_predictor(args, synth.PREDICTORS[args.workload], rank, world, local_rank)
+    cfg = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, cfg, rank, world)
     if world > 1:

@@ -99,6 +99,18 @@ typedef struct {
                        * of 20 (slot, patch row, patch column); in group a the pair
                        * (20a + 2i, 20a + 2i + 1) of q and k turns by pos_a * 10000^(-2i/20),
                        * i < 10; dims 60..63 stay as they are. */
+  int quant_f16_copy; /* 1: also keep an f16 copy of every q8_0 / q4_0 matrix (dequantised once at
+                       * load) and run the GEMMs of 256 rows or more on it; 0 (default): keep the
+                       * blocks only, every GEMM unpacks them in its loader. */
+  /* Masked predictor (pred_depth 0: none), run by jepa_b200_predict: width, blocks,
+   * heads (pred_dim / pred_heads = 32 or 64) and MLP width of the V-JEPA 2 predictor
+   * ("jepa.cpp -- measured benchmarks", "Masked predictor": 12 blocks, width 384,
+   * head dim 32). */
+  int pred_depth, pred_dim, pred_heads, pred_mlp;
+  int act_bf16;       /* 1: every 16-bit activation and MMA operand (LayerNorm outputs, Q, K, V, P,
+                       * the attention output, the MLP's hidden values, the weights' 16-bit form)
+                       * is bf16 instead of f16; the residual stream, LayerNorm statistics,
+                       * softmax and every accumulation stay f32. */
 } jepa_b200_config;
 
 /* One entry of the tensor table.  Host memory, owned by the caller; it is
@@ -122,14 +134,19 @@ typedef struct jepa_b200_model jepa_b200_model;
  * [N, D] (not with rope), enc.cls_token [D] (has_cls), enc.blk.<i>.{ln1,attn_qkv,attn_out,ln2,
  * ffn_up,ffn_down}.{weight,bias}, enc.norm.{weight,bias}; with a head also
  * head.blk.<i>.*, head.query [D], head.ln_kv.*, head.xattn.{q,k,v,out,
- * ffn_up,ffn_down}.{weight,bias}, head.xattn.ln2.*, head.cls.{weight,bias}.
+ * ffn_up,ffn_down}.{weight,bias}, head.xattn.ln2.*, head.cls.{weight,bias};
+ * with a predictor pred.embed.{weight [Dp, D], bias}, pred.mask_tokens
+ * [1, Dp], pred.pos_embed [N, Dp], pred.blk.<i>.* (the encoder block's
+ * tensors at width Dp = pred_dim), pred.norm.*, pred.proj.{weight [D, Dp],
+ * bias [D]}.
  * q8_0 / q4_0 are accepted only for the matrices that page re-types and only
  * when the input dimension is a multiple of 64.  f32 matrices are rounded to
  * f16 once here; 1-D tensors and pos_embed are kept in f32.  A q8_0 / q4_0
- * matrix is kept as its blocks (unpacked in the GEMM's loader and by the
- * head's few-row kernels) and also dequantised once, on the device, to f16
- * (each q*d or (q-8)*d rounded once: the values the loader unpack produces),
- * which the GEMMs with 256 or more rows use.
+ * matrix is kept as its blocks, which every GEMM's loader and the head's
+ * few-row kernels unpack (each q*d or (q-8)*d rounded once to f16); with
+ * cfg->quant_f16_copy it is also dequantised once, on the device, to an f16
+ * copy holding those same values, which the GEMMs of 256 or more rows then
+ * read instead.
  * Names the model does not use (a predictor's, say) are ignored; a name given
  * twice is ERR_ARG.
  * On success *out_model owns its device memory until jepa_b200_free.
@@ -150,6 +167,25 @@ JEPA_B200_API int jepa_b200_load_weights(const jepa_b200_config *cfg, const jepa
  * ERR_CUDA. */
 JEPA_B200_API int jepa_b200_encode(jepa_b200_model *m, const float *pixels, int B, int pool, float *out, size_t out_bytes,
                      void *stream);
+
+/* The masked predictor of a model loaded with pred_depth > 0 ("jepa.cpp --
+ * measured benchmarks", "Masked predictor"): each clip's context tokens are
+ * projected to the predictor's width (pred.embed), the learned mask token
+ * stands at every target position, both add the pred.pos_embed row of their
+ * token index, the sequence [context | targets] runs through the predictor's
+ * pre-LN blocks with bidirectional attention, and the target rows leave
+ * through pred.norm and pred.proj.
+ * tokens: device, f32 [B, N, dim] (the encoder's last_hidden_state, e.g. from
+ *         jepa_b200_encode with POOL_NONE);
+ * ctx_idx, tgt_idx: HOST int arrays of n_ctx / n_tgt token indices in
+ *         [0, N), the same for every clip (copied to the device by the call);
+ * out:    device, f32 [B, n_tgt, dim]; out_bytes its size.
+ * Enqueued on `stream`; the predictor's workspace grows to the largest
+ * B * (n_ctx + n_tgt) seen.  Errors: ERR_ARG (null pointers, B or counts
+ * < 1, an index out of range, no predictor), ERR_SHAPE (out_bytes too small,
+ * B * (n_ctx + n_tgt) above 524288 rows), ERR_CUDA. */
+JEPA_B200_API int jepa_b200_predict(jepa_b200_model *m, const float *tokens, int B, const int *ctx_idx, int n_ctx,
+                                    const int *tgt_idx, int n_tgt, float *out, size_t out_bytes, void *stream);
 
 /* End-to-end variant with HOST buffers: copies pixels (host, f32 [B, frames,
  * 3, H, W]; pinned memory makes the copy asynchronous) to model-owned device

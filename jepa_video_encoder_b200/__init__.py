@@ -66,18 +66,27 @@ def check_out(out, on_cuda: bool, device: Optional[int] = None) -> None:
         raise ValueError(f"out on {out.device}; expected " + (f"cuda:{device}" if on_cuda else "the host"))
 
 
-def make_config(cfg: "synth.EncoderConfig") -> _abi.Config:
+def make_config(cfg: "synth.EncoderConfig", quant_f16_copy: bool = False,
+                predictor: Optional["synth.PredictorConfig"] = None) -> _abi.Config:
+    pr = predictor
     return _abi.Config(dim=cfg.dim, depth=cfg.depth, heads=cfg.heads, mlp=cfg.mlp, patch=cfg.patch,
                        tubelet=cfg.tubelet, img_h=cfg.img_h, img_w=cfg.img_w, frames=cfg.frames,
                        has_cls=1 if cfg.has_cls else 0, mask=synth.MASK_IDS[cfg.mask],
                        head_sa_blocks=cfg.head_sa_blocks, n_classes=cfg.n_classes, ln_eps=cfg.ln_eps,
-                       rope=1 if cfg.rope else 0)
+                       rope=1 if cfg.rope else 0, quant_f16_copy=1 if quant_f16_copy else 0,
+                       pred_depth=pr.depth if pr else 0, pred_dim=pr.dim if pr else 0,
+                       pred_heads=pr.heads if pr else 0, pred_mlp=pr.mlp if pr else 0,
+                       act_bf16=1 if cfg.act_bf16 else 0)
 
 
 class Model:
-    """A loaded encoder on one CUDA device."""
+    """A loaded encoder on one CUDA device.  quant_f16_copy: also keep an f16
+    copy of the q8_0 / q4_0 matrices for the large GEMMs (default: blocks
+    only, unpacked in every GEMM's loader).  predictor: the shape of a masked
+    predictor whose pred.* tensors are in the table (see predict)."""
 
-    def __init__(self, cfg: "synth.EncoderConfig", table: List["synth.Tensor"], device: int = 0):
+    def __init__(self, cfg: "synth.EncoderConfig", table: List["synth.Tensor"], device: int = 0,
+                 quant_f16_copy: bool = False, predictor: Optional["synth.PredictorConfig"] = None):
         lib = load_library()
         self.cfg = cfg
         self.device = device
@@ -94,7 +103,7 @@ class Model:
                 e.shape[j] = s
             e.data = t.data.ctypes.data
             e.nbytes = t.nbytes
-        self._cfg = make_config(cfg)
+        self._cfg = make_config(cfg, quant_f16_copy, predictor)
         h = ctypes.c_void_p()
         check(lib.jepa_b200_load_weights(ctypes.byref(self._cfg), entries, len(table), device, ctypes.byref(h)),
               "load_weights")
@@ -152,6 +161,26 @@ class Model:
         check_out(out, True, self.device)
         check(load_library().jepa_b200_encode(self._h, pixels.data_ptr(), B, POOLS[pool], out.data_ptr(),
                                               out.numel() * 4, _stream_ptr(stream)), "encode")
+        return out
+
+    def predict(self, tokens, ctx_idx, tgt_idx, out=None, stream=None):
+        """Masked predictor: tokens CUDA float32 [B, N, dim] (the encoder's
+        last_hidden_state), ctx_idx / tgt_idx sequences of token indices ->
+        float32 [B, len(tgt_idx), dim].  Asynchronous."""
+        import numpy as np
+        import torch
+        if not isinstance(tokens, torch.Tensor) or not tokens.is_cuda or tokens.dtype != torch.float32 \
+                or not tokens.is_contiguous() or tokens.dim() != 3 or tokens.device.index != self.device:
+            raise ValueError(f"tokens must be a contiguous float32 tensor [B, N, D] on cuda:{self.device}")
+        ci = np.ascontiguousarray(np.asarray(ctx_idx, dtype=np.int32))
+        ti = np.ascontiguousarray(np.asarray(tgt_idx, dtype=np.int32))
+        B = int(tokens.shape[0])
+        if out is None:
+            out = torch.empty((B, len(ti), int(tokens.shape[2])), dtype=torch.float32, device=tokens.device)
+        check_out(out, True, self.device)
+        check(load_library().jepa_b200_predict(self._h, tokens.data_ptr(), B, ci.ctypes.data, len(ci), ti.ctypes.data,
+                                               len(ti), out.data_ptr(), out.numel() * 4, _stream_ptr(stream)),
+              "predict")
         return out
 
     def encode_host(self, pixels, pool: Optional[str] = None, out=None, stream=None):

@@ -19,7 +19,9 @@ class Config(ctypes.Structure):
     _fields_ = [("dim", c_int), ("depth", c_int), ("heads", c_int), ("mlp", c_int),
                 ("patch", c_int), ("tubelet", c_int), ("img_h", c_int), ("img_w", c_int),
                 ("frames", c_int), ("has_cls", c_int), ("mask", c_int),
-                ("head_sa_blocks", c_int), ("n_classes", c_int), ("ln_eps", c_float), ("rope", c_int)]
+                ("head_sa_blocks", c_int), ("n_classes", c_int), ("ln_eps", c_float), ("rope", c_int),
+                ("quant_f16_copy", c_int), ("pred_depth", c_int), ("pred_dim", c_int), ("pred_heads", c_int),
+                ("pred_mlp", c_int), ("act_bf16", c_int)]
 
 
 class TensorEntry(ctypes.Structure):
@@ -32,6 +34,8 @@ SIGNATURES = {
     "jepa_b200_load_weights": (c_int, [POINTER(Config), POINTER(TensorEntry), c_int, c_int, POINTER(c_void_p)]),
     "jepa_b200_encode": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_size_t, c_void_p]),
     "jepa_b200_encode_host": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_size_t, c_void_p]),
+    "jepa_b200_predict": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_int, c_void_p, c_int, c_void_p, c_size_t,
+                                  c_void_p]),
     "jepa_b200_out_shape": (c_int, [c_void_p, c_int, c_int, POINTER(c_int64)]),
     "jepa_b200_debug_stage": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_size_t, c_void_p]),
     "jepa_b200_sync_status": (c_int, [c_void_p, c_void_p]),

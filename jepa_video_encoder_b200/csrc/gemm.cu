@@ -82,7 +82,7 @@ __device__ __forceinline__ void rope_position(const QkvDst& q, int row, int& pt,
 }
 
 // Epilogue for 32 consecutive output columns col0..col0+31 of one row.
-template <bool LOWREG, bool ROPE>
+template <bool LOWREG, bool ROPE, bool BF>
 __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int col0, const uint32_t (&r)[32]) {
   float v[32];
 #pragma unroll
@@ -107,8 +107,8 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int
       uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(p.out) + static_cast<size_t>(row) * p.ldo + col0);
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        dst[j] = make_uint4(pack_half2(v[8 * j], v[8 * j + 1]), pack_half2(v[8 * j + 2], v[8 * j + 3]),
-                            pack_half2(v[8 * j + 4], v[8 * j + 5]), pack_half2(v[8 * j + 6], v[8 * j + 7]));
+        dst[j] = make_uint4(pack2<BF>(v[8 * j], v[8 * j + 1]), pack2<BF>(v[8 * j + 2], v[8 * j + 3]),
+                            pack2<BF>(v[8 * j + 4], v[8 * j + 5]), pack2<BF>(v[8 * j + 6], v[8 * j + 7]));
     } break;
     case EPI_RESID_F32: {
       float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + static_cast<size_t>(row) * p.ldo + col0);
@@ -131,7 +131,9 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int
       const int D = p.qkv.dim;
       const int part = col0 / D + p.qkv.first_part;
       const int within = col0 % D;
-      const int hd = within >> 6, d0 = within & 63;
+      // head hd of head_dim dims (32 or 64); its values go to dims d0.. of
+      // a 64-dim row (with 32-dim heads, dims 32..63 stay zero)
+      const int hd = within / p.qkv.head_dim, d0 = within % p.qkv.head_dim;
       const int b = row / p.qkv.ntok, t = row % p.qkv.ntok;
       const size_t bh = static_cast<size_t>(b) * p.qkv.heads + hd;
       if (ROPE && part < 2) {
@@ -146,13 +148,13 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int
           uint4* dst = reinterpret_cast<uint4*>(base + (bh * p.qkv.ntok + t) * 64 + d0);
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            dst[j] = make_uint4(pack_half2(v[8 * j], v[8 * j + 1]), pack_half2(v[8 * j + 2], v[8 * j + 3]),
-                                pack_half2(v[8 * j + 4], v[8 * j + 5]), pack_half2(v[8 * j + 6], v[8 * j + 7]));
+            dst[j] = make_uint4(pack2<BF>(v[8 * j], v[8 * j + 1]), pack2<BF>(v[8 * j + 2], v[8 * j + 3]),
+                                pack2<BF>(v[8 * j + 4], v[8 * j + 5]), pack2<BF>(v[8 * j + 6], v[8 * j + 7]));
         }
       } else if (p.qkv.vt) {
         __half* base = p.qkv.vt + (bh * 64 + d0) * static_cast<size_t>(p.qkv.npad) + t;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) base[static_cast<size_t>(j) * p.qkv.npad] = __float2half_rn(v[j]);
+        for (int j = 0; j < 32; ++j) base[static_cast<size_t>(j) * p.qkv.npad] = __ushort_as_half(pack1<BF>(v[j]));
       }
     } break;
     case EPI_PATCH: {
@@ -172,48 +174,102 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int
   }
 }
 
-// Unpack a [BN x 64] slice of a q8_0 / q4_0 weight matrix into the swizzled
-// f16 B tile.  Each thread converts 8 consecutive K elements of one row per
-// step: value = q * d (q8_0) or (q - 8) * d (q4_0), rounded once to f16.
-template <int BMODE, int BN>
+// Two weights to an f16 pair without integer-to-float conversions: the two
+// code bytes (selected by sel from x) are placed under the f16 exponent of
+// 1024, where the spacing is 1, so 0x64XX reads 1024 + XX exactly; the offset
+// (1024 + 128 for a q8_0 code stored XOR 0x80, 1024 + 8 for a q4_0 nibble) is
+// subtracted exactly, leaving the signed code q (or q - 8); the product with
+// the block scale d is then rounded once, RN(q * d): the same f16 value as
+// rounding the (exact) f32 product q * d.
+__device__ __forceinline__ uint32_t codes_to_h2(uint32_t x, uint32_t sel, __half2 off, __half2 d2) {
+  const uint32_t h = __byte_perm(x, 0x64646464u, sel);
+  const __half2 v = __hmul2_rn(__hsub2_rn(*reinterpret_cast<const __half2*>(&h), off), d2);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// 8 consecutive weights of one block (8 code bytes of q8_0, or the 8 low or
+// high nibbles, nsh = 0 or 4, of 8 bytes of q4_0) scaled by d -> 4 f16 pairs.
+template <int BMODE>
+__device__ __forceinline__ void unpack8(uint2 q, int nsh, __half2 d2, uint32_t (&w)[4]) {
+  uint32_t x0, x1;
+  __half2 off;
+  if (BMODE == B_Q8) {
+    x0 = q.x ^ 0x80808080u;
+    x1 = q.y ^ 0x80808080u;
+    off = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6480)));  // 1152
+  } else {
+    x0 = (q.x >> nsh) & 0x0F0F0F0Fu;
+    x1 = (q.y >> nsh) & 0x0F0F0F0Fu;
+    off = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6408)));  // 1032
+  }
+  w[0] = codes_to_h2(x0, 0x4140u, off, d2);
+  w[1] = codes_to_h2(x0, 0x4342u, off, d2);
+  w[2] = codes_to_h2(x1, 0x4140u, off, d2);
+  w[3] = codes_to_h2(x1, 0x4342u, off, d2);
+}
+
+// The same 8 weights rounded once to bf16: each code is made an exact f32
+// (the byte under the exponent of 2^23, where the spacing is 1, minus the
+// offset), multiplied by the scale (exact: an 8-bit integer times an 11-bit
+// significand) and rounded to bf16, RN(q * d).
+template <int BMODE>
+__device__ __forceinline__ void unpack8_bf16(uint2 q, int nsh, float d, uint32_t (&w)[4]) {
+  uint32_t x[2];
+  float off;
+  if (BMODE == B_Q8) {
+    x[0] = q.x ^ 0x80808080u;
+    x[1] = q.y ^ 0x80808080u;
+    off = 8388608.0f + 128.0f;
+  } else {
+    x[0] = (q.x >> nsh) & 0x0F0F0F0Fu;
+    x[1] = (q.y >> nsh) & 0x0F0F0F0Fu;
+    off = 8388608.0f + 8.0f;
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float v[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) v[b] = (__uint_as_float(__byte_perm(x[h], 0x4B000000u, 0x7540u + b)) - off) * d;
+    w[2 * h] = pack2<true>(v[0], v[1]);
+    w[2 * h + 1] = pack2<true>(v[2], v[3]);
+  }
+}
+
+// Address of the 8 codes of weights k..k+7 (k % 8 == 0) of row n, and the
+// nibble shift for q4_0 (byte j of a block holds elements j and j + 16).
+template <int BMODE>
+__device__ __forceinline__ const uint2* quant_src(const void* bq, int K, int n, int k, int& nsh) {
+  if (BMODE == B_Q8) {
+    nsh = 0;
+    return reinterpret_cast<const uint2*>(static_cast<const int8_t*>(bq) + static_cast<size_t>(n) * K + k);
+  }
+  const int j0 = k & 31;
+  nsh = j0 >= 16 ? 4 : 0;
+  return reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(bq) + static_cast<size_t>(n) * (K >> 1) +
+                                        (k >> 5) * 16 + (j0 & 15));
+}
+
+// Unpack a [rows x 64] slice (rows n0 .. n0 + rows - 1, K block kb) of a q8_0
+// / q4_0 weight matrix into the swizzled f16 B tile.  Each thread converts 8
+// consecutive K elements of one row per step: value = q * d (q8_0) or
+// (q - 8) * d (q4_0), rounded once to f16.
+template <int BMODE, int ROWS, bool BF>
 __device__ __forceinline__ void fill_b_quant(uint8_t* sB, const GemmParams& p, int n0, int kb, int ct) {
   const int K = p.K;
   const uint32_t sbase = smem_u32(sB);
 #pragma unroll 4
-  for (int idx = ct; idx < BN * 8; idx += 128) {
+  for (int idx = ct; idx < ROWS * 8; idx += 128) {
     const int r = idx >> 3, u = idx & 7;
     const int n = n0 + r;
     const int k = kb * 64 + u * 8;
-    const float d = __half2float(p.bscale[static_cast<size_t>(n) * (K >> 5) + (k >> 5)]);
+    const __half d = p.bscale[static_cast<size_t>(n) * (K >> 5) + (k >> 5)];
+    int nsh;
+    const uint2 q = __ldg(quant_src<BMODE>(p.bq, K, n, k, nsh));
     uint32_t w[4];
-    if (BMODE == B_Q8) {
-      const uint2 q = __ldg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(p.bq) +
-                                                           static_cast<size_t>(n) * K + k));
-      const uint32_t qq[2] = {q.x, q.y};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t word = qq[e >> 1];
-        const int sh = (e & 1) * 16;
-        const float a = static_cast<float>(static_cast<int8_t>((word >> sh) & 0xFF));
-        const float b = static_cast<float>(static_cast<int8_t>((word >> (sh + 8)) & 0xFF));
-        w[e] = pack_half2(a * d, b * d);
-      }
-    } else {
-      const int j0 = k & 31;
-      const uint2 q = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(p.bq) +
-                                                           static_cast<size_t>(n) * (K >> 1) + (k >> 5) * 16 +
-                                                           (j0 & 15)));
-      const int nsh = j0 >= 16 ? 4 : 0;
-      const uint32_t qq[2] = {q.x, q.y};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t word = qq[e >> 1];
-        const int sh = (e & 1) * 16;
-        const float a = static_cast<float>(static_cast<int>((word >> (sh + nsh)) & 0xF) - 8);
-        const float b = static_cast<float>(static_cast<int>((word >> (sh + 8 + nsh)) & 0xF) - 8);
-        w[e] = pack_half2(a * d, b * d);
-      }
-    }
+    if constexpr (BF)
+      unpack8_bf16<BMODE>(q, nsh, __half2float(d), w);
+    else
+      unpack8<BMODE>(q, nsh, __half2half2(d), w);
     st_shared_v4(sbase + sw128_offset(r, u * 8), w[0], w[1], w[2], w[3]);
   }
 }
@@ -255,6 +311,7 @@ __device__ __forceinline__ void patch_rowbases(const GemmParams& p, int m0, int 
   }
 }
 
+template <bool BF>
 __device__ __forceinline__ void fill_a_patch_vec8(uint8_t* sA, const GemmParams& p, int kb, int ct,
                                                   const long long (&rowbase)[8]) {
   const PatchSrc& s = p.patch;
@@ -276,10 +333,10 @@ __device__ __forceinline__ void fill_a_patch_vec8(uint8_t* sA, const GemmParams&
     if (rowbase[it] >= 0 && koff >= 0) {
       const float4* src = reinterpret_cast<const float4*>(s.pixels + rowbase[it] + koff);
       const float4 a = __ldg(src), b = __ldg(src + 1);
-      w0 = pack_half2(a.x, a.y);
-      w1 = pack_half2(a.z, a.w);
-      w2 = pack_half2(b.x, b.y);
-      w3 = pack_half2(b.z, b.w);
+      w0 = pack2<BF>(a.x, a.y);
+      w1 = pack2<BF>(a.z, a.w);
+      w2 = pack2<BF>(b.x, b.y);
+      w3 = pack2<BF>(b.z, b.w);
     }
     st_shared_v4(sbase + sw128_offset(r, u * 8), w0, w1, w2, w3);
   }
@@ -288,6 +345,7 @@ __device__ __forceinline__ void fill_a_patch_vec8(uint8_t* sA, const GemmParams&
 // General gather (any patch size, pixels 4-byte aligned): the ownership of
 // the fast path above, with the 8 column offsets of the thread's unit taken
 // once per K block and 4-byte loads, all 64 of a K block independent.
+template <bool BF>
 __device__ __forceinline__ void fill_a_patch_rows(uint8_t* sA, const GemmParams& p, int kb, int ct,
                                                   const long long (&rowbase)[8]) {
   const PatchSrc& s = p.patch;
@@ -313,14 +371,14 @@ __device__ __forceinline__ void fill_a_patch_rows(uint8_t* sA, const GemmParams&
 #pragma unroll
     for (int e = 0; e < 8; ++e)
       f[e] = (rowbase[it] >= 0 && koff[e] >= 0) ? __ldg(s.pixels + rowbase[it] + koff[e]) : 0.0f;
-    st_shared_v4(sbase + sw128_offset(r, u * 8), pack_half2(f[0], f[1]), pack_half2(f[2], f[3]),
-                 pack_half2(f[4], f[5]), pack_half2(f[6], f[7]));
+    st_shared_v4(sbase + sw128_offset(r, u * 8), pack2<BF>(f[0], f[1]), pack2<BF>(f[2], f[3]),
+                 pack2<BF>(f[4], f[5]), pack2<BF>(f[6], f[7]));
   }
 }
 
 // Epilogue of one output tile for one thread: its row, half of the BN
 // columns (chalf), read from TMEM at tb (lane quadrant already applied).
-template <int BN, bool LOWREG, bool ROPE = false>
+template <int BN, bool LOWREG, bool ROPE, bool BF>
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tb, int row, int nb, int chalf) {
   if (p.epi == EPI_RESID_F32) {
     // residual add: the residual's loads are issued before the TMEM load
@@ -354,7 +412,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tb, 
     for (int c = chalf * (BN / 64); c < (chalf + 1) * (BN / 64); ++c) {
       uint32_t r[32];
       tmem_ld32(tb + static_cast<uint32_t>(c * 32), r);
-      if (row < p.M) epilogue_chunk<LOWREG, ROPE>(p, row, nb * BN + c * 32, r);
+      if (row < p.M) epilogue_chunk<LOWREG, ROPE, BF>(p, row, nb * BN + c * 32, r);
     }
   }
 }
@@ -372,7 +430,7 @@ __device__ __forceinline__ void load_bias32(const float* bias, int col0, float4 
 // 128-byte-swizzled layout and sent with one TMA store (f16 / f32 outputs)
 // or one TMA reduce-add (f32 residual: X += A W^T + b), so every global
 // write is a full, coalesced line.
-template <int BN, bool LOWREG>
+template <int BN, bool LOWREG, bool BF>
 __device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUtensorMap* tmC, uint32_t tb,
                                                   int row0, int nb, int chalf, uint8_t* stage_buf, int lane,
                                                   bool& pending) {
@@ -452,8 +510,8 @@ __device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUt
             gelu_pair<LOWREG>(x0, x1);
             gelu_pair<LOWREG>(x2, x3);
           }
-          w[h * 16 + 2 * j] = pack_half2(x0, x1);
-          w[h * 16 + 2 * j + 1] = pack_half2(x2, x3);
+          w[h * 16 + 2 * j] = pack2<BF>(x0, x1);
+          w[h * 16 + 2 * j + 1] = pack2<BF>(x2, x3);
         }
       }
       if (pending) {
@@ -481,7 +539,7 @@ __device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUt
 // TMA store at (0, t0, b*h + head) when the 32 rows lie in one clip, else
 // written row by row.  V goes to V^T [B*h, 64, Npad] column by column (one
 // coalesced 64-byte store per dimension and warp).
-template <int BN, bool LOWREG, bool ROPE = false>
+template <int BN, bool LOWREG, bool ROPE, bool BF>
 __device__ __forceinline__ void epilogue_tile_qkv(const GemmParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
                                                   uint32_t tb, int row0, int nb, int chalf, uint8_t* stage_buf,
                                                   int lane, bool& pending) {
@@ -511,10 +569,10 @@ __device__ __forceinline__ void epilogue_tile_qkv(const GemmParams& p, const CUt
           __half* base = p.qkv.vt + ((static_cast<size_t>(b) * heads + hd) * 64 + h * 32) * p.qkv.npad + t;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            base[static_cast<size_t>(4 * j) * p.qkv.npad] = __float2half_rn(__uint_as_float(r[4 * j]) + bb[j].x);
-            base[static_cast<size_t>(4 * j + 1) * p.qkv.npad] = __float2half_rn(__uint_as_float(r[4 * j + 1]) + bb[j].y);
-            base[static_cast<size_t>(4 * j + 2) * p.qkv.npad] = __float2half_rn(__uint_as_float(r[4 * j + 2]) + bb[j].z);
-            base[static_cast<size_t>(4 * j + 3) * p.qkv.npad] = __float2half_rn(__uint_as_float(r[4 * j + 3]) + bb[j].w);
+            base[static_cast<size_t>(4 * j) * p.qkv.npad] = __ushort_as_half(pack1<BF>(__uint_as_float(r[4 * j]) + bb[j].x));
+            base[static_cast<size_t>(4 * j + 1) * p.qkv.npad] = __ushort_as_half(pack1<BF>(__uint_as_float(r[4 * j + 1]) + bb[j].y));
+            base[static_cast<size_t>(4 * j + 2) * p.qkv.npad] = __ushort_as_half(pack1<BF>(__uint_as_float(r[4 * j + 2]) + bb[j].z));
+            base[static_cast<size_t>(4 * j + 3) * p.qkv.npad] = __ushort_as_half(pack1<BF>(__uint_as_float(r[4 * j + 3]) + bb[j].w));
           }
         }
       }
@@ -539,8 +597,8 @@ __device__ __forceinline__ void epilogue_tile_qkv(const GemmParams& p, const CUt
           rope_pair(x0, x1, h * 32 + 4 * j, pt, py, px, p.qkv.rope);
           rope_pair(x2, x3, h * 32 + 4 * j + 2, pt, py, px, p.qkv.rope);
         }
-        w[h * 16 + 2 * j] = pack_half2(x0, x1);
-        w[h * 16 + 2 * j + 1] = pack_half2(x2, x3);
+        w[h * 16 + 2 * j] = pack2<BF>(x0, x1);
+        w[h * 16 + 2 * j + 1] = pack2<BF>(x2, x3);
       }
     }
     if (!base) continue;
@@ -569,7 +627,7 @@ __device__ __forceinline__ void epilogue_tile_qkv(const GemmParams& p, const CUt
   }
 }
 
-template <int BN, int BMODE, bool GATHER, bool ROPE>
+template <int BN, int BMODE, bool GATHER, bool ROPE, bool BF>
 __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
@@ -656,7 +714,7 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16_f32(128, BN);
+      constexpr uint32_t idesc = idesc_f16_f32(128, BN, BF);
       int stage = 0, acc = 0;
       uint32_t phase = 0, aphase = 0;
       bool ok = true;
@@ -722,16 +780,16 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
       bool done = false;
       if constexpr (!kLowReg) {  // the 128-register kernels keep the row-by-row QKV stores
         if (p.tma_epi && p.epi == EPI_QKV) {
-          epilogue_tile_qkv<BN, false, ROPE>(p, &tmC, &tmC2, tb, mb * 128 + quad * 32, nb, chalf, stage_buf, lane,
+          epilogue_tile_qkv<BN, false, ROPE, BF>(p, &tmC, &tmC2, tb, mb * 128 + quad * 32, nb, chalf, stage_buf, lane,
                                              pending);
           done = true;
         }
       }
       if (done) {
       } else if (p.tma_epi && p.epi != EPI_QKV)
-        epilogue_tile_tma<BN, kLowReg>(p, &tmC, tb, mb * 128 + quad * 32, nb, chalf, stage_buf, lane, pending);
+        epilogue_tile_tma<BN, kLowReg, BF>(p, &tmC, tb, mb * 128 + quad * 32, nb, chalf, stage_buf, lane, pending);
       else
-        epilogue_tile<BN, kLowReg, ROPE>(p, tb, row, nb, chalf);
+        epilogue_tile<BN, kLowReg, ROPE, BF>(p, tb, row, nb, chalf);
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
       if (++acc == 2) {
@@ -760,11 +818,11 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
         uint8_t* sA = smem + stage * C::STAGE_BYTES;
         uint8_t* sB = sA + C::A_BYTES;
         if (GATHER && vec8)
-          fill_a_patch_vec8(sA, p, kb, ct, rowbase);
+          fill_a_patch_vec8<BF>(sA, p, kb, ct, rowbase);
         else if (GATHER)
-          fill_a_patch_rows(sA, p, kb, ct, rowbase);
+          fill_a_patch_rows<BF>(sA, p, kb, ct, rowbase);
         else
-          fill_b_quant<BMODE, BN>(sB, p, nb * BN, kb, ct);
+          fill_b_quant<BMODE, BN, BF>(sB, p, nb * BN, kb, ct);
         fence_proxy_async_smem();
         mbar_arrive(&conv_bar[stage]);
         if (++stage == S) {
@@ -784,34 +842,116 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
 
 
 // ---------------------------------------------------------------------------
-// CTA-pair variant (f16 weights): a cluster of two CTAs on two SMs computes a
-// 256 x BN tile with tcgen05.mma.cta_group::2 (M = 256).  Each CTA loads the
-// 128 A rows of its half and half of the B tile (BN/2 rows), so per SM a
-// stage is 16 KB + BN*64 bytes instead of 16 KB + BN*128: the same MMA work
-// per SM with two thirds of the shared-memory traffic and more stages in
-// flight.  The leader CTA (rank 0) issues the MMAs; its commits arrive on the
+// CTA-pair variant: a cluster of two CTAs on two SMs computes a 256 x BN
+// tile with tcgen05.mma.cta_group::2 (M = 256).  Each CTA holds the 128 A
+// rows of its half and half of the B tile (BN/2 rows), so per SM a stage is
+// 16 KB + BN*64 bytes instead of 16 KB + BN*128: the same MMA work per SM
+// with two thirds of the shared-memory traffic and more stages in flight.
+// The leader CTA (rank 0) issues the MMAs; its commits arrive on the
 // barriers of both CTAs (multicast commit).  TMA loads are plain (no
 // multicast): each CTA loads its own tiles, the bytes counted on the
 // leader's barrier.
-template <int BN>
+//
+// B operand: f16 weights come by TMA (BMODE B_F16, 320 threads).  q8_0 /
+// q4_0 weights (BMODE B_Q8 / B_Q4, 448 threads) are unpacked in the loader:
+// four converter warps per CTA read the codes and scales of their CTA's
+// BN/2 weight rows straight from global memory, one K block ahead of the
+// one they convert (the loads need no shared-memory stage), and write the
+// f16 values into the swizzled B tile; each converter warp then arrives on
+// the leader's conversion barrier (cluster scope), which the MMA issuer
+// waits for beside the TMA barrier of the A tiles.
+template <int BN, int BMODE>
 struct Gemm2Cfg {
+  static constexpr bool CONV = BMODE != B_F16;
   static constexpr int A_BYTES = 128 * 64 * 2;
   static constexpr int B_BYTES = (BN / 2) * 64 * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = BN == 256 ? 6 : (BN == 192 ? 6 : 8);
+  // quantised weights: the raw codes of this CTA's BN/2 rows for one K block
+  // (64 bytes a row for q8_0, 32 for q4_0) and a 16-byte group of 8 scales
+  // a row holding the K block's two scales, both staged by TMA
+  static constexpr int RAW_W = BMODE == B_Q8 ? 64 : 32;
+  static constexpr int RAW_BYTES = CONV ? (BN / 2) * RAW_W : 0;
+  static constexpr int SC_BYTES = CONV ? (BN / 2) * 16 : 0;
+  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + RAW_BYTES + SC_BYTES + 1023) / 1024 * 1024;
+  static constexpr int STAGING = 8 * 4096;  // epilogue staging
+  static constexpr int MAX_STAGES = (227 * 1024 - STAGING - 1024) / STAGE_BYTES;
+  // quantised: four stages, converter warp w always converting stage w (its
+  // barrier phases then follow one another, never two apart)
+  static constexpr int STAGES = CONV ? 4 : (BN == 256 ? 6 : (BN == 192 ? 6 : 8));
+  static_assert(!CONV || MAX_STAGES >= 4, "four quantised stages must fit in shared memory");
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + 8 * 4096 + 1024;  // + epilogue staging
+  static constexpr int SMEM = STAGES * STAGE_BYTES + STAGING + 1024;
+  static constexpr int THREADS = CONV ? 448 : 320;
 };
 
-template <int BN, bool ROPE>
-__global__ void __launch_bounds__(320, 1)
+// One converter warp unpacks a whole stage: this CTA's BN/2 weight rows of
+// one K block, read from the staged codes and scales, to f16 in the
+// swizzled B tile.  Lane l takes the K offset 8 (l % 8) of rows l / 8 + 4 j.
+template <int BMODE, int ROWS, bool BF>
+__device__ __forceinline__ void quant_stage_convert(const uint8_t* sRaw, const uint8_t* sSc, uint8_t* sB, int kb,
+                                                    int lane) {
+  constexpr int RAW_W = BMODE == B_Q8 ? 64 : 32;
+  const uint32_t raw = smem_u32(sRaw), sc = smem_u32(sSc), sbase = smem_u32(sB);
+  const int u = lane & 7;
+  // q8_0: bytes 8u..8u+7 of the row's 64; q4_0: the K offset's block (u / 4)
+  // holds 16 bytes, its elements j and j + 16 in byte j (low, high nibble)
+  const int off = BMODE == B_Q8 ? 8 * u : 16 * (u >> 2) + 8 * (u & 1);
+  const int nsh = (BMODE == B_Q4 && (u & 2)) ? 4 : 0;
+  const int sidx = ((2 * kb) & 7) + (u >> 2);  // the unit's scale in the row's group of 8
+#pragma unroll 8
+  for (int r = lane >> 3; r < ROWS; r += 4) {
+    uint2 q;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(q.x), "=r"(q.y) : "r"(raw + r * RAW_W + off));
+    unsigned short dbits;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(dbits) : "r"(sc + r * 16 + sidx * 2));
+    uint32_t w[4];
+    if constexpr (BF)
+      unpack8_bf16<BMODE>(q, nsh, __half2float(__ushort_as_half(dbits)), w);
+    else
+      unpack8<BMODE>(q, nsh, __half2half2(__ushort_as_half(dbits)), w);
+    st_shared_v4(sbase + sw128_offset(r, u * 8), w[0], w[1], w[2], w[3]);
+  }
+}
+
+// Wait on a local barrier whose arrivals come from another CTA of the
+// cluster (acquire at cluster scope); bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
+  if (w.timeout_ns == 0) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    raise_error(w, DERR_TIMEOUT);
+    return false;
+  }
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*w.abort) return false;
+    if (globaltimer() - t0 > w.timeout_ns) {
+      raise_error(w, DERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+template <int BN, bool ROPE, int BMODE, bool BF>
+__global__ void __launch_bounds__(Gemm2Cfg<BN, BMODE>::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
-                     const GemmParams p) {
-  using C = Gemm2Cfg<BN>;
+                     const __grid_constant__ CUtensorMap tmS, const GemmParams p) {
+  using C = Gemm2Cfg<BN, BMODE>;
   constexpr int S = C::STAGES;
+  constexpr bool CONV = C::CONV;
   extern __shared__ uint8_t dsmem[];
-  __shared__ uint64_t full_bar[S], empty_bar[S], tfull_bar[2], tempty_bar[2], drain_bar;
+  __shared__ uint64_t full_bar[S], empty_bar[S], conv_bar[S], raw_bar[S], tfull_bar[2], tempty_bar[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -824,6 +964,8 @@ __global__ void __launch_bounds__(320, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&full_bar[s], 1);     // leader: one expect-tx arrival + the bytes of both CTAs
       mbar_init(&empty_bar[s], 1);    // both: the leader's multicast commit
+      mbar_init(&conv_bar[s], 2);     // leader: the stage's converter warp in each CTA
+      mbar_init(&raw_bar[s], 1);      // both: this CTA's codes and scales (expect-tx + bytes)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);    // both: the leader's multicast commit
@@ -840,6 +982,7 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (CONV) tma_prefetch_desc(&tmS);
   }
   tc_fence_before();
   cluster_sync();  // barriers of both CTAs initialised before any remote arrival
@@ -873,10 +1016,18 @@ __global__ void __launch_bounds__(320, 1)
           }
           uint8_t* sA = smem + stage * C::STAGE_BYTES;
           uint8_t* sB = sA + C::A_BYTES;
-          if (rank == 0) mbar_expect_tx(&full_bar[stage], 2u * C::STAGE_BYTES);
+          if (rank == 0) mbar_expect_tx(&full_bar[stage], CONV ? 2u * C::A_BYTES : 2u * (C::A_BYTES + C::B_BYTES));
           const uint32_t fb = leader_full0 + static_cast<uint32_t>(stage * sizeof(uint64_t));
+          const int n0 = nb * BN + static_cast<int>(rank) * (BN / 2);
           tma_load_2d_pair(sA, &tmA, fb, kb * 64, mb * 256 + static_cast<int>(rank) * 128);
-          tma_load_2d_pair(sB, &tmB, fb, kb * 64, nb * BN + static_cast<int>(rank) * (BN / 2));
+          if (!CONV) {
+            tma_load_2d_pair(sB, &tmB, fb, kb * 64, n0);
+          } else {  // this CTA's codes and scales, counted on its own barrier
+            uint8_t* sRaw = sB + C::B_BYTES;
+            mbar_expect_tx(&raw_bar[stage], static_cast<uint32_t>(C::RAW_BYTES + C::SC_BYTES));
+            tma_load_2d(sRaw, &tmB, &raw_bar[stage], kb * C::RAW_W, n0);
+            tma_load_2d(sRaw + C::RAW_BYTES, &tmS, &raw_bar[stage], (2 * kb) & ~7, n0);
+          }
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           if (++stage == S) {
@@ -885,14 +1036,17 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
       }
-      if (!ok && rank == 0) {  // let the copies already counted on the leader's barriers land
+      if (!ok) {  // let the copies already counted on the barriers land
         for (int s = 0; s < S; ++s)
-          if ((armed >> s) & 1u) mbar_wait_drain(&full_bar[s], (armed_par >> s) & 1u);
+          if ((armed >> s) & 1u) {
+            if (rank == 0) mbar_wait_drain(&full_bar[s], (armed_par >> s) & 1u);
+            if (CONV) mbar_wait_drain(&raw_bar[s], (armed_par >> s) & 1u);
+          }
       }
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_f16_f32(256, BN);
+      constexpr uint32_t idesc = idesc_f16_f32(256, BN, BF);
       int stage = 0, acc = 0;
       uint32_t phase = 0, aphase = 0;
       bool ok = true;
@@ -905,6 +1059,10 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t dtm = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, w)) {
+            ok = false;
+            break;
+          }
+          if (CONV && !mbar_wait_cluster(&conv_bar[stage], phase, w)) {
             ok = false;
             break;
           }
@@ -932,7 +1090,7 @@ __global__ void __launch_bounds__(320, 1)
       tc_commit_pair_mc(&drain_bar, 0x1);
       mbar_wait_drain(&drain_bar, 0);
     }
-  } else {
+  } else if (warp < 10) {
     const int quad = warp & 3;
     const int chalf = (warp - 2) >> 2;
     const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
@@ -949,11 +1107,11 @@ __global__ void __launch_bounds__(320, 1)
       const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quad * 32;
       const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
       if (p.tma_epi && p.epi == EPI_QKV)
-        epilogue_tile_qkv<BN, true, ROPE>(p, &tmC, &tmC2, tb, row0, nb, chalf, stage_buf, lane, pending);
+        epilogue_tile_qkv<BN, true, ROPE, BF>(p, &tmC, &tmC2, tb, row0, nb, chalf, stage_buf, lane, pending);
       else if (p.tma_epi)
-        epilogue_tile_tma<BN, false>(p, &tmC, tb, row0, nb, chalf, stage_buf, lane, pending);
+        epilogue_tile_tma<BN, CONV, BF>(p, &tmC, tb, row0, nb, chalf, stage_buf, lane, pending);
       else
-        epilogue_tile<BN, false, ROPE>(p, tb, row0 + lane, nb, chalf);
+        epilogue_tile<BN, CONV, ROPE, BF>(p, tb, row0 + lane, nb, chalf);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tempty0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
@@ -963,6 +1121,27 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     if (pending && lane == 0) bulk_wait0();
+  } else if (CONV) {
+    // converter warps 10-13: warp cw takes K-block positions cw, cw + 4, ...
+    // of the MMA's sequence (all in stage cw of the four), so four stages
+    // convert at once; once a stage's
+    // codes and scales have landed it unpacks this CTA's BN/2 weight rows
+    // into the stage's f16 B tile (shared memory to shared memory) and
+    // signals the leader
+    const int cw = warp - 10;
+    const uint32_t leader_conv0 = mapa_shared(smem_u32(&conv_bar[0]), 0);
+    const int total = ((num_tiles - cid + n_clusters - 1) / n_clusters) * kblocks;  // K blocks this pair runs
+    for (int i = cw; i < total; i += 4) {
+      const int stage = i % S;
+      const uint32_t phase = static_cast<uint32_t>(i / S) & 1u;
+      bool okw = mbar_wait(&raw_bar[stage], phase, w);
+      if (!__all_sync(0xffffffffu, okw)) break;
+      uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
+      quant_stage_convert<BMODE, BN / 2, BF>(sB + C::B_BYTES, sB + C::B_BYTES + C::RAW_BYTES, sB, i % kblocks, lane);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_conv0 + static_cast<uint32_t>(stage * sizeof(uint64_t)));
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -1016,6 +1195,18 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, int esize, uint64_t cols, ui
   return r == CUDA_SUCCESS;
 }
 
+// 2-D map without swizzle (staged raw bytes: uint8 codes, f16 scale groups).
+static bool make_tmap_plain(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols, uint64_t rows,
+                            uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[2] = {cols, rows}, st[1] = {row_bytes};
+  cuuint32_t b[2] = {box_cols, box_rows}, es[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), d, st, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int num_sms() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -1029,9 +1220,11 @@ int num_sms() {
 
 int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& Win, const float* bias, int epi,
                  void* out, int ldo, const QkvDst* qkv, const PatchSrc* patch) {
-  // A quantised matrix with a dequantised f16 copy runs as f16 once there
-  // are at least 256 rows: unpacking a 256 x 64 weight tile per 128 x 256 x
-  // 64 product in the loader costs more issue slots than the MMA takes.
+  // A quantised matrix loaded with a dequantised f16 copy runs on that copy
+  // once there are at least 256 rows; without one, GEMMs of 256 rows or more
+  // unpack it in the CTA-pair kernel's loader (each SM unpacks half of the
+  // 256 x 64 weight tile of a 256 x 256 x 64 product) and smaller ones in
+  // the single-CTA kernel's.
   DevMatrix W = Win;
   if (W.bmode != B_F16 && W.f16 && !patch && M >= 256) {
     W.bmode = B_F16;
@@ -1050,6 +1243,7 @@ int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& Win
   memset(op, 0, sizeof(*op));
   op->bn = bn;
   op->bmode = W.bmode;
+  op->bf16 = W.bf16;  // the model's 16-bit type: A, the unpacked weights and 16-bit outputs
   op->gather = patch ? 1 : 0;
   GemmParams& p = op->p;
   p.M = M;
@@ -1085,7 +1279,8 @@ int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& Win
     p.tma_epi = 1;
   }
   // QKV epilogue: Q and K as [B*h, N, 64] maps, 32 token rows per store
-  if (epi == EPI_QKV && qkv && (bn / 64) % 2 == 0 && qkv->ntok > 0 && M % qkv->ntok == 0 && qkv->dim % 64 == 0) {
+  if (epi == EPI_QKV && qkv && (bn / 64) % 2 == 0 && qkv->ntok > 0 && M % qkv->ntok == 0 && qkv->dim % 64 == 0 &&
+      qkv->head_dim == 64) {
     const uint64_t BHn = static_cast<uint64_t>(M / qkv->ntok) * qkv->heads;
     const uint64_t dims[3] = {64, static_cast<uint64_t>(qkv->ntok), BHn};
     const uint64_t str[2] = {128, static_cast<uint64_t>(qkv->ntok) * 128};
@@ -1100,18 +1295,30 @@ int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& Win
       p.tma_epi = 1;
     }
   }
-  // f16 weights and at least two 128-row blocks: the CTA-pair kernel
-  op->pair = (W.bmode == B_F16 && !patch && M >= 256) ? 1 : 0;
+  // at least two 128-row blocks: the CTA-pair kernel (quantised weights need
+  // a scale table whose rows TMA can address: 8-scale groups, 16-byte rows)
+  op->pair = (!patch && M >= 256 && (W.bmode == B_F16 || (W.scales_pad && W.sc_ld % 8 == 0))) ? 1 : 0;
   if (W.bmode == B_F16) {
     const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
     const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
     const uint32_t box[2] = {64, static_cast<uint32_t>(op->pair ? bn / 2 : bn)};
     if (!make_tmap_f16(&op->tmB, W.data, 2, dims, str, box)) return JEPA_B200_ERR_CUDA;
+  } else if (op->pair) {
+    // codes [N, K] bytes (q8_0) or [N, K/2] (q4_0): one K block of BN/2 rows
+    // per load; scales [N, sc_ld] f16: the 8-scale group holding the K block's two
+    const uint64_t row = W.bmode == B_Q8 ? static_cast<uint64_t>(K) : static_cast<uint64_t>(K) / 2;
+    if (!make_tmap_plain(&op->tmB, W.data, CU_TENSOR_MAP_DATA_TYPE_UINT8, row, static_cast<uint64_t>(N), row,
+                         W.bmode == B_Q8 ? 64u : 32u, static_cast<uint32_t>(bn / 2)))
+      return JEPA_B200_ERR_CUDA;
+    if (!make_tmap_plain(&op->tmS, W.scales_pad, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, static_cast<uint64_t>(W.sc_ld),
+                         static_cast<uint64_t>(N), static_cast<uint64_t>(W.sc_ld) * 2, 8u,
+                         static_cast<uint32_t>(bn / 2)))
+      return JEPA_B200_ERR_CUDA;
   }
   if (op->pair) {
     const int cluster_tiles = ((M + 255) / 256) * p.n_tiles;
     op->grid = 2 * std::min(cluster_tiles, num_sms() / 2);
-    op->smem = bn == 256 ? Gemm2Cfg<256>::SMEM : (bn == 192 ? Gemm2Cfg<192>::SMEM : Gemm2Cfg<128>::SMEM);
+    op->smem = bn == 256 ? Gemm2Cfg<256, B_F16>::SMEM : (bn == 192 ? Gemm2Cfg<192, B_F16>::SMEM : Gemm2Cfg<128, B_F16>::SMEM);
   } else {
     op->grid = std::min(p.m_tiles * p.n_tiles, num_sms());
     op->smem = bn == 256 ? GemmCfg<256>::SMEM : (bn == 192 ? GemmCfg<192>::SMEM : GemmCfg<128>::SMEM);
@@ -1119,9 +1326,9 @@ int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& Win
   return JEPA_B200_OK;
 }
 
-template <int BN, int BMODE, bool GATHER, bool ROPE = false>
+template <int BN, int BMODE, bool GATHER, bool ROPE, bool BF>
 static int launch_impl(const GemmOp& op, cudaStream_t st) {
-  auto kern = gemm_tc_kernel<BN, BMODE, GATHER, ROPE>;
+  auto kern = gemm_tc_kernel<BN, BMODE, GATHER, ROPE, BF>;
   static std::atomic<unsigned long long> attr_done{0};
   if (!smem_attr_once(attr_done, kern, GemmCfg<BN>::SMEM)) return JEPA_B200_ERR_CUDA;
   constexpr int threads = (BMODE != B_F16 || GATHER) ? 448 : 320;
@@ -1131,53 +1338,66 @@ static int launch_impl(const GemmOp& op, cudaStream_t st) {
   return JEPA_B200_OK;
 }
 
-template <int BN, bool ROPE = false>
+template <int BN, bool ROPE, int BMODE, bool BF>
 static int launch_pair(const GemmOp& op, cudaStream_t st) {
-  auto kern = gemm_pair_kernel<BN, ROPE>;
+  using C = Gemm2Cfg<BN, BMODE>;
+  auto kern = gemm_pair_kernel<BN, ROPE, BMODE, BF>;
   static std::atomic<unsigned long long> attr_done{0};
-  if (!smem_attr_once(attr_done, kern, Gemm2Cfg<BN>::SMEM)) return JEPA_B200_ERR_CUDA;
-  if (launch_pdl(kern, dim3(op.grid), dim3(320), Gemm2Cfg<BN>::SMEM, st, 2, op.tmA, op.tmB, op.tmC, op.tmC2, op.p) !=
-      cudaSuccess)
+  if (!smem_attr_once(attr_done, kern, C::SMEM)) return JEPA_B200_ERR_CUDA;
+  if (launch_pdl(kern, dim3(op.grid), dim3(C::THREADS), C::SMEM, st, 2, op.tmA, op.tmB, op.tmC, op.tmC2, op.tmS,
+                 op.p) != cudaSuccess)
     return JEPA_B200_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+}
+
+// Every instance is selected here from the op: tile width, weight format,
+// patch gather, rotary q / k, 16-bit activation type.
+template <bool BF>
+static int launch_typed(const GemmOp& op, cudaStream_t st) {
+  // rotary q / k only in the QKV GEMMs of a rotary model: their own instances,
+  // so that the others carry no rotation code
+  const bool rope = op.p.epi == EPI_QKV && op.p.qkv.rope;
+#define JB_PAIR(BNV)                                                                                              \
+  switch (op.bmode) {                                                                                             \
+    case B_Q8: return rope ? launch_pair<BNV, true, B_Q8, BF>(op, st) : launch_pair<BNV, false, B_Q8, BF>(op, st); \
+    case B_Q4: return rope ? launch_pair<BNV, true, B_Q4, BF>(op, st) : launch_pair<BNV, false, B_Q4, BF>(op, st); \
+    default: return rope ? launch_pair<BNV, true, B_F16, BF>(op, st) : launch_pair<BNV, false, B_F16, BF>(op, st); \
+  }
+#define JB_SINGLE(BNV)                                                                                              \
+  switch (op.bmode) {                                                                                               \
+    case B_Q8: return rope ? launch_impl<BNV, B_Q8, false, true, BF>(op, st) : launch_impl<BNV, B_Q8, false, false, BF>(op, st); \
+    case B_Q4: return rope ? launch_impl<BNV, B_Q4, false, true, BF>(op, st) : launch_impl<BNV, B_Q4, false, false, BF>(op, st); \
+    default: return rope ? launch_impl<BNV, B_F16, false, true, BF>(op, st) : launch_impl<BNV, B_F16, false, false, BF>(op, st); \
+  }
+  if (op.pair) {
+    switch (op.bn) {
+      case 256: JB_PAIR(256)
+      case 192: JB_PAIR(192)
+      default: JB_PAIR(128)
+    }
+  }
+  if (op.gather) {
+    switch (op.bn) {
+      case 256: return launch_impl<256, B_F16, true, false, BF>(op, st);
+      case 192: return launch_impl<192, B_F16, true, false, BF>(op, st);
+      default: return launch_impl<128, B_F16, true, false, BF>(op, st);
+    }
+  }
+  switch (op.bn) {
+    case 256: JB_SINGLE(256)
+    case 192: JB_SINGLE(192)
+    case 128: JB_SINGLE(128)
+    default: return JEPA_B200_ERR_SHAPE;
+  }
+#undef JB_SINGLE
+#undef JB_PAIR
 }
 
 int gemm_launch(const GemmOp& op_in, cudaStream_t st, DevErr* err, unsigned long long timeout_ns) {
   GemmOp op = op_in;
   op.p.err = err;
   op.p.timeout_ns = timeout_ns;
-  // rotary q / k only in the QKV GEMMs of a rotary model: their own instances,
-  // so that the others carry no rotation code
-  const bool rope = op.p.epi == EPI_QKV && op.p.qkv.rope;
-  if (op.pair) {
-    switch (op.bn) {
-      case 256: return rope ? launch_pair<256, true>(op, st) : launch_pair<256>(op, st);
-      case 192: return rope ? launch_pair<192, true>(op, st) : launch_pair<192>(op, st);
-      default: return rope ? launch_pair<128, true>(op, st) : launch_pair<128>(op, st);
-    }
-  }
-  if (op.gather) {
-    switch (op.bn) {
-      case 256: return launch_impl<256, B_F16, true>(op, st);
-      case 192: return launch_impl<192, B_F16, true>(op, st);
-      default: return launch_impl<128, B_F16, true>(op, st);
-    }
-  }
-#define JB_GEMM_CASE(BNV)                                                                                      \
-  case BNV:                                                                                                    \
-    switch (op.bmode) {                                                                                        \
-      case B_Q8: return rope ? launch_impl<BNV, B_Q8, false, true>(op, st) : launch_impl<BNV, B_Q8, false>(op, st); \
-      case B_Q4: return rope ? launch_impl<BNV, B_Q4, false, true>(op, st) : launch_impl<BNV, B_Q4, false>(op, st); \
-      default: return rope ? launch_impl<BNV, B_F16, false, true>(op, st) : launch_impl<BNV, B_F16, false>(op, st); \
-    }
-  switch (op.bn) {
-    JB_GEMM_CASE(256)
-    JB_GEMM_CASE(192)
-    JB_GEMM_CASE(128)
-    default:
-      return JEPA_B200_ERR_SHAPE;
-  }
-#undef JB_GEMM_CASE
+  return op.bf16 ? launch_typed<true>(op, st) : launch_typed<false>(op, st);
 }
 
 }  // namespace jb

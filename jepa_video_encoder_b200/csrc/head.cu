@@ -27,18 +27,18 @@ __device__ __forceinline__ float warp_max_h(float v) {
 
 constexpr int kGemvRows = 8;
 
-// 8 consecutive weights of row n starting at k (k a multiple of 8).
-template <int BMODE>
+// 8 consecutive weights of row n starting at k (k a multiple of 8); 16-bit
+// weights are f16, or bf16 (BF).
+template <int BMODE, bool BF>
 __device__ __forceinline__ void load_w8(const void* __restrict__ w, const __half* __restrict__ scales, int K, int n,
                                         int k, float (&o)[8]) {
   if (BMODE == B_F16) {
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(static_cast<const __half*>(w) + static_cast<size_t>(n) * K + k));
-    const __half2* h = reinterpret_cast<const __half2*>(&v);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 f = __half22float2(h[e]);
-      o[2 * e] = f.x;
-      o[2 * e + 1] = f.y;
+      o[2 * e] = widen1<BF>(static_cast<unsigned short>(u[e] & 0xFFFFu));
+      o[2 * e + 1] = widen1<BF>(static_cast<unsigned short>(u[e] >> 16));
     }
   } else {
     const float d = __half2float(scales[static_cast<size_t>(n) * (K >> 5) + (k >> 5)]);
@@ -62,7 +62,7 @@ __device__ __forceinline__ void load_w8(const void* __restrict__ w, const __half
   }
 }
 
-template <int BMODE>
+template <int BMODE, bool BF>
 __global__ void __launch_bounds__(256) gemv_kernel(const float* __restrict__ x, int M, int K,
                                                   const void* __restrict__ w, const __half* __restrict__ scales,
                                                   int N, const float* __restrict__ bias, int epi, const float* resid,
@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(256) gemv_kernel(const float* __restrict__ x, 
   for (int m = 0; m < kGemvRows; ++m) acc[m] = 0.0f;
   for (int k = lane * 8; k < K; k += 256) {
     float wv[8];
-    load_w8<BMODE>(w, scales, K, n, k, wv);
+    load_w8<BMODE, BF>(w, scales, K, n, k, wv);
 #pragma unroll
     for (int m = 0; m < kGemvRows; ++m) {
       if (m < M) {
@@ -115,11 +115,12 @@ int launch_gemv(const float* x, int M, int K, const DevMatrix& W, const float* b
   while (rows_per > 1 && static_cast<size_t>(rows_per) * K * 4 > 200 * 1024) rows_per >>= 1;
   if (static_cast<size_t>(K) * 4 > 200 * 1024) return JEPA_B200_ERR_SHAPE;
   const int smem_max = rows_per * K * 4;
-  static std::atomic<unsigned long long> attr_done[3] = {};
-  const int bm = W.bmode == B_Q8 ? 1 : (W.bmode == B_Q4 ? 2 : 0);
-  const bool attr_ok = bm == 1   ? smem_attr_once(attr_done[1], gemv_kernel<B_Q8>, 200 * 1024)
-                       : bm == 2 ? smem_attr_once(attr_done[2], gemv_kernel<B_Q4>, 200 * 1024)
-                                 : smem_attr_once(attr_done[0], gemv_kernel<B_F16>, 200 * 1024);
+  static std::atomic<unsigned long long> attr_done[4] = {};
+  const int bm = W.bmode == B_Q8 ? 1 : (W.bmode == B_Q4 ? 2 : (W.bf16 ? 3 : 0));
+  const bool attr_ok = bm == 1   ? smem_attr_once(attr_done[1], gemv_kernel<B_Q8, false>, 200 * 1024)
+                       : bm == 2 ? smem_attr_once(attr_done[2], gemv_kernel<B_Q4, false>, 200 * 1024)
+                       : bm == 3 ? smem_attr_once(attr_done[3], gemv_kernel<B_F16, true>, 200 * 1024)
+                                 : smem_attr_once(attr_done[0], gemv_kernel<B_F16, false>, 200 * 1024);
   if (!attr_ok) return JEPA_B200_ERR_CUDA;
   (void)smem_max;
   for (int m0 = 0; m0 < M; m0 += rows_per) {
@@ -129,20 +130,18 @@ int launch_gemv(const float* x, int M, int K, const DevMatrix& W, const float* b
     const float* xr = x + static_cast<size_t>(m0) * K;
     const float* rr = resid ? resid + static_cast<size_t>(m0) * resid_stride : nullptr;
     float* yr = y + static_cast<size_t>(m0) * N;
-    if (bm == 1)
-      launch_pdl(gemv_kernel<B_Q8>, grid, dim3(256), smem, st, 1, xr, mc, K, static_cast<const void*>(W.data),
-                 static_cast<const __half*>(W.scales), N, bias, epi, rr, resid_stride, yr);
-    else if (bm == 2)
-      launch_pdl(gemv_kernel<B_Q4>, grid, dim3(256), smem, st, 1, xr, mc, K, static_cast<const void*>(W.data),
-                 static_cast<const __half*>(W.scales), N, bias, epi, rr, resid_stride, yr);
-    else
-      launch_pdl(gemv_kernel<B_F16>, grid, dim3(256), smem, st, 1, xr, mc, K, static_cast<const void*>(W.data),
-                 static_cast<const __half*>(W.scales), N, bias, epi, rr, resid_stride, yr);
+    auto kern = bm == 1 ? gemv_kernel<B_Q8, false>
+              : bm == 2 ? gemv_kernel<B_Q4, false>
+              : bm == 3 ? gemv_kernel<B_F16, true>
+                        : gemv_kernel<B_F16, false>;
+    launch_pdl(kern, grid, dim3(256), smem, st, 1, xr, mc, K, static_cast<const void*>(W.data),
+               static_cast<const __half*>(W.scales), N, bias, epi, rr, resid_stride, yr);
   }
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 
 // One query per (clip, head) over all ntok keys: softmax(q k^T / 8) v.
+template <bool BF>
 __global__ void __launch_bounds__(256) xattn_1q_kernel(const float* __restrict__ q, const __half* __restrict__ k,
                                                        const __half* __restrict__ vt, int heads, int ntok, int npad,
                                                        float* __restrict__ out) {
@@ -163,12 +162,11 @@ __global__ void __launch_bounds__(256) xattn_1q_kernel(const float* __restrict__
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const uint4 v = __ldg(kr + u);
-      const __half2* h = reinterpret_cast<const __half2*>(&v);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float2 f = __half22float2(h[e]);
-        s = fmaf(qh[u * 8 + 2 * e], f.x, s);
-        s = fmaf(qh[u * 8 + 2 * e + 1], f.y, s);
+        s = fmaf(qh[u * 8 + 2 * e], widen1<BF>(static_cast<unsigned short>(w4[e] & 0xFFFFu)), s);
+        s = fmaf(qh[u * 8 + 2 * e + 1], widen1<BF>(static_cast<unsigned short>(w4[e] >> 16)), s);
       }
     }
     s *= 0.125f;
@@ -196,20 +194,21 @@ __global__ void __launch_bounds__(256) xattn_1q_kernel(const float* __restrict__
   for (int d = warp; d < 64; d += 8) {
     const __half* vr = vt + (static_cast<size_t>(bh) * 64 + d) * npad;
     float acc = 0.0f;
-    for (int j = lane; j < ntok; j += 32) acc = fmaf(sc[j], __half2float(vr[j]), acc);
+    for (int j = lane; j < ntok; j += 32) acc = fmaf(sc[j], widen1<BF>(__half_as_ushort(vr[j])), acc);
     acc = warp_sum_h(acc);
     if (lane == 0) out[static_cast<size_t>(b) * heads * 64 + hd * 64 + d] = acc * invL;
   }
 }
 
 int launch_xattn_1q(const float* q, const __half* k, const __half* vt, int B, int heads, int ntok, int npad,
-                    float* out, cudaStream_t st) {
+                    float* out, cudaStream_t st, bool bf16) {
   if (!q || !k || !vt || !out) return JEPA_B200_ERR_ARG;
   if (B < 1 || heads < 1 || ntok < 1 || ntok > 16384 || npad < ntok) return JEPA_B200_ERR_SHAPE;
   const size_t smem = static_cast<size_t>(ntok) * 4;
-  static std::atomic<unsigned long long> attr_done{0};
-  if (!smem_attr_once(attr_done, xattn_1q_kernel, 16384 * 4)) return JEPA_B200_ERR_CUDA;
-  launch_pdl(xattn_1q_kernel, dim3(B * heads), dim3(256), smem, st, 1, q, k, vt, heads, ntok, npad, out);
+  static std::atomic<unsigned long long> attr_done[2] = {};
+  auto kern = bf16 ? xattn_1q_kernel<true> : xattn_1q_kernel<false>;
+  if (!smem_attr_once(attr_done[bf16 ? 1 : 0], kern, 16384 * 4)) return JEPA_B200_ERR_CUDA;
+  launch_pdl(kern, dim3(B * heads), dim3(256), smem, st, 1, q, k, vt, heads, ntok, npad, out);
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 

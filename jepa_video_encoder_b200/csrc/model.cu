@@ -13,6 +13,7 @@
 // "jepa.cpp -- measured benchmarks", "Attentive-pool head".
 #include <string.h>
 
+#include <algorithm>
 #include <cmath>
 #include <string>
 #include <unordered_map>
@@ -74,6 +75,11 @@ struct jepa_b200_model {
   DevMatrix xq, xkv, xout, xup, xdown, hcls;
   float *b_xq = nullptr, *b_xkv = nullptr, *b_xout = nullptr, *b_xup = nullptr, *b_xdown = nullptr,
         *b_cls = nullptr;
+  // masked predictor (cfg.pred_depth > 0)
+  DevMatrix pembed, pproj;
+  float *b_pembed = nullptr, *pmask = nullptr, *ppos = nullptr, *pnorm_g = nullptr, *pnorm_b = nullptr,
+        *b_pproj = nullptr;
+  std::vector<LayerW> pred;
   std::vector<void*> allocs;
   size_t weight_bytes = 0;
 
@@ -88,6 +94,22 @@ struct jepa_b200_model {
   std::vector<BlockOps> enc_ops, head_ops;
   GemmOp pe_op, kv_op;
   AttnOp attn_enc, attn_head;
+
+  // predictor workspace, for up to pws_rows sequence rows (B * (n_ctx + n_tgt))
+  // and the ops of the last (B, n_ctx, n_tgt, tokens, out)
+  size_t pws_rows = 0, pws_ctx_rows = 0, pws_tgt_rows = 0, pws_vt = 0;
+  float *pX = nullptr, *pE = nullptr;
+  __half *pY = nullptr, *pQ = nullptr, *pK = nullptr, *pVt = nullptr, *pO = nullptr, *pH = nullptr, *pA = nullptr,
+         *pT = nullptr;
+  int *pidx = nullptr;  // device ctx_idx [N] then tgt_idx [N]
+  std::vector<int> pidx_host;
+  std::vector<void*> pws_allocs;
+  int pops_B = 0, pops_ctx = 0, pops_tgt = 0, pops_Lpad = 0;
+  const float* pops_tokens = nullptr;
+  float* pops_out = nullptr;
+  std::vector<BlockOps> pred_ops;
+  GemmOp pembed_op, pproj_op;
+  AttnOp pattn;
 
   float* stage_pix = nullptr;
   size_t stage_pix_bytes = 0;
@@ -126,7 +148,8 @@ typedef std::unordered_map<std::string, const jepa_b200_tensor*> TableMap;
 bool is_retyped(const std::string& n) {
   static const char* suffixes[] = {"attn_qkv.weight",     "attn_out.weight",     "ffn_up.weight",
                                    "ffn_down.weight",     "head.xattn.q.weight", "head.xattn.k.weight",
-                                   "head.xattn.v.weight", "head.xattn.out.weight", "head.cls.weight"};
+                                   "head.xattn.v.weight", "head.xattn.out.weight", "head.cls.weight",
+                                   "pred.embed.weight",   "pred.proj.weight"};
   for (const char* s : suffixes) {
     const size_t L = strlen(s);
     if (n.size() >= L && n.compare(n.size() - L, L, s) == 0) return true;
@@ -274,18 +297,27 @@ struct Loader {
       M.bmode = dt == JEPA_B200_Q8_0 ? B_Q8 : (dt == JEPA_B200_Q4_0 ? B_Q4 : B_F16);
       M.data = dalloc(1);
       M.scales = quant ? static_cast<__half*>(dalloc(1)) : nullptr;
-      M.f16 = quant ? static_cast<__half*>(dalloc(1)) : nullptr;
+      M.scales_pad = M.scales;
+      M.sc_ld = static_cast<int>((K / 32 + 7) / 8 * 8);
+      M.f16 = quant && m->cfg.quant_f16_copy ? static_cast<__half*>(dalloc(1)) : nullptr;
       return M;
     }
+    const bool bf = m->cfg.act_bf16 != 0;
+    M.bf16 = bf ? 1 : 0;
     if (dt == JEPA_B200_F32 || dt == JEPA_B200_F16) {
-      std::vector<__half> h(static_cast<size_t>(N * Kpad), __float2half_rn(0.0f));
+      // the 16-bit operand: each value rounded once to f16, or to bf16 in a
+      // bf16 model (from the table's f32 or f16 value)
+      std::vector<uint16_t> h(static_cast<size_t>(N * Kpad), 0);
       int64_t row = 0;
       for (auto* t : parts) {
         std::vector<float> v = host_floats(t);
         const int64_t rows = numel(t) / K;
         for (int64_t r = 0; r < rows; ++r)
-          for (int64_t k = 0; k < K; ++k)
-            h[static_cast<size_t>((row + r) * Kpad + k)] = __float2half_rn(v[static_cast<size_t>(r * K + k)]);
+          for (int64_t k = 0; k < K; ++k) {
+            const float x = v[static_cast<size_t>(r * K + k)];
+            h[static_cast<size_t>((row + r) * Kpad + k)] =
+                bf ? __bfloat16_as_ushort(__float2bfloat16_rn(x)) : __half_as_ushort(__float2half_rn(x));
+          }
         row += rows;
       }
       M.bmode = B_F16;
@@ -314,11 +346,27 @@ struct Loader {
     M.scales = static_cast<__half*>(dalloc(sc.size() * 2));
     if (M.data) upload(M.data, qs.data(), qs.size());
     if (M.scales) upload(M.scales, sc.data(), sc.size() * 2);
-    // the dequantised f16 copy for the large-M GEMMs, made on the device
-    M.f16 = static_cast<__half*>(dalloc(static_cast<size_t>(N * K) * 2));
-    if (M.f16 && status == JEPA_B200_OK &&
-        launch_dequant_f16(M.bmode, M.data, M.scales, M.N, M.K, M.f16, nullptr) != JEPA_B200_OK)
-      status = JEPA_B200_ERR_CUDA;
+    // the scales again in rows padded to whole 8-scale (16-byte) groups, for
+    // the CTA-pair kernel's TMA-staged loader (the same array when K / 32 is
+    // a multiple of 8)
+    const int64_t kq = K / 32, ld = (kq + 7) / 8 * 8;
+    M.sc_ld = static_cast<int>(ld);
+    if (ld == kq) {
+      M.scales_pad = M.scales;
+    } else {
+      std::vector<uint16_t> sp(static_cast<size_t>(N * ld), 0);
+      for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < kq; ++j) sp[static_cast<size_t>(n * ld + j)] = sc[static_cast<size_t>(n * kq + j)];
+      M.scales_pad = static_cast<__half*>(dalloc(sp.size() * 2));
+      if (M.scales_pad) upload(M.scales_pad, sp.data(), sp.size() * 2);
+    }
+    // on request, the dequantised f16 copy for the large-M GEMMs, made on the device
+    if (m->cfg.quant_f16_copy) {
+      M.f16 = static_cast<__half*>(dalloc(static_cast<size_t>(N * K) * 2));
+      if (M.f16 && status == JEPA_B200_OK &&
+          launch_dequant_f16(M.bmode, M.data, M.scales, M.N, M.K, M.f16, nullptr, bf) != JEPA_B200_OK)
+        status = JEPA_B200_ERR_CUDA;
+    }
     return M;
   }
   DevMatrix mat(const std::string& name, int64_t N, int64_t K) {
@@ -366,6 +414,16 @@ int validate_config(const jepa_b200_config* c) {
   if (c->n_classes < 0 || c->head_sa_blocks < 0) return JEPA_B200_ERR_ARG;
   if (!(c->ln_eps > 0.0f)) return JEPA_B200_ERR_ARG;
   if (c->rope != 0 && c->rope != 1) return JEPA_B200_ERR_ARG;
+  if (c->quant_f16_copy != 0 && c->quant_f16_copy != 1) return JEPA_B200_ERR_ARG;
+  if (c->act_bf16 != 0 && c->act_bf16 != 1) return JEPA_B200_ERR_ARG;
+  if (c->pred_depth < 0) return JEPA_B200_ERR_ARG;
+  if (c->pred_depth > 0) {
+    if (c->pred_dim < 64 || c->pred_dim % 64 || c->pred_dim > 4096 || c->pred_heads < 1 ||
+        c->pred_dim % c->pred_heads || c->pred_mlp < 64 || c->pred_mlp % 64 || c->pred_mlp > 16384)
+      return JEPA_B200_ERR_SHAPE;
+    const int hd = c->pred_dim / c->pred_heads;
+    if (hd != 32 && hd != 64) return JEPA_B200_ERR_SHAPE;
+  }
   if (c->rope && (c->has_cls || c->frames / c->tubelet > kRopeMaxPos || c->img_h / c->patch > kRopeMaxPos ||
                   c->img_w / c->patch > kRopeMaxPos))
     return JEPA_B200_ERR_SHAPE;
@@ -494,6 +552,7 @@ int prepare_ops(jepa_b200_model* m, int B) {
   if ((s = attn_prepare(&m->attn_head, m->Q, m->Kb, m->Vt, B, c.heads, m->N, m->npad, JEPA_B200_MASK_BIDIR, 0, 1,
                         m->O)))
     return s;
+  m->attn_enc.bf16 = m->attn_head.bf16 = c.act_bf16 != 0;
   if (m->has_head) {
     QkvDst qd;
     qd.q = nullptr;
@@ -581,13 +640,16 @@ struct ProfScope {
     if (_s != JEPA_B200_OK) return _s; \
   } while (0)
 
+// One pre-LN block on the residual Xres [R, D] (D: the encoder's width, or
+// the predictor's with its own LN output buffer Y).
 int run_block(jepa_b200_model* m, const LayerW& L, const BlockOps& ops, const AttnOp& at, float* Xres, int R,
-              cudaStream_t st) {
-  const int D = m->cfg.dim;
+              cudaStream_t st, int D = 0, __half* Y = nullptr) {
+  if (!D) D = m->cfg.dim;
+  if (!Y) Y = m->Y;
   const float eps = m->cfg.ln_eps;
   {
     ProfScope ps(m, JEPA_B200_KC_LAYERNORM, st);
-    JB_TRY(launch_layernorm(Xres, R, D, 1, L.ln1_g, L.ln1_b, eps, m->Y, true, st));
+    JB_TRY(launch_layernorm(Xres, R, D, 1, L.ln1_g, L.ln1_b, eps, Y, true, st, m->cfg.act_bf16 != 0));
   }
   {
     ProfScope ps(m, JEPA_B200_KC_GEMM_QKV, st);
@@ -603,7 +665,7 @@ int run_block(jepa_b200_model* m, const LayerW& L, const BlockOps& ops, const At
   }
   {
     ProfScope ps(m, JEPA_B200_KC_LAYERNORM, st);
-    JB_TRY(launch_layernorm(Xres, R, D, 1, L.ln2_g, L.ln2_b, eps, m->Y, true, st));
+    JB_TRY(launch_layernorm(Xres, R, D, 1, L.ln2_g, L.ln2_b, eps, Y, true, st, m->cfg.act_bf16 != 0));
   }
   {
     ProfScope ps(m, JEPA_B200_KC_GEMM_UP, st);
@@ -642,11 +704,11 @@ int run_head(jepa_b200_model* m, int B, float* out, cudaStream_t st) {
   for (size_t l = 0; l < m->head.size(); ++l)
     JB_TRY(run_block(m, m->head[l], m->head_ops[l], m->attn_head, m->Yf, R, st));
   ProfScope ps(m, JEPA_B200_KC_POOL_HEAD, st);
-  JB_TRY(launch_layernorm(m->Yf, R, D, 1, m->lnkv_g, m->lnkv_b, eps, m->Y, true, st));
+  JB_TRY(launch_layernorm(m->Yf, R, D, 1, m->lnkv_g, m->lnkv_b, eps, m->Y, true, st, c.act_bf16 != 0));
   JB_TRY(gemm_launch(m->kv_op, st, m->err, m->timeout_ns));
   // q = W_q query + b_q (the learned query, shared by every clip)
   JB_TRY(launch_gemv(m->query, 1, D, m->xq, m->b_xq, 0, nullptr, 0, m->hq, st));
-  JB_TRY(launch_xattn_1q(m->hq, m->Kb, m->Vt, B, c.heads, m->N, m->npad, m->hattn, st));
+  JB_TRY(launch_xattn_1q(m->hq, m->Kb, m->Vt, B, c.heads, m->N, m->npad, m->hattn, st, c.act_bf16 != 0));
   // z = query + W_out attn + b_out
   JB_TRY(launch_gemv(m->hattn, B, D, m->xout, m->b_xout, 2, m->query, 0, m->hz, st));
   JB_TRY(launch_layernorm(m->hz, B, D, 1, m->ln2x_g, m->ln2x_b, eps, m->hzn, false, st));
@@ -700,6 +762,120 @@ int enqueue_forward(jepa_b200_model* m, const float* pixels, int B, int pool, fl
   }
   if (!s && pool == JEPA_B200_POOL_ATTENTIVE) s = run_head(m, B, out, st);
   return s;
+}
+
+// ------------------------------------------------------------ predictor --
+// Workspace for `rows` sequence rows (B * (n_ctx + n_tgt)), `crows` context
+// rows and `trows` target rows, grown and never shrunk; every buffer whose
+// 64-dim head rows the QKV epilogue fills only partly (32-dim heads) starts
+// zeroed, so the dims it never writes stay zero.
+int pred_workspace(jepa_b200_model* m, size_t rows, size_t crows, size_t trows, size_t vt_elems) {
+  if (rows <= m->pws_rows && crows <= m->pws_ctx_rows && trows <= m->pws_tgt_rows && vt_elems <= m->pws_vt)
+    return JEPA_B200_OK;
+  rows = std::max(rows, m->pws_rows);
+  crows = std::max(crows, m->pws_ctx_rows);
+  trows = std::max(trows, m->pws_tgt_rows);
+  const size_t vt_cap = std::max(vt_elems, m->pws_vt);
+  cudaDeviceSynchronize();
+  free_list(m->pws_allocs);
+  m->pws_rows = m->pws_ctx_rows = m->pws_tgt_rows = m->pws_vt = 0;
+  m->pops_B = 0;
+  const jepa_b200_config& c = m->cfg;
+  const size_t Dp = c.pred_dim, Mp = c.pred_mlp, D = c.dim;
+  // Q, K: [B*h, L, 64] = rows * h * 64 halves; V^T: [B*h, 64, Lpad] (vt_cap)
+  const size_t qk_elems = rows * c.pred_heads * 64;
+  auto get = [&](void** p, size_t bytes, bool zero) -> int {
+    if (cudaMalloc(p, bytes) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+    m->pws_allocs.push_back(*p);
+    if (zero && cudaMemset(*p, 0, bytes) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+    return JEPA_B200_OK;
+  };
+  int s = JEPA_B200_OK;
+  s = s ? s : get(reinterpret_cast<void**>(&m->pX), rows * Dp * 4, false);
+  s = s ? s : get(reinterpret_cast<void**>(&m->pY), rows * Dp * 2, false);
+  s = s ? s : get(reinterpret_cast<void**>(&m->pQ), qk_elems * 2, true);
+  s = s ? s : get(reinterpret_cast<void**>(&m->pK), qk_elems * 2, true);
+  s = s ? s : get(reinterpret_cast<void**>(&m->pVt), vt_cap * 2, true);
+  s = s ? s : get(reinterpret_cast<void**>(&m->pO), rows * Dp * 2, false);
+  s = s ? s : get(reinterpret_cast<void**>(&m->pH), rows * Mp * 2, false);
+  s = s ? s : get(reinterpret_cast<void**>(&m->pA), crows * D * 2, false);
+  s = s ? s : get(reinterpret_cast<void**>(&m->pE), crows * Dp * 4, false);
+  s = s ? s : get(reinterpret_cast<void**>(&m->pT), trows * Dp * 2, false);
+  s = s ? s : get(reinterpret_cast<void**>(&m->pidx), static_cast<size_t>(2) * m->N * sizeof(int), false);
+  if (s) {
+    free_list(m->pws_allocs);
+    return s;
+  }
+  m->pws_rows = rows;
+  m->pws_ctx_rows = crows;
+  m->pws_tgt_rows = trows;
+  m->pws_vt = vt_cap;
+  m->pidx_host.clear();
+  return JEPA_B200_OK;
+}
+
+int prepare_pred_ops(jepa_b200_model* m, const float* tokens, int B, int nc, int nt, float* out) {
+  const jepa_b200_config& c = m->cfg;
+  const int Dp = c.pred_dim, Mp = c.pred_mlp, L = nc + nt, R = B * L;
+  const int hd = Dp / c.pred_heads, Lpad = (L + 127) / 128 * 128;
+  int s;
+  // context rows: tokens (gathered, f16) -> pred.embed -> pE f32
+  if ((s = gemm_prepare(&m->pembed_op, m->pA, B * nc, c.dim, m->pembed, m->b_pembed, EPI_F32, m->pE, Dp, nullptr,
+                        nullptr)))
+    return s;
+  m->pred_ops.assign(m->pred.size(), BlockOps());
+  for (size_t l = 0; l < m->pred.size(); ++l) {
+    const LayerW& W = m->pred[l];
+    BlockOps& ops = m->pred_ops[l];
+    QkvDst qd;
+    qd.q = m->pQ;
+    qd.k = m->pK;
+    qd.vt = m->pVt;
+    qd.ntok = L;
+    qd.heads = c.pred_heads;
+    qd.npad = Lpad;
+    qd.dim = Dp;
+    qd.head_dim = hd;
+    if ((s = gemm_prepare(&ops.qkv, m->pY, R, Dp, W.qkv, W.b_qkv, EPI_QKV, m->pQ, 3 * Dp, &qd, nullptr))) return s;
+    if ((s = gemm_prepare(&ops.out, m->pO, R, Dp, W.out, W.b_out, EPI_RESID_F32, m->pX, Dp, nullptr, nullptr)))
+      return s;
+    if ((s = gemm_prepare(&ops.up, m->pY, R, Dp, W.up, W.b_up, EPI_GELU_F16, m->pH, Mp, nullptr, nullptr))) return s;
+    if ((s = gemm_prepare(&ops.down, m->pH, R, Mp, W.down, W.b_down, EPI_RESID_F32, m->pX, Dp, nullptr, nullptr)))
+      return s;
+  }
+  if ((s = attn_prepare(&m->pattn, m->pQ, m->pK, m->pVt, B, c.pred_heads, L, Lpad, JEPA_B200_MASK_BIDIR, 0, 1, m->pO,
+                        hd)))
+    return s;
+  m->pattn.bf16 = c.act_bf16 != 0;
+  // target rows: pred.norm -> pT f16 -> pred.proj -> out f32 [B * nt, dim]
+  if ((s = gemm_prepare(&m->pproj_op, m->pT, B * nt, Dp, m->pproj, m->b_pproj, EPI_F32, out, c.dim, nullptr,
+                        nullptr)))
+    return s;
+  return JEPA_B200_OK;
+}
+
+int enqueue_predict(jepa_b200_model* m, const float* tokens, int B, int nc, int nt, cudaStream_t st) {
+  const jepa_b200_config& c = m->cfg;
+  const int Dp = c.pred_dim, L = nc + nt, R = B * L;
+  const int* ctx = m->pidx;
+  const int* tgt = m->pidx + m->N;
+  {
+    ProfScope ps(m, JEPA_B200_KC_PATCH_EMBED, st);
+    JB_TRY(launch_gather_rows_f16(tokens, ctx, B, m->N, nc, c.dim, m->pA, st, c.act_bf16 != 0));
+    JB_TRY(gemm_launch(m->pembed_op, st, m->err, m->timeout_ns));
+    JB_TRY(launch_pred_assemble(m->pE, m->pmask, m->ppos, ctx, tgt, B, nc, nt, Dp, m->pX, st));
+  }
+  m->launches += 3;
+  for (size_t l = 0; l < m->pred.size(); ++l)
+    JB_TRY(run_block(m, m->pred[l], m->pred_ops[l], m->pattn, m->pX, R, st, Dp, m->pY));
+  {
+    ProfScope ps(m, JEPA_B200_KC_POOL_HEAD, st);
+    JB_TRY(launch_layernorm_rows(m->pX, B * nt, Dp, nt, L, nc, m->pnorm_g, m->pnorm_b, c.ln_eps, m->pT, true, st,
+                                 c.act_bf16 != 0));
+    JB_TRY(gemm_launch(m->pproj_op, st, m->err, m->timeout_ns));
+  }
+  m->launches += 2;
+  return JEPA_B200_OK;
 }
 
 }  // namespace
@@ -859,6 +1035,19 @@ static void load_sequence(Loader& L) {
     m->hcls = L.mat("head.cls.weight", c.n_classes, D);
     m->b_cls = L.vec("head.cls.bias", c.n_classes);
   }
+  if (c.pred_depth > 0) {
+    const int64_t Dp = c.pred_dim, Mp = c.pred_mlp;
+    m->pembed = L.mat("pred.embed.weight", Dp, D);
+    m->b_pembed = L.vec("pred.embed.bias", Dp);
+    m->pmask = L.table2d("pred.mask_tokens", 1, Dp);
+    m->ppos = L.table2d("pred.pos_embed", m->N, Dp);
+    m->pred.resize(c.pred_depth);
+    for (int l = 0; l < c.pred_depth; ++l) L.block(m->pred[l], "pred.blk." + std::to_string(l) + ".", Dp, Mp);
+    m->pnorm_g = L.vec("pred.norm.weight", Dp);
+    m->pnorm_b = L.vec("pred.norm.bias", Dp);
+    m->pproj = L.mat("pred.proj.weight", D, Dp);
+    m->b_pproj = L.vec("pred.proj.bias", D);
+  }
 }
 
 extern "C" {
@@ -914,6 +1103,60 @@ int jepa_b200_encode(jepa_b200_model* m, const float* pixels, int B, int pool, f
     if (cudaEventRecord(m->ev0, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
     if (cudaGraphLaunch(m->graph, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
   }
+  if (cudaEventRecord(m->ev1, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+  m->have_timing = true;
+  return JEPA_B200_OK;
+}
+
+int jepa_b200_predict(jepa_b200_model* m, const float* tokens, int B, const int* ctx_idx, int n_ctx,
+                      const int* tgt_idx, int n_tgt, float* out, size_t out_bytes, void* stream) {
+  if (!m || !tokens || !ctx_idx || !tgt_idx || !out || B < 1 || n_ctx < 1 || n_tgt < 1) return JEPA_B200_ERR_ARG;
+  if (m->cfg.pred_depth < 1) return JEPA_B200_ERR_ARG;
+  if (n_ctx > m->N || n_tgt > m->N) return JEPA_B200_ERR_ARG;
+  for (int i = 0; i < n_ctx; ++i)
+    if (ctx_idx[i] < 0 || ctx_idx[i] >= m->N) return JEPA_B200_ERR_ARG;
+  for (int i = 0; i < n_tgt; ++i)
+    if (tgt_idx[i] < 0 || tgt_idx[i] >= m->N) return JEPA_B200_ERR_ARG;
+  const long long rows = static_cast<long long>(B) * (n_ctx + n_tgt);
+  if (rows * std::max(m->cfg.pred_mlp, 4096) >= (1ll << 31) ||
+      static_cast<long long>(B) * m->N * m->cfg.dim >= (1ll << 31))
+    return JEPA_B200_ERR_SHAPE;
+  if (out_bytes < static_cast<size_t>(B) * n_tgt * m->cfg.dim * 4) return JEPA_B200_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(tokens) & 15) || (reinterpret_cast<uintptr_t>(out) & 15)) return JEPA_B200_ERR_ARG;
+  DeviceGuard guard(m->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int L = n_ctx + n_tgt, Lpad = (L + 127) / 128 * 128;
+  int s;
+  if ((s = pred_workspace(m, static_cast<size_t>(rows), static_cast<size_t>(B) * n_ctx,
+                          static_cast<size_t>(B) * n_tgt, static_cast<size_t>(B) * m->cfg.pred_heads * 64 * Lpad)))
+    return s;
+  // index lists, uploaded when they change (ctx at [0, N), tgt at [N, 2N))
+  std::vector<int> h(static_cast<size_t>(2) * m->N, 0);
+  std::copy(ctx_idx, ctx_idx + n_ctx, h.begin());
+  std::copy(tgt_idx, tgt_idx + n_tgt, h.begin() + m->N);
+  h.push_back(n_ctx);
+  h.push_back(n_tgt);
+  if (h != m->pidx_host) {
+    if (cudaMemcpyAsync(m->pidx, h.data(), static_cast<size_t>(2) * m->N * sizeof(int), cudaMemcpyHostToDevice, st) !=
+        cudaSuccess)
+      return JEPA_B200_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return JEPA_B200_ERR_CUDA;  // h is a temporary
+    m->pidx_host = h;
+  }
+  if (B != m->pops_B || n_ctx != m->pops_ctx || n_tgt != m->pops_tgt || tokens != m->pops_tokens ||
+      out != m->pops_out) {
+    m->pops_B = 0;
+    if ((s = prepare_pred_ops(m, tokens, B, n_ctx, n_tgt, out))) return s;
+    m->pops_B = B;
+    m->pops_ctx = n_ctx;
+    m->pops_tgt = n_tgt;
+    m->pops_tokens = tokens;
+    m->pops_out = out;
+  }
+  m->launches = 0;
+  m->have_timing = false;
+  if (cudaEventRecord(m->ev0, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+  if ((s = enqueue_predict(m, tokens, B, n_ctx, n_tgt, st))) return s;
   if (cudaEventRecord(m->ev1, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
   m->have_timing = true;
   return JEPA_B200_OK;
@@ -1040,6 +1283,7 @@ void jepa_b200_free(jepa_b200_model* m) {
   DeviceGuard guard(m->device);
   cudaDeviceSynchronize();
   free_list(m->ws_allocs);
+  free_list(m->pws_allocs);
   free_list(m->allocs);
   if (m->stage_pix) cudaFree(m->stage_pix);
   if (m->stage_out) cudaFree(m->stage_out);

@@ -18,17 +18,29 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-template <int MAXV, bool OUT_F16>
-__global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict__ x, int rows, int D,
-                                                       long long in_stride, const float* __restrict__ g,
-                                                       const float* __restrict__ b, float eps, void* out) {
+// Output row r reads input row (r / grp) * grp_stride + grp_off + r % grp:
+// consecutive rows (grp >= rows, grp_stride 0, grp_off 0), every in_stride-th
+// row (grp 1, grp_stride in_stride), or a block of grp rows at offset grp_off
+// in every group of grp_stride rows.
+struct RowMap {
+  int grp;
+  long long grp_stride;
+  int grp_off;
+};
+
+template <int MAXV, bool OUT_F16, bool BF>
+__global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict__ x, int rows, int D, RowMap map,
+                                                       const float* __restrict__ g, const float* __restrict__ b,
+                                                       float eps, void* out) {
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nv = D >> 2;
   // grid-stride over rows: the grid is sized to the resident capacity
   for (int row = blockIdx.x * 8 + warp; row < rows; row += gridDim.x * 8) {
-    const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(row) * in_stride * D);
+    const int gi = row / map.grp;
+    const long long in_row = gi * map.grp_stride + map.grp_off + (row - gi * map.grp);
+    const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(in_row) * D);
     float4 v[MAXV];
     float s = 0.0f;
 #pragma unroll
@@ -64,7 +76,7 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
         const float y3 = (v[i].w - mean) * rstd * gg.w + bb.w;
         if (OUT_F16) {
           uint2* o = reinterpret_cast<uint2*>(static_cast<__half*>(out) + static_cast<size_t>(row) * D) + idx;
-          *o = make_uint2(pack_half2(y0, y1), pack_half2(y2, y3));
+          *o = make_uint2(pack2<BF>(y0, y1), pack2<BF>(y2, y3));
         } else {
           float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + static_cast<size_t>(row) * D) + idx;
           *o = make_float4(y0, y1, y2, y3);
@@ -74,23 +86,41 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
   }
 }
 
-int launch_layernorm(const float* x, int rows, int D, long long in_stride, const float* g, const float* b,
-                     float eps, void* out, bool out_f16, cudaStream_t st) {
-  if (!x || !g || !b || !out) return JEPA_B200_ERR_ARG;
-  if (rows < 1 || D < 4 || D % 4 != 0 || D > 4096 || in_stride < 1) return JEPA_B200_ERR_SHAPE;
+template <bool BF>
+static void launch_ln(const float* x, int rows, int D, RowMap map, const float* g, const float* b, float eps,
+                      void* out, bool out16, cudaStream_t st) {
   const dim3 grid(std::min((rows + 7) / 8, num_sms() * 8));
   if (D <= 1024) {
-    if (out_f16)
-      launch_pdl(layernorm_kernel<8, true>, grid, dim3(256), 0, st, 1, x, rows, D, in_stride, g, b, eps, out);
+    if (out16)
+      launch_pdl(layernorm_kernel<8, true, BF>, grid, dim3(256), 0, st, 1, x, rows, D, map, g, b, eps, out);
     else
-      launch_pdl(layernorm_kernel<8, false>, grid, dim3(256), 0, st, 1, x, rows, D, in_stride, g, b, eps, out);
+      launch_pdl(layernorm_kernel<8, false, BF>, grid, dim3(256), 0, st, 1, x, rows, D, map, g, b, eps, out);
   } else {
-    if (out_f16)
-      launch_pdl(layernorm_kernel<32, true>, grid, dim3(256), 0, st, 1, x, rows, D, in_stride, g, b, eps, out);
+    if (out16)
+      launch_pdl(layernorm_kernel<32, true, BF>, grid, dim3(256), 0, st, 1, x, rows, D, map, g, b, eps, out);
     else
-      launch_pdl(layernorm_kernel<32, false>, grid, dim3(256), 0, st, 1, x, rows, D, in_stride, g, b, eps, out);
+      launch_pdl(layernorm_kernel<32, false, BF>, grid, dim3(256), 0, st, 1, x, rows, D, map, g, b, eps, out);
   }
+}
+
+int launch_layernorm_rows(const float* x, int rows, int D, int grp, long long grp_stride, int grp_off, const float* g,
+                          const float* b, float eps, void* out, bool out_f16, cudaStream_t st, bool bf16) {
+  if (!x || !g || !b || !out) return JEPA_B200_ERR_ARG;
+  if (rows < 1 || D < 4 || D % 4 != 0 || D > 4096 || grp < 1 || grp_stride < 0 || grp_off < 0)
+    return JEPA_B200_ERR_SHAPE;
+  const RowMap map{grp, grp_stride, grp_off};
+  if (bf16)
+    launch_ln<true>(x, rows, D, map, g, b, eps, out, out_f16, st);
+  else
+    launch_ln<false>(x, rows, D, map, g, b, eps, out, out_f16, st);
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+}
+
+int launch_layernorm(const float* x, int rows, int D, long long in_stride, const float* g, const float* b,
+                     float eps, void* out, bool out_f16, cudaStream_t st, bool bf16) {
+  if (in_stride < 1) return JEPA_B200_ERR_SHAPE;
+  return in_stride == 1 ? launch_layernorm_rows(x, rows, D, rows, 0, 0, g, b, eps, out, out_f16, st, bf16)
+                        : launch_layernorm_rows(x, rows, D, 1, in_stride, 0, g, b, eps, out, out_f16, st, bf16);
 }
 
 // x[b, 0, :] = cls + pos[0]
@@ -105,6 +135,67 @@ __global__ void cls_rows_kernel(float* x, int B, int ntok, int D, const float* c
 int launch_cls_rows(float* x, int B, int ntok, int D, const float* cls, const float* pos, cudaStream_t st) {
   if (!x || !cls || !pos) return JEPA_B200_ERR_ARG;
   launch_pdl(cls_rows_kernel, dim3((D + 255) / 256, B), dim3(256), 0, st, 1, x, B, ntok, D, cls, pos);
+  return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+}
+
+// Masked predictor, input side: the context rows of the encoder output
+// gathered and rounded to f16 (the A operand of pred.embed), and the
+// predictor's sequence [context | targets] of every clip assembled in f32.
+// One CTA per output row.
+// a[b * nsel + i, :] = f16(tokens[b, idx[i], :]); 8 columns per thread.
+template <bool BF>
+__global__ void gather_rows_f16_kernel(const float* __restrict__ tokens, const int* __restrict__ idx, int ntok,
+                                       int nsel, int D, __half* __restrict__ a) {
+  pdl_wait();
+  pdl_trigger();
+  const long long r = blockIdx.x;  // b * nsel + i
+  const long long b = r / nsel;
+  const int i = static_cast<int>(r - b * nsel);
+  const float* src = tokens + (b * ntok + idx[i]) * D;
+  __half* dst = a + r * D;
+  for (int c = threadIdx.x * 8; c < D; c += blockDim.x * 8) {
+    const float4 u = *reinterpret_cast<const float4*>(src + c), v = *reinterpret_cast<const float4*>(src + c + 4);
+    *reinterpret_cast<uint4*>(dst + c) =
+        make_uint4(pack2<BF>(u.x, u.y), pack2<BF>(u.z, u.w), pack2<BF>(v.x, v.y), pack2<BF>(v.z, v.w));
+  }
+}
+
+int launch_gather_rows_f16(const float* tokens, const int* idx, int B, int ntok, int nsel, int D, __half* a,
+                           cudaStream_t st, bool bf16) {
+  if (!tokens || !idx || !a) return JEPA_B200_ERR_ARG;
+  if (B < 1 || nsel < 1 || ntok < 1 || D < 8 || D % 8 != 0) return JEPA_B200_ERR_SHAPE;
+  launch_pdl(bf16 ? gather_rows_f16_kernel<true> : gather_rows_f16_kernel<false>,
+             dim3(static_cast<unsigned>(B) * nsel), dim3(128), 0, st, 1, tokens, idx, ntok, nsel, D, a);
+  return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+}
+
+// x[b, i, :] = e[b * nctx + i, :] + pos[ctx[i], :]            (i < nctx)
+// x[b, nctx + t, :] = mask[:] + pos[tgt[t], :]                 (t < ntgt)
+__global__ void pred_assemble_kernel(const float* __restrict__ e, const float* __restrict__ mask,
+                                     const float* __restrict__ pos, const int* __restrict__ ctx,
+                                     const int* __restrict__ tgt, int nctx, int ntgt, int D, float* __restrict__ x) {
+  pdl_wait();
+  pdl_trigger();
+  const int L = nctx + ntgt;
+  const long long r = blockIdx.x;  // b * L + j
+  const long long b = r / L;
+  const int j = static_cast<int>(r - b * L);
+  const bool is_ctx = j < nctx;
+  const float* prow = pos + static_cast<size_t>(is_ctx ? ctx[j] : tgt[j - nctx]) * D;
+  const float* srow = is_ctx ? e + (b * nctx + j) * D : mask;
+  float* xrow = x + r * D;
+  for (int c = threadIdx.x * 4; c < D; c += blockDim.x * 4) {
+    const float4 u = *reinterpret_cast<const float4*>(srow + c), v = *reinterpret_cast<const float4*>(prow + c);
+    *reinterpret_cast<float4*>(xrow + c) = make_float4(u.x + v.x, u.y + v.y, u.z + v.z, u.w + v.w);
+  }
+}
+
+int launch_pred_assemble(const float* e, const float* mask, const float* pos, const int* ctx, const int* tgt, int B,
+                         int nctx, int ntgt, int D, float* x, cudaStream_t st) {
+  if (!e || !mask || !pos || !ctx || !tgt || !x) return JEPA_B200_ERR_ARG;
+  if (B < 1 || nctx < 1 || ntgt < 1 || D < 4 || D % 4 != 0) return JEPA_B200_ERR_SHAPE;
+  launch_pdl(pred_assemble_kernel, dim3(static_cast<unsigned>(B) * (nctx + ntgt)), dim3(128), 0, st, 1, e, mask, pos,
+             ctx, tgt, nctx, ntgt, D, x);
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 
@@ -189,6 +280,7 @@ int launch_repack(int bmode, const uint8_t* blocks, int N, int K, void* qs, __ha
 // (q4_0), d the scale of its 32-element block; the product is exact in f32
 // (an 8-bit integer times an 11-bit significand) and rounded once to f16.
 // One thread writes 8 consecutive elements of one block.
+template <bool BF>
 __global__ void dequant_f16_kernel(int bmode, const uint8_t* __restrict__ qs, const uint16_t* __restrict__ scales,
                                    long long n_units, int K, __half* __restrict__ out) {
   pdl_wait();
@@ -212,18 +304,20 @@ __global__ void dequant_f16_kernel(int bmode, const uint8_t* __restrict__ qs, co
     for (int i = 0; i < 8; ++i) v[i] = static_cast<float>(static_cast<int>((q[i] >> sh) & 0xF) - 8) * d;
   }
   uint4 w;
-  w.x = pack_half2(v[0], v[1]);
-  w.y = pack_half2(v[2], v[3]);
-  w.z = pack_half2(v[4], v[5]);
-  w.w = pack_half2(v[6], v[7]);
+  w.x = pack2<BF>(v[0], v[1]);
+  w.y = pack2<BF>(v[2], v[3]);
+  w.z = pack2<BF>(v[4], v[5]);
+  w.w = pack2<BF>(v[6], v[7]);
   *reinterpret_cast<uint4*>(out + e0) = w;
 }
 
-int launch_dequant_f16(int bmode, const void* qs, const __half* scales, int N, int K, __half* out, cudaStream_t st) {
+int launch_dequant_f16(int bmode, const void* qs, const __half* scales, int N, int K, __half* out, cudaStream_t st,
+                       bool bf16) {
   if (!qs || !scales || !out) return JEPA_B200_ERR_ARG;
   if ((bmode != B_Q8 && bmode != B_Q4) || N < 1 || K < 32 || K % 32 != 0) return JEPA_B200_ERR_SHAPE;
   const long long units = static_cast<long long>(N) * K / 8;
-  launch_pdl(dequant_f16_kernel, dim3(static_cast<unsigned>((units + 255) / 256)), dim3(256), 0, st, 1, bmode,
+  launch_pdl(bf16 ? dequant_f16_kernel<true> : dequant_f16_kernel<false>,
+             dim3(static_cast<unsigned>((units + 255) / 256)), dim3(256), 0, st, 1, bmode,
              static_cast<const uint8_t*>(qs), reinterpret_cast<const uint16_t*>(scales), units, K, out);
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }

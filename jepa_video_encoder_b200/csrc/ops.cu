@@ -52,6 +52,12 @@ int make_matrix(DevMatrix* W, const void* w, const void* scales, int dtype, int 
   W->K = K;
   W->data = const_cast<void*>(w);
   W->scales = static_cast<__half*>(const_cast<void*>(scales));
+  // the caller's [N, K/32] scales serve the CTA-pair kernel's staged loader
+  // when their rows are whole 16-byte groups (K a multiple of 256) and 16-byte aligned
+  if (bm != B_F16 && (K / 32) % 8 == 0 && aligned16(scales)) {
+    W->scales_pad = W->scales;
+    W->sc_ld = K / 32;
+  }
   return JEPA_B200_OK;
 }
 

@@ -72,6 +72,7 @@ class EncoderConfig:
     pix_std: tuple = IMAGENET_STD
     random_ln_affine: bool = False   # tests: exercise gamma/beta instead of 1/0
     rope: bool = False               # 3-D rotary positions in the attention instead of pos_embed (no CLS)
+    act_bf16: bool = False           # bf16 instead of f16 for the kernels' 16-bit activations and operands
 
     # -- derived shapes ---------------------------------------------------
     @property
@@ -143,11 +144,15 @@ VJEPA2_LONG = EncoderConfig(
 # (instead of an additive table).
 VJEPA2_LONG_ROPE = VJEPA2_LONG.with_(name="vjepa2_vit_l16_64f256_rope_b2", rope=True)
 VJEPA2_SSV2_ROPE = VJEPA2_SSV2.with_(name="vjepa2_vit_l16_16f256_ssv2_q8_rope_b8", rope=True)
+# The LeVJEPA workload with bf16 activations (the same f16 weight table,
+# rounded to bf16 at load).
+LEVJEPA_VIT_L_BF16 = LEVJEPA_VIT_L.with_(name="levjepa_vit_l16_16f224_b4_bf16", act_bf16=True)
 
 WORKLOADS: Dict[str, EncoderConfig] = {
     c.name: c for c in (LEWM_VIT_TI, LEWM_VIT_TI_B8, LEWM_VIT_TI_B32, LEVJEPA_VIT_L,
                         VJEPA2_SSV2, LEVJEPA_VIT_L_Q4, LEVJEPA_VIT_L_Q4_B1,
-                        LEVJEPA_VIT_L_Q4_B32, VJEPA2_LONG, VJEPA2_LONG_ROPE, VJEPA2_SSV2_ROPE)}
+                        LEVJEPA_VIT_L_Q4_B32, VJEPA2_LONG, VJEPA2_LONG_ROPE, VJEPA2_SSV2_ROPE,
+                        LEVJEPA_VIT_L_BF16)}
 
 
 @dataclass(frozen=True)

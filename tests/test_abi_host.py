@@ -57,7 +57,7 @@ def _tiny_cfg(**kw):
     return base.with_(**kw)
 
 
-def _load(lib, cfg, table):
+def _load(lib, cfg, table, predictor=None):
     entries = (_abi.TensorEntry * len(table))()
     keep = []
     for i, t in enumerate(table):
@@ -70,7 +70,7 @@ def _load(lib, cfg, table):
             entries[i].shape[j] = s
         entries[i].data = t.data.ctypes.data
         entries[i].nbytes = t.nbytes
-    c = make_config(cfg)
+    c = make_config(cfg, predictor=predictor)
     h = ctypes.c_void_p()
     st = lib.jepa_b200_load_weights(ctypes.byref(c), entries, len(table), 0, ctypes.byref(h))
     if st == 0:
@@ -201,3 +201,30 @@ def test_null_arguments(lib):
     assert lib.jepa_b200_model_n_bytes(None) == 0
     assert lib.jepa_b200_last_ms(None) < 0
     lib.jepa_b200_free(None)
+
+
+def test_predictor_config_and_table_validation(lib):
+    """The predictor's shape limits (width a multiple of 64, head dim 32 or
+    64, MLP a multiple of 64) and its tensors, checked on the host."""
+    cfg = _tiny_cfg(mask="bidir", has_cls=False)
+    ok = 0 if _has_gpu() else _abi.ERR_CUDA
+    pc = synth.PredictorConfig(name="p", enc=cfg, dim=128, depth=1, heads=4, mlp=256)
+    table = synth.make_tensor_table(cfg) + synth.make_predictor_table(pc)
+    assert _load(lib, cfg, table, pc) == ok
+    assert _load(lib, cfg, table, pc.with_(heads=2)) == ok                       # head dim 64
+    assert _load(lib, cfg, table, pc.with_(heads=8)) == _abi.ERR_SHAPE           # head dim 16
+    assert _load(lib, cfg, table, pc.with_(dim=96, heads=3)) == _abi.ERR_SHAPE    # width not a multiple of 64
+    assert _load(lib, cfg, table, pc.with_(mlp=200)) == _abi.ERR_SHAPE
+    assert _load(lib, cfg, table, pc.with_(depth=-1)) == _abi.ERR_ARG
+    assert _load(lib, cfg, [t for t in table if t.name != "pred.mask_tokens"], pc) == _abi.ERR_MISSING_TENSOR
+    assert _load(lib, cfg, [t for t in table if t.name != "pred.blk.0.ffn_down.bias"], pc) == \
+        _abi.ERR_MISSING_TENSOR
+    # pred.embed / pred.proj may be quantised (re-typed), pred.pos_embed may not
+    q = synth.make_tensor_table(cfg) + synth.make_predictor_table(pc.with_(weights="q8_0"))
+    assert {t.name: t.dtype for t in q}["pred.embed.weight"] == synth.DT_Q8_0
+    assert _load(lib, cfg, q, pc) == ok
+    bad = list(table)
+    i = [t.name for t in bad].index("pred.pos_embed")
+    bad[i] = synth.Tensor("pred.pos_embed", synth.DT_Q8_0, bad[i].shape,
+                          synth.quantize_q8_0(np.zeros(bad[i].shape, np.float32)))
+    assert _load(lib, cfg, bad, pc) == _abi.ERR_DTYPE

@@ -309,3 +309,29 @@ def test_vjepa2_long_rope_full_size_sampled():
     cfg = synth.VJEPA2_LONG.with_(name="vjepa2_vit_l16_64f256_rope_b2", rope=True)
     m, table, pix, W = _full_size_layers(cfg, [0, 23], [0, 1], _rows)
     m.close()
+
+
+@pytest.mark.parametrize("name", ["vjepa2_ssv2", "levjepa_q4"])
+def test_quant_loader_unpack_matches_f16_copy_bitwise(name):
+    """A q8_0 / q4_0 model keeps its blocks only (every GEMM unpacks them in
+    its loader) or, on request, also an f16 copy for the large GEMMs: the
+    copy holds exactly the unpacked values, so both forwards agree bit for
+    bit, and the blocks-only model holds fewer bytes.  (Batches of 320 and
+    258 rows: the CTA-pair GEMMs with and without the copy.)"""
+    need_cuda()
+    cfg = SMALL[name] if name != "vjepa2_ssv2" else SMALL[name].with_(batch=5)
+    table = synth.make_tensor_table(cfg)
+    pix = synth.make_pixels(cfg)
+    outs, sizes = [], []
+    for copy in (False, True):
+        m = jb.Model(cfg, table, quant_f16_copy=copy)
+        outs.append(m.encode(dev(pix), pool="none").cpu().numpy())
+        if cfg.pool == "attentive":
+            outs.append(m.encode(dev(pix), pool="attentive").cpu().numpy())
+        assert m.sync_status() == 0
+        sizes.append(m.n_bytes)
+        m.close()
+    half = len(outs) // 2
+    for a, b in zip(outs[:half], outs[half:]):
+        assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    assert sizes[0] < sizes[1]
