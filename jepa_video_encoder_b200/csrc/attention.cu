@@ -640,388 +640,6 @@ __global__ void __launch_bounds__(AttnCfg<TILES>::kThreads, TILES == 2 ? 1 : 2)
   }
 }
 
-// ---------------------------------------------------------------------------
-// Block-causal layout with 64-key KV sub-tiles.  One 128-query tile per CTA,
-// two CTAs per SM; TMEM holds two S buffers (64 keys each), O and two P
-// buffers (256 columns), so S of sub-tile j + 1 is computed into the other
-// buffer while the softmax works on sub-tile j, and S_j stays in TMEM until
-// the row maxima of sub-tile j are known.  The softmax therefore starts its
-// exponentials against the running max right after loading the scores
-// (speculatively) and reduces the maxima alongside; only where a row's max
-// grew by more than 2^8 (the lazy-rescale rule, so the result is the same
-// either way) are the scores read again and the exponentials redone.
-// Four threads of one warp share each pair of query rows (16x256b /
-// 16x128b TMEM shapes), each with 16 of a sub-tile's 64 keys of two rows.
-namespace {
-constexpr int kSub = 64;                   // keys per KV sub-tile
-constexpr int kSubTile = kSub * 64 * 2;    // one [64 x 64] f16 tile, 8 KB
-struct Attn64Cfg {
-  static constexpr int kStages = 4;
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kTile;                       // K ring: [64 keys x 64 dims] each
-  static constexpr int kOffV = kOffK + kStages * kSubTile;  // V^T ring: [64 dims x 64 keys] each
-  static constexpr int kSmem = kOffV + kStages * kSubTile + 1024;
-  // TMEM columns: S (2 x 64 keys, f32), O (64 dims, f32), P (2 x 32 columns of f16 pairs)
-  static constexpr uint32_t kColS = 0, kColO = 128, kColP = 192, kTmemCols = 256;
-  static constexpr int kThreads = 10 * 32;
-};
-}  // namespace
-
-// KV sub-tiles query tile q0 must visit (0: no valid row).
-__device__ __forceinline__ int kv_subtiles(const AttnParams& p, int q0) {
-  if (q0 >= p.N) return 0;
-  int lo_a, hi_a, lo_b, hi_b;
-  key_range(p, q0, lo_a, hi_a);
-  key_range(p, min(q0 + 127, p.N - 1), lo_b, hi_b);
-  return (max(hi_a, hi_b) + kSub) / kSub;
-}
-
-// Scores of sub-tile j for this thread's 16 keys of rows a and b (16x256b
-// shape, 8 repetitions of 8 columns), masked outside [lo, hi].
-__device__ __forceinline__ void bc64_load(uint32_t tS, int j, int kq, int loa, int hia, int lob, int hib,
-                                          float (&sc)[32]) {
-  uint32_t u[32];
-  tmem_ld_16x256b_x8(tS, u);
-#pragma unroll
-  for (int e = 0; e < 32; ++e) sc[e] = __uint_as_float(u[e]);
-  const int kbase = j * kSub;
-  const bool full = loa <= kbase && hia >= kbase + kSub - 1 && lob <= kbase && hib >= kbase + kSub - 1;
-  if (!__all_sync(0xffffffffu, full)) {
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      const int key = kbase + 8 * m + 2 * kq;
-      sc[4 * m] = (key >= loa && key <= hia) ? sc[4 * m] : -INFINITY;
-      sc[4 * m + 1] = (key + 1 >= loa && key + 1 <= hia) ? sc[4 * m + 1] : -INFINITY;
-      sc[4 * m + 2] = (key >= lob && key <= hib) ? sc[4 * m + 2] : -INFINITY;
-      sc[4 * m + 3] = (key + 1 >= lob && key + 1 <= hib) ? sc[4 * m + 3] : -INFINITY;
-    }
-  }
-}
-
-// P = exp2(s*c - m) for rows a and b (m finite): 16 words of f16 (or bf16)
-// pairs in the 16x128b order and the two row sums.
-template <bool BF>
-__device__ __forceinline__ void bc64_exp(const float (&sc)[32], float c, float ma, float mb, uint32_t (&pk)[16],
-                                         float& suma, float& sumb) {
-  const uint64_t c2 = f2_pack(c, c), nma = f2_pack(-ma, -ma), nmb = f2_pack(-mb, -mb);
-  uint64_t sa[2] = {0ull, 0ull}, sb[2] = {0ull, 0ull};
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    float x0, x1, x2, x3;
-    f2_unpack(f2_fma(f2_pack(sc[4 * m], sc[4 * m + 1]), c2, nma), x0, x1);
-    f2_unpack(f2_fma(f2_pack(sc[4 * m + 2], sc[4 * m + 3]), c2, nmb), x2, x3);
-    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-    const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
-    sa[m & 1] = f2_add(sa[m & 1], f2_pack(p0, p1));
-    sb[m & 1] = f2_add(sb[m & 1], f2_pack(p2, p3));
-    pk[2 * m] = pack2<BF>(p0, p1);
-    pk[2 * m + 1] = pack2<BF>(p2, p3);
-  }
-  float t0, t1, t2, t3;
-  f2_unpack(f2_add(sa[0], sa[1]), t0, t1);
-  f2_unpack(f2_add(sb[0], sb[1]), t2, t3);
-  suma = t0 + t1;
-  sumb = t2 + t3;
-}
-
-template <bool BF>
-__global__ void __launch_bounds__(Attn64Cfg::kThreads, 2)
-    attn_bc64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using C = Attn64Cfg;
-  constexpr int S = C::kStages;
-  extern __shared__ uint8_t dsmem[];
-  __shared__ uint64_t q_full, k_full[S], k_empty[S], v_full[S], v_empty[S];
-  __shared__ uint64_t s_full[2], s_free[2], p_full[2], pv_done[2], drain_bar;
-  __shared__ uint32_t tmem_sh;
-  __shared__ int abort_sh;
-
-  const uint32_t raw = smem_u32(dsmem);
-  uint8_t* sm = dsmem + ((1024u - (raw & 1023u)) & 1023u);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // grid (clip*head, unit): the hardware starts the heaviest units of every head first
-  const int unit = static_cast<int>(blockIdx.y), bh = static_cast<int>(blockIdx.x);
-  const int cls_unit = p.cls_separate && !p.cls_tail;
-  const bool cls_cta = cls_unit && unit == 0;
-  const int q0 = cls_cta ? 0 : (p.n_q_tiles - 1 - (unit - cls_unit)) * 128;
-  const int nkv = cls_cta ? (p.N + kSub - 1) / kSub : kv_subtiles(p, q0);
-  // the CLS query rides in row N, the first padding row of the last query tile
-  const bool tail_cls = p.cls_tail && !cls_cta && q0 == (p.n_q_tiles - 1) * 128;
-
-  if (threadIdx.x == 0) {
-    mbar_init(&q_full, 1);
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 256);
-      mbar_init(&p_full[b], 256);
-      mbar_init(&pv_done[b], 1);
-    }
-    mbar_init(&drain_bar, 1);
-    abort_sh = 0;
-    mbar_fence_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(&tmem_sh, C::kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_sh;
-  pdl_wait();  // Q, K, V^T come from the previous kernel
-  pdl_trigger();
-
-  WaitCtl w;
-  w.abort = reinterpret_cast<volatile int*>(&abort_sh);
-  w.err = p.err;
-  w.timeout_ns = p.timeout_ns;
-  w.where = (KID_ATTN << 8) | 0x40u | static_cast<unsigned>(warp);
-
-  if (warp == 0) {
-    if (lane == 0) {
-      bool ok = true;
-      uint32_t karmed = 0, kpar = 0, varmed = 0, vpar = 0;
-      mbar_expect_tx(&q_full, kTile);
-      tma_load_3d(sm + C::kOffQ, &tmQ, &q_full, 0, q0, bh);
-      for (int j = 0; j < nkv; ++j) {
-        const int s = j % S;
-        const uint32_t ph = (j / S) & 1;
-        if (!mbar_wait(&k_empty[s], ph ^ 1, w)) {
-          ok = false;
-          break;
-        }
-        mbar_expect_tx(&k_full[s], kSubTile);
-        tma_load_3d(sm + C::kOffK + s * kSubTile, &tmK, &k_full[s], 0, j * kSub, bh);
-        karmed |= 1u << s;
-        kpar = (kpar & ~(1u << s)) | (ph << s);
-        if (!mbar_wait(&v_empty[s], ph ^ 1, w)) {
-          ok = false;
-          break;
-        }
-        mbar_expect_tx(&v_full[s], kSubTile);
-        tma_load_3d(sm + C::kOffV + s * kSubTile, &tmV, &v_full[s], j * kSub, 0, bh);
-        varmed |= 1u << s;
-        vpar = (vpar & ~(1u << s)) | (ph << s);
-      }
-      if (!ok) {  // let the copies already issued land before the CTA exits
-        mbar_wait_drain(&q_full, 0);
-        for (int s = 0; s < S; ++s) {
-          if ((karmed >> s) & 1u) mbar_wait_drain(&k_full[s], (kpar >> s) & 1u);
-          if ((varmed >> s) & 1u) mbar_wait_drain(&v_full[s], (vpar >> s) & 1u);
-        }
-      }
-    }
-  } else if (warp == 1) {
-    bool okq = true;
-    if (tail_cls) {
-      // once the Q tile has landed (rows past N zero-filled), eight lanes
-      // write Q[bh, 0, :] into row N - q0 in the 128-byte-swizzled layout
-      okq = __all_sync(0xffffffffu, mbar_wait(&q_full, 0, w));
-      if (okq && lane < 8) {
-        const uint4 v = *reinterpret_cast<const uint4*>(p.q + static_cast<size_t>(bh) * p.N * 64 + lane * 8);
-        st_shared_v4(smem_u32(sm + C::kOffQ) + sw128_offset(p.N - q0, lane * 8), v.x, v.y, v.z, v.w);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-    }
-    if (lane == 0 && okq) {
-      constexpr uint32_t idesc_s = idesc_f16_f32(128, kSub, BF);
-      constexpr uint32_t idesc_o = idesc_f16_f32(128, 64, BF);
-      const uint64_t qd = sdesc_kmajor_sw128(smem_u32(sm + C::kOffQ));
-      bool ok = mbar_wait(&q_full, 0, w);
-      for (int j = 0; ok && j <= nkv; ++j) {
-        if (j < nkv) {  // S[j & 1] = Q K_j^T once sub-tile j - 2 released that buffer
-          const int ks = j % S;
-          if (!mbar_wait(&k_full[ks], (j / S) & 1, w)) {
-            ok = false;
-            break;
-          }
-          if (j >= 2 && !mbar_wait(&s_free[j & 1], ((j - 2) >> 1) & 1, w)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t kd = sdesc_kmajor_sw128(smem_u32(sm + C::kOffK + ks * kSubTile));
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc_mma_f16_ss(tmem + C::kColS + kSub * (j & 1), qd + static_cast<uint64_t>(2 * k),
-                          kd + static_cast<uint64_t>(2 * k), idesc_s, k > 0 ? 1u : 0u);
-          tc_commit(&s_full[j & 1]);
-          tc_commit(&k_empty[ks]);
-        }
-        if (j >= 1) {  // O += P[(j-1) & 1] V_{j-1} once the softmax published P_{j-1}
-          const int i = j - 1, vs = i % S;
-          if (!mbar_wait(&v_full[vs], (i / S) & 1, w)) {
-            ok = false;
-            break;
-          }
-          if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, w)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t vd = sdesc_kmajor_sw128(smem_u32(sm + C::kOffV + vs * kSubTile));
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc_mma_f16_ts(tmem + C::kColO, tmem + C::kColP + 32 * (i & 1) + 8 * k, vd + static_cast<uint64_t>(2 * k),
-                          idesc_o, (i > 0 || k > 0) ? 1u : 0u);
-          tc_commit(&pv_done[i & 1]);
-          tc_commit(&v_empty[vs]);
-        }
-      }
-      tc_commit(&drain_bar);
-      mbar_wait_drain(&drain_bar, 0);
-    }
-  } else {
-    // softmax warps 2-9: the two warps of a TMEM lane quadrant take its 32
-    // rows in halves of 16; four threads share a pair of rows (ra, ra + 8)
-    const int hh = ((warp - 2) >> 2) & 1;
-    const int quad = warp & 3;
-    const int lane_base = quad * 32 + hh * 16;
-    const int kq = lane & 3;
-    const int ra = lane_base + (lane >> 2);
-    const int ia = q0 + ra, ib = ia + 8;
-    const uint32_t lane_off = static_cast<uint32_t>(lane_base) << 16;
-    const uint32_t tS = tmem + C::kColS + lane_off;
-    const uint32_t tO = tmem + C::kColO + lane_off;
-    const uint32_t tP = tmem + C::kColP + lane_off;
-    int loa, hia, lob, hib;
-    row_keys(p, cls_cta, ia, loa, hia);
-    row_keys(p, cls_cta, ib, lob, hib);
-    const float c = p.scale_log2;
-    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.0f, l_b = 0.0f;  // l: this thread's share of the row sum
-    bool ok = true;
-    for (int j = 0; ok && j < nkv; ++j) {
-      const int bsel = j & 1;
-      const uint32_t tSj = tS + static_cast<uint32_t>(kSub * bsel);
-      bool okw = mbar_wait(&s_full[bsel], (j >> 1) & 1, w);
-      if (!__all_sync(0xffffffffu, okw)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const bool spec = __all_sync(0xffffffffu, m_a != -INFINITY && m_b != -INFINITY);
-      uint32_t pk[16];
-      float suma = 0.0f, sumb = 0.0f;
-      float xa, xb;
-      {
-        float sc[32];
-        bc64_load(tSj, j, kq, loa, hia, lob, hib, sc);
-        xa = fmaxf(sc[0], sc[1]);
-        xb = fmaxf(sc[2], sc[3]);
-#pragma unroll
-        for (int m = 1; m < 8; ++m) {
-          xa = fmax3(xa, sc[4 * m], sc[4 * m + 1]);
-          xb = fmax3(xb, sc[4 * m + 2], sc[4 * m + 3]);
-        }
-        if (spec) bc64_exp<BF>(sc, c, m_a, m_b, pk, suma, sumb);
-      }
-      xa = fmaxf(xa, __shfl_xor_sync(0xffffffffu, xa, 1));
-      xb = fmaxf(xb, __shfl_xor_sync(0xffffffffu, xb, 1));
-      xa = fmaxf(xa, __shfl_xor_sync(0xffffffffu, xa, 2));
-      xb = fmaxf(xb, __shfl_xor_sync(0xffffffffu, xb, 2));
-      const float mna = fmaxf(m_a, xa * c), mnb = fmaxf(m_b, xb * c);
-      const bool ga = mna > m_a + kRescaleLog2, gb = mnb > m_b + kRescaleLog2;
-      const float alpha_a = ga ? ex2_approx(m_a - mna) : 1.0f;  // exp2(-inf) = 0 before the first key
-      const float alpha_b = gb ? ex2_approx(m_b - mnb) : 1.0f;
-      l_a *= alpha_a;
-      l_b *= alpha_b;
-      if (ga) m_a = mna;
-      if (gb) m_b = mnb;
-      const bool regrow = __any_sync(0xffffffffu, ga || gb);
-      if (!spec || regrow) {  // warp-collective: S_j is still in TMEM
-        float sc[32];
-        bc64_load(tSj, j, kq, loa, hia, lob, hib, sc);
-        // a row that has seen no allowed key yet keeps m = -inf: all its p are 0
-        bc64_exp<BF>(sc, c, m_a == -INFINITY ? 0.0f : m_a, m_b == -INFINITY ? 0.0f : m_b, pk, suma, sumb);
-      }
-      tc_fence_before();
-      mbar_arrive(&s_free[bsel]);  // S buffer bsel may take sub-tile j + 2
-      // P buffer bsel is free once PV_{j-2} is done; O is stable for a
-      // rescale once PV_{j-1} is done
-      if (j >= 2) {
-        okw = mbar_wait(&pv_done[bsel], ((j - 2) >> 1) & 1, w);
-        if (!__all_sync(0xffffffffu, okw)) {
-          ok = false;
-          break;
-        }
-      }
-      if (j >= 1 && regrow) {
-        okw = mbar_wait(&pv_done[bsel ^ 1], ((j - 1) >> 1) & 1, w);
-        if (!__all_sync(0xffffffffu, okw)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        uint32_t o[32];
-        tmem_ld_16x256b_x8(tO, o);
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          o[4 * m] = __float_as_uint(__uint_as_float(o[4 * m]) * alpha_a);
-          o[4 * m + 1] = __float_as_uint(__uint_as_float(o[4 * m + 1]) * alpha_a);
-          o[4 * m + 2] = __float_as_uint(__uint_as_float(o[4 * m + 2]) * alpha_b);
-          o[4 * m + 3] = __float_as_uint(__uint_as_float(o[4 * m + 3]) * alpha_b);
-        }
-        tmem_st_16x256b_x8(tO, o);
-      }
-      tc_fence_after();
-      tmem_st_16x128b_x8(tP + static_cast<uint32_t>(32 * bsel), pk);
-      l_a += suma;
-      l_b += sumb;
-      tc_fence_before();
-      mbar_arrive(&p_full[bsel]);
-    }
-    if (ok && nkv > 0) {  // the last PV product completes after all earlier ones
-      bool okw = mbar_wait(&pv_done[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1, w);
-      okw = __all_sync(0xffffffffu, okw);
-      l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-      l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-      l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-      l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-      if (okw) {
-        tc_fence_after();
-        const float inv_a = l_a > 0.0f ? 1.0f / l_a : 0.0f;
-        const float inv_b = l_b > 0.0f ? 1.0f / l_b : 0.0f;
-        const int b = bh / p.heads, hd = bh % p.heads;
-        uint32_t o[32];
-        tmem_ld_16x256b_x8(tO, o);
-        // rows this CTA writes: the CLS CTA only row 0; the others every
-        // valid row but a separately computed CLS row; row N of the last tile
-        // holds the CLS query (tail_cls): output row 0
-        const bool st_a = cls_cta ? (ia == 0) : ((ia < p.N && !(ia == 0 && p.cls_separate)) || (tail_cls && ia == p.N));
-        const bool st_b = cls_cta ? (ib == 0) : ((ib < p.N && !(ib == 0 && p.cls_separate)) || (tail_cls && ib == p.N));
-        const int oa = ia == p.N ? 0 : ia, ob = ib == p.N ? 0 : ib;
-        if (st_a) {
-          uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (static_cast<size_t>(b) * p.N + oa) * p.ldo + hd * p.dv + 2 * kq);
-#pragma unroll
-          for (int m = 0; m < 8; ++m)
-            if (8 * m < p.dv)
-              dst[4 * m] = pack2<BF>(__uint_as_float(o[4 * m]) * inv_a, __uint_as_float(o[4 * m + 1]) * inv_a);
-        }
-        if (st_b) {
-          uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (static_cast<size_t>(b) * p.N + ob) * p.ldo + hd * p.dv + 2 * kq);
-#pragma unroll
-          for (int m = 0; m < 8; ++m)
-            if (8 * m < p.dv)
-              dst[4 * m] = pack2<BF>(__uint_as_float(o[4 * m + 2]) * inv_b, __uint_as_float(o[4 * m + 3]) * inv_b);
-        }
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_sh, C::kTmemCols);
-  }
-}
-
 int attn_prepare(AttnOp* op, const __half* q, const __half* k, const __half* vt, int B, int heads, int ntok,
                  int npad, int mask, int has_cls, int ppf, __half* out, int head_dim) {
   if (!op || !q || !k || !vt || !out) return JEPA_B200_ERR_ARG;
@@ -1039,8 +657,6 @@ int attn_prepare(AttnOp* op, const __half* q, const __half* k, const __half* vt,
     const uint32_t box[3] = {64, 128, 1};
     if (!make_tmap_f16(&op->tmQ, q, 3, dims, str, box)) return JEPA_B200_ERR_CUDA;
     if (!make_tmap_f16(&op->tmK, k, 3, dims, str, box)) return JEPA_B200_ERR_CUDA;
-    const uint32_t box64[3] = {64, 64, 1};  // the 64-key sub-tiles of the block-causal layout
-    if (!make_tmap_f16(&op->tmK64, k, 3, dims, str, box64)) return JEPA_B200_ERR_CUDA;
   }
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(npad), 64, BH};
@@ -1094,23 +710,6 @@ constexpr int kTilesBidir = 2;
 constexpr bool kRowsInWarpBlockCausal = true;
 constexpr bool kRowsInWarpBidir = false;
 
-template <bool BF>
-static int attn_launch_bc64(const AttnParams& p, const AttnOp& op, cudaStream_t st) {
-  using C = Attn64Cfg;
-  auto kern = attn_bc64_kernel<BF>;
-  static std::atomic<unsigned long long> attr_done{0};
-  if (!smem_attr_once(attr_done, kern, C::kSmem)) return JEPA_B200_ERR_CUDA;
-  const int units = p.n_q_tiles + (p.cls_separate && !p.cls_tail ? 1 : 0);
-  if (launch_pdl(kern, dim3(op.B * p.heads, units), dim3(C::kThreads), C::kSmem, st, 1, op.tmQ, op.tmK64, op.tmV, p) !=
-      cudaSuccess)
-    return JEPA_B200_ERR_CUDA;
-  return JEPA_B200_OK;
-}
-
-#ifndef JB_ATTN_BC64
-#define JB_ATTN_BC64 0
-#endif
-
 int attn_launch(const AttnOp& op, cudaStream_t st, DevErr* err, unsigned long long timeout_ns) {
   AttnParams p = op.p;
   p.err = err;
@@ -1119,8 +718,6 @@ int attn_launch(const AttnOp& op, cudaStream_t st, DevErr* err, unsigned long lo
   // exchange between warps is a large share: rows kept inside one warp.
   // Bidirectional tiles are long and bound by the exponentials, where the
   // cross-warp layout issues fewer instructions.
-  if (JB_ATTN_BC64 && p.mask == JEPA_B200_MASK_BLOCK_CAUSAL)
-    return op.bf16 ? attn_launch_bc64<true>(p, op, st) : attn_launch_bc64<false>(p, op, st);
   if (p.mask == JEPA_B200_MASK_BLOCK_CAUSAL)
     return op.bf16 ? attn_launch_impl<kRowsInWarpBlockCausal, kTilesBlockCausal, true>(p, op, st)
                    : attn_launch_impl<kRowsInWarpBlockCausal, kTilesBlockCausal, false>(p, op, st);

@@ -116,7 +116,6 @@ struct AttnParams {
 
 struct AttnOp {
   CUtensorMap tmQ, tmK, tmV;
-  CUtensorMap tmK64;  // K in 64-key boxes (block-causal sub-tile layout)
   AttnParams p;
   int bf16 = 0;  // Q, K, V^T, P and the output in bf16 instead of f16
   const __half* q = nullptr;
