@@ -251,6 +251,116 @@ VJEPA2_PREDICTOR = PredictorConfig(name="vjepa2_predictor_l16_16f256_all_b8", en
                                    batch=8)
 PREDICTORS: Dict[str, "PredictorConfig"] = {VJEPA2_PREDICTOR.name: VJEPA2_PREDICTOR}
 
+@dataclass(frozen=True)
+class WorldModelConfig:
+    """The LeWM world model ("LeWorldModel Push-T" card, intro: the ViT-Ti/14
+    encoder's CLS row projected to a world-model state, six AdaLN-zero causal
+    blocks conditioned on a 10-d action; benchmarks page, "LeWM world model":
+    a 3-frame window of 192-d states).  ``dim`` is the state width (the
+    encoder's width), ``window`` the frames one predictor call reads (the
+    rows of pred.pos_embed); ``proj_hidden`` / ``pred_hidden`` the hidden
+    widths of the projector (enc.proj) and of the output MLP (pred.proj),
+    which the pages do not give (read as the blocks' MLP width).  A workload
+    is ``candidates`` independent sequences: ``frames`` observed states, and
+    ``steps`` rollout steps after them (0: one predictor call over the
+    observed frames, every row an output)."""
+    name: str
+    enc: EncoderConfig
+    dim: int = 192
+    depth: int = 6
+    heads: int = 3
+    mlp: int = 768
+    action_dim: int = 10
+    window: int = 3
+    proj_hidden: int = 768
+    pred_hidden: int = 768
+    weights: str = "f16"
+    candidates: int = 1
+    frames: int = 3
+    steps: int = 0
+    seed: int = 11
+    ln_eps: float = 1e-6
+
+    @property
+    def n_actions(self) -> int:
+        """Actions per candidate: one per observed frame, plus one per
+        predicted frame that is read again (all but the last)."""
+        return self.frames + max(0, self.steps - 1)
+
+    def with_(self, **kw) -> "WorldModelConfig":
+        return dataclasses.replace(self, **kw)
+
+
+def world_model_specs(wc: WorldModelConfig) -> List[tuple]:
+    """(name, shape, kind) of the world model's tensors in table order; the
+    kind ``w32`` marks the matrices the pages keep in f32 (adaLN, action
+    embedder)."""
+    De, D, M, A = wc.enc.dim, wc.dim, wc.mlp, wc.action_dim
+    s = [("enc.proj.0.weight", (wc.proj_hidden, De), "w"), ("enc.proj.0.bias", (wc.proj_hidden,), "b"),
+         ("enc.proj.2.weight", (D, wc.proj_hidden), "w"), ("enc.proj.2.bias", (D,), "b"),
+         ("pred.action_embed.0.weight", (D, A), "w32_act0"), ("pred.action_embed.0.bias", (D,), "b32"),
+         ("pred.action_embed.2.weight", (D, D), "w32_act2"), ("pred.action_embed.2.bias", (D,), "b32"),
+         ("pred.pos_embed", (wc.window, D), "pos")]
+    for i in range(wc.depth):
+        p = f"pred.blk.{i}."
+        s += [(p + "adaln.weight", (6 * D, D), "w32_ada"), (p + "adaln.bias", (6 * D,), "b32_ada"),
+              (p + "attn_qkv.weight", (3 * D, D), "w_in"), (p + "attn_qkv.bias", (3 * D,), "b"),
+              (p + "attn_out.weight", (D, D), "w_in"), (p + "attn_out.bias", (D,), "b"),
+              (p + "ffn_up.weight", (M, D), "w_in"), (p + "ffn_up.bias", (M,), "b"),
+              (p + "ffn_down.weight", (D, M), "w_hid"), (p + "ffn_down.bias", (D,), "b")]
+    s += [("pred.norm.weight", (D,), "ln_g"), ("pred.norm.bias", (D,), "ln_b"),
+          ("pred.proj.0.weight", (wc.pred_hidden, D), "w_in"), ("pred.proj.0.bias", (wc.pred_hidden,), "b"),
+          ("pred.proj.2.weight", (D, wc.pred_hidden), "w_hid"), ("pred.proj.2.bias", (D,), "b")]
+    return s
+
+
+def make_world_model_table(wc: WorldModelConfig) -> List["Tensor"]:
+    """Seeded world-model tensors.  Scales are chosen so that every part of
+    the computation moves the result: matrices ~ N(0, 0.7 / sqrt(fan_in))
+    (0.3 / sqrt(fan_in) for the adaLN, whose shifts, scales and gates then
+    have a spread of about 0.3), biases ~ N(0, 0.02), the action embedder
+    ~ N(0, 1 / sqrt(fan_in)), pos_embed ~ N(0, 0.5), LayerNorm gamma ~
+    1 + N(0, 0.1), beta ~ N(0, 0.02).  f32 for adaLN and the action embedder,
+    the model's weight type for the re-typed matrices."""
+    rng = np.random.default_rng(wc.seed)
+    table = []
+    for name, shape, kind in world_model_specs(wc):
+        z = rng.standard_normal(shape, dtype=np.float32)
+        fan_in = shape[-1]
+        scale = {"w": 0.7 / np.sqrt(fan_in), "w_in": 0.7 / np.sqrt(fan_in), "w_hid": 0.7 / np.sqrt(fan_in),
+                 "w32_ada": 0.3 / np.sqrt(fan_in), "w32_act0": 1.0 / np.sqrt(fan_in),
+                 "w32_act2": 1.0 / np.sqrt(fan_in), "b": 0.02, "b32": 0.02, "b32_ada": 0.02, "pos": 0.5,
+                 "ln_b": 0.02}.get(kind)
+        if kind == "ln_g":
+            v = np.float32(1.0) + np.float32(0.1) * z
+        else:
+            v = np.float32(scale) * z
+        table.append(_store(name, shape, v, "f32" if kind.startswith(("w32", "b32")) else wc.weights))
+    return table
+
+
+def make_world_model_inputs(wc: WorldModelConfig, candidates: Optional[int] = None):
+    """Seeded inputs: observed states [C, frames, D] ~ N(0, 1) (projector
+    outputs stand-in) and actions [C, n_actions, A] ~ U(-1, 1)."""
+    C = wc.candidates if candidates is None else candidates
+    rng = np.random.default_rng(wc.seed + 3000)
+    states = rng.standard_normal((C, wc.frames, wc.dim), dtype=np.float32)
+    actions = rng.uniform(-1.0, 1.0, (C, wc.n_actions, wc.action_dim)).astype(np.float32)
+    return states, actions
+
+
+# LeWM world model workloads of the benchmarks page ("LeWM world model"):
+# one predictor call over the full 3-frame window, and a 20-step rollout from
+# one observed frame (the window grows to 3, then slides); plus a planner-sized
+# batch of candidate action sequences (the axis the V-JEPA 2-AC planner rows
+# of the same page scale on).
+LEWM_WM_STEP = WorldModelConfig(name="lewm_wm_step_3f", enc=LEWM_VIT_TI, frames=3, steps=0, candidates=1)
+LEWM_WM_ROLLOUT = WorldModelConfig(name="lewm_wm_rollout_20", enc=LEWM_VIT_TI, frames=1, steps=20, candidates=1)
+LEWM_WM_PLAN = WorldModelConfig(name="lewm_wm_rollout_20_c1024", enc=LEWM_VIT_TI, frames=1, steps=20,
+                                candidates=1024)
+WORLD_MODELS: Dict[str, "WorldModelConfig"] = {w.name: w for w in (LEWM_WM_STEP, LEWM_WM_ROLLOUT, LEWM_WM_PLAN)}
+
+
 def small_config(base: EncoderConfig, **kw) -> EncoderConfig:
     """A shrunk copy of a workload that the oracle runs in seconds."""
     d = dict(dim=256, depth=2, heads=4, mlp=1024, img_h=64, img_w=64,
@@ -286,7 +396,8 @@ _RETYPED_SUFFIXES = ("attn_qkv.weight", "attn_out.weight", "ffn_up.weight",
                      "ffn_down.weight", "head.xattn.q.weight",
                      "head.xattn.k.weight", "head.xattn.v.weight",
                      "head.xattn.out.weight", "head.cls.weight",
-                     "pred.embed.weight", "pred.proj.weight")
+                     "pred.embed.weight", "pred.proj.weight", "enc.proj.0.weight",
+                     "enc.proj.2.weight", "pred.proj.0.weight", "pred.proj.2.weight")
 
 
 def is_retyped(name: str) -> bool:

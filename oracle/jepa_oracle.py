@@ -23,10 +23,13 @@ matmul as the only primitive), in the order the pages describe the model:
   across frames, CLS a read-only sink ("LeVJEPA" card, intro);
 * the final ``norm`` before last_hidden_state ("Quantization" page, "Reading
   the numbers");
-* pooling mean / cls / none ("LeVJEPA" card, "Run it": --pool) and the
+* pooling mean / cls / none / lewm ("LeVJEPA" card, "Run it": --pool) and the
   attentive-pool classifier: 3 self-attention blocks over the tokens, one
   cross-attention query, MLP, linear ("jepa.cpp — measured benchmarks",
   "Attentive-pool head");
+* the LeWM world model: the projector of the CLS row and the AdaLN-zero
+  causal predictor with its rollout ("LeWorldModel Push-T" card, intro;
+  readings in its section below);
 * q8_0 / q4_0 dequantisation: value = q*d and (q-8)*d per 32-element block
   with one fp16 scale (ggml's published block formats; the "Quantization"
   page, "File sizes", gives their 8.5 / 4.5 bits per weight).
@@ -396,6 +399,8 @@ def forward(cfg, W, pixels, pool_mode: Optional[str] = None) -> np.ndarray:
     y = encoder(cfg, W, pixels)
     if mode == "attentive":
         return attentive_head(cfg, W, y)
+    if mode == "lewm":
+        return lewm_project(W, pool(cfg, y, "cls"))
     return pool(cfg, y, mode)
 
 
@@ -426,6 +431,109 @@ def predictor(pc, W, tokens: np.ndarray, ctx_idx: Sequence[int], tgt_idx: Sequen
         x = block(x, W, f"pred.blk.{i}.", pc.heads, pc.ln_eps, None)
     y = layer_norm(x[:, len(ctx_idx):], W["pred.norm.weight"], W["pred.norm.bias"], pc.ln_eps)
     return linear(y, W["pred.proj.weight"], W["pred.proj.bias"])
+
+
+# ---------------------------------------------------------------------------
+# LeWM world model ("LeWorldModel Push-T" card, intro: the encoder's CLS token
+# is projected to a world-model state, and six AdaLN-zero causal blocks
+# conditioned on a 10-d action roll that state forward; "Measured": the
+# projector and predictor MLPs are BatchNorm-folded; "Quantization" page,
+# "The rule": enc.proj.* (the projector) and pred.proj.0 / pred.proj.2 are
+# re-typed matrices, pred.blk.*.adaln.* and pred.action_embed.* stay f32;
+# benchmarks page, "LeWM world model": one predictor call covers a window of
+# 3 frames of 192-d states, a rollout grows that window one predicted state
+# per step).  Readings where the pages are silent:
+#   * projector: emb = W2 GELU(W1 cls + b1) + b2 on the final-normed CLS row
+#     (BatchNorm folded into W1, b1);
+#   * action embedding: c_t = W2 SiLU(W1 a_t + b1) + b2 (pred.action_embed.0
+#     / .2), one per frame;
+#   * AdaLN-zero block (the diffusion-transformer form): [shift1, scale1,
+#     gate1, shift2, scale2, gate2] = adaln(SiLU(c_t)) split in six; LayerNorms
+#     without affine parameters; x += gate1 * attn_out(attention(LN(x) (1 +
+#     scale1) + shift1)); x += gate2 * MLP(LN(x) (1 + scale2) + shift2); the
+#     attention causal over the frames (frame t reads frames <= t), the MLP
+#     ffn_up -> GELU -> ffn_down as in the encoder;
+#   * the input states plus the predictor's positional rows pred.pos_embed
+#     [window, D] (row t for the t-th frame of the window);
+#   * output: pred.proj.2 GELU(pred.proj.0 pred.norm(x)): row t predicts the
+#     state of frame t + 1;
+#   * rollout: the window holds the last `window` states; each step appends
+#     the prediction of its last row; the action of a state is the one taken
+#     in that frame.
+# ---------------------------------------------------------------------------
+def silu(x: np.ndarray) -> np.ndarray:
+    """x * sigmoid(x)."""
+    x = np.asarray(x, np.float64)
+    return x / (1.0 + np.exp(-x))
+
+
+def lewm_project(W, cls: np.ndarray) -> np.ndarray:
+    """The LeWM projector (enc.proj.0 / enc.proj.2) on final-normed CLS rows
+    [B, D] -> world-model states [B, D_s]."""
+    h = gelu(linear(cls, W["enc.proj.0.weight"], W["enc.proj.0.bias"]))
+    return linear(h, W["enc.proj.2.weight"], W["enc.proj.2.bias"])
+
+
+def lewm_action_embed(W, act: np.ndarray) -> np.ndarray:
+    """Actions [.., A] -> conditioning vectors [.., D] (pred.action_embed)."""
+    h = silu(linear(act, W["pred.action_embed.0.weight"], W["pred.action_embed.0.bias"]))
+    return linear(h, W["pred.action_embed.2.weight"], W["pred.action_embed.2.bias"])
+
+
+def causal_allow(T: int) -> np.ndarray:
+    """Boolean [T, T]: frame i reads frames j <= i."""
+    return np.tril(np.ones((T, T), bool))
+
+
+def adaln_block(x, c, W, prefix: str, heads: int, eps: float) -> np.ndarray:
+    """One AdaLN-zero block over x [B, T, D] conditioned on c [B, T, D]."""
+    D = x.shape[-1]
+    mod = linear(silu(c), W[prefix + "adaln.weight"], W[prefix + "adaln.bias"])
+    shift1, scale1, gate1, shift2, scale2, gate2 = (mod[..., i * D:(i + 1) * D] for i in range(6))
+    one, zero = np.ones(D), np.zeros(D)
+    h = layer_norm(x, one, zero, eps) * (1.0 + scale1) + shift1
+    qkv = linear(h, W[prefix + "attn_qkv.weight"], W[prefix + "attn_qkv.bias"])
+    q, k, v = (split_heads(qkv[..., i * D:(i + 1) * D], heads) for i in range(3))
+    o = merge_heads(attention(q, k, v, causal_allow(x.shape[1])))
+    x = x + gate1 * linear(o, W[prefix + "attn_out.weight"], W[prefix + "attn_out.bias"])
+    h = layer_norm(x, one, zero, eps) * (1.0 + scale2) + shift2
+    u = gelu(linear(h, W[prefix + "ffn_up.weight"], W[prefix + "ffn_up.bias"]))
+    return x + gate2 * linear(u, W[prefix + "ffn_down.weight"], W[prefix + "ffn_down.bias"])
+
+
+def lewm_predict(wc, W, states: np.ndarray, actions: np.ndarray) -> np.ndarray:
+    """One predictor call: states [B, T, D], actions [B, T, A] (T <= the
+    window) -> predictions [B, T, D], row t the predicted state of frame
+    t + 1."""
+    states = np.asarray(states, np.float64)
+    T = states.shape[1]
+    if T > wc.window:
+        raise ValueError("window")
+    x = states + W["pred.pos_embed"][:T][None]
+    c = lewm_action_embed(W, actions)
+    for i in range(wc.depth):
+        x = adaln_block(x, c, W, f"pred.blk.{i}.", wc.heads, wc.ln_eps)
+    y = layer_norm(x, W["pred.norm.weight"], W["pred.norm.bias"], wc.ln_eps)
+    h = gelu(linear(y, W["pred.proj.0.weight"], W["pred.proj.0.bias"]))
+    return linear(h, W["pred.proj.2.weight"], W["pred.proj.2.bias"])
+
+
+def lewm_rollout(wc, W, states0: np.ndarray, actions: np.ndarray, steps: int) -> np.ndarray:
+    """Rollout: states0 [B, T0, D] (the observed frames), actions
+    [B, T0 + steps - 1, A] (action t belongs to frame t) -> the predicted
+    states of frames T0 .. T0 + steps - 1, [B, steps, D].  Each step runs the
+    predictor on the last min(window, frames so far) frames and appends the
+    prediction of the last one."""
+    seq = [np.asarray(states0[:, t], np.float64) for t in range(states0.shape[1])]
+    out = []
+    for _ in range(steps):
+        n = len(seq)
+        lo = max(0, n - wc.window)
+        win = np.stack(seq[lo:n], axis=1)
+        nxt = lewm_predict(wc, W, win, actions[:, lo:n])[:, -1]
+        seq.append(nxt)
+        out.append(nxt)
+    return np.stack(out, axis=1)
 
 
 # ---------------------------------------------------------------------------
