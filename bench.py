@@ -578,13 +578,130 @@ def run_predictor(args, pc, rank, world, local_rank):
     return 0
 
 
+def _wm_flops_per_call(wc, T: int) -> float:
+    """Algorithmic FLOPs of one LeWM predictor call over T frames of one
+    candidate (matrix products, the causal attention's T (T + 1) / 2 pairs)."""
+    D, M, H = wc.dim, wc.mlp, wc.pred_hidden
+    per_row_block = 2.0 * (6 * D * D + 3 * D * D + D * D + 2 * D * M)
+    attn = 4.0 * D * T * (T + 1) / 2 * wc.depth
+    return T * (wc.depth * per_row_block + 2.0 * D * D + 2.0 * wc.action_dim * D + 4.0 * D * H) + attn
+
+
+def _wm_tile_bytes(wc) -> int:
+    """Weight bytes one CTA streams per predictor call: every 128-row x
+    64-column f16 tile the fused kernel loads (adaLN chunks start on tile
+    boundaries, so a 192-wide chunk takes two tiles)."""
+    D, M, H = wc.dim, wc.mlp, wc.pred_hidden
+    tc = -(-D // 128)
+    kd = D // 64
+    t = tc * kd + wc.depth * (6 * tc * kd + -(-3 * D // 128) * kd + tc * kd + -(-M // 128) * kd + tc * (M // 64))
+    t += -(-H // 128) * kd + tc * (H // 64)
+    return t * 16384
+
+
+def run_world_model(args, wc, rank, world, local_rank):
+    """The LeWM world model alone on seeded states and actions resident in
+    HBM: one step = one jepa_b200_lewm_predict (wc.steps == 0) or one whole
+    jepa_b200_lewm_rollout of every candidate, each a single kernel launch;
+    the rate counts predictor calls (one pass over a candidate's window)."""
+    import torch
+    import jepa_video_encoder_b200 as jb
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    table = synth.make_tensor_table(wc.enc) + synth.make_world_model_table(wc)
+    model = jb.Model(wc.enc, table, device=local_rank, world_model=wc)
+    st_np, ac_np = synth.make_world_model_inputs(wc)
+    st, ac = torch.from_numpy(st_np).to(dev), torch.from_numpy(ac_np).to(dev)
+    C = wc.candidates
+    calls = C * (wc.steps if wc.steps > 0 else 1)
+    out = torch.empty((C, wc.steps if wc.steps > 0 else wc.frames, wc.dim), dtype=torch.float32, device=dev)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        if wc.steps > 0:
+            model.lewm_rollout(st, ac, wc.steps, out=out, stream=stream)
+        else:
+            model.lewm_predict(st, ac, out=out, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if model.sync_status(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    clock_path = os.path.join(tempfile.gettempdir(), f"jepa_clocks_rank{rank}.csv")
+    proc, fh = _clock_sampler_start(clock_path)
+    time.sleep(0.3)
+    launches = 0
+    t0 = time.time()
+    for k in range(args.steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        step()
+        ev[k][1].record(stream)
+        launches += model.last_launch_count()
+    torch.cuda.synchronize(dev)
+    clocks = _clock_sampler_stop(proc, fh, clock_path, local_rank, t0, time.time())
+    if model.sync_status(stream) != 0:
+        raise RuntimeError("device error in the timed region")
+    ms_steps = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(sum(ms_steps), world, dev)
+    value = whole_job_rate(calls, world, args.steps, total_ms)
+    if rank != 0:
+        model.close()
+        return 0
+    ms_per_step = total_ms / args.steps
+    # FLOPs: the window grows from `frames` (capped at the window) during a rollout
+    if wc.steps > 0:
+        fl = sum(_wm_flops_per_call(wc, min(wc.window, wc.frames + s)) for s in range(wc.steps)) * C
+    else:
+        fl = _wm_flops_per_call(wc, wc.frames) * C
+    cpc = 32 // (min(wc.window, wc.frames + wc.steps - 1) if wc.steps > 0 else wc.frames)
+    ctas = -(-C // cpc)
+    tile_bytes = _wm_tile_bytes(wc) * (wc.steps if wc.steps > 0 else 1)
+    peaks, peak_src = _peaks()
+    cpu = None
+    if not args.no_cpu:
+        from oracle import jepa_oracle as orc
+        W = orc.weights_f64([t for t in table if t.name.startswith(("pred.", "enc.proj."))])
+        tc = time.perf_counter()
+        if wc.steps > 0:
+            orc.lewm_rollout(wc, W, st_np[:1], ac_np[:1], wc.steps)
+            n_calls = wc.steps
+        else:
+            orc.lewm_predict(wc, W, st_np[:1], ac_np[:1])
+            n_calls = 1
+        t_c = time.perf_counter() - tc
+        cpu = {"value": n_calls / t_c, "unit": "predictor calls/s", "cores": _oracle_threads(), "kind": "oracle",
+               "sample": f"1 candidate, {n_calls} call(s), float64 numpy, timed whole ({t_c * 1e3:.1f} ms)"}
+    line = {"metric": "LeWM world-model predictor calls/s on 1 B200", "value": value, "unit": "predictor calls/s",
+            "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
+            "ms_per_step_min": min(ms_steps), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16", "data": "synthetic",
+            "config": {"workload": wc.name, "candidates": C, "frames": wc.frames, "rollout_steps": wc.steps,
+                       "window": wc.window, "dim": wc.dim, "depth": wc.depth, "weights": wc.weights,
+                       "ctas": ctas, "l2": "flushed between steps (256 MiB write)"},
+            "us_per_call_per_candidate_group": ms_per_step * 1e3 / (wc.steps if wc.steps > 0 else 1),
+            "tflops": fl / (ms_per_step / 1000.0) / 1e12,
+            "weight_stream": {"bytes_per_cta": tile_bytes, "gbs_per_cta": tile_bytes / (ms_per_step / 1000.0) / 1e9},
+            "cpu_baseline": cpu, "gpu_launches": launches, "clocks": clocks,
+            "when": datetime.datetime.now(datetime.timezone.utc).strftime("%Y-%m-%dT%H:%M:%S.%fZ")}
+    del peaks, peak_src
+    print(json.dumps(line), flush=True)
+    model.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS) + sorted(synth.PREDICTORS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(synth.WORKLOADS) + sorted(synth.PREDICTORS) + sorted(synth.WORLD_MODELS))
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
     ap.add_argument("--clock-log", default=None,
                     help="CSV of the nvidia-smi clock samples taken during the timed region ({rank} is replaced)")
@@ -601,6 +718,11 @@ def main():
             print(json.dumps({"impl": args.impl, "unavailable": "the predictor workload runs on one GPU, ours only"}))
             return 0
         return run_predictor(args, synth.PREDICTORS[args.workload], rank, world, local_rank)
+    if args.workload in synth.WORLD_MODELS:
+        if args.impl == "reference" or world > 1:
+            print(json.dumps({"impl": args.impl, "unavailable": "the world-model workload runs on one GPU, ours only"}))
+            return 0
+        return run_world_model(args, synth.WORLD_MODELS[args.workload], rank, world, local_rank)
     cfg = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, cfg, rank, world)

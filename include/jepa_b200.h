@@ -71,7 +71,9 @@ typedef enum {
   JEPA_B200_POOL_NONE = 0,     /* full token map, f32 [B, N, D] */
   JEPA_B200_POOL_MEAN = 1,     /* mean over the patch tokens (CLS excluded), f32 [B, D] */
   JEPA_B200_POOL_CLS = 2,      /* the CLS row, f32 [B, D] */
-  JEPA_B200_POOL_ATTENTIVE = 3 /* attentive-pool classifier logits, f32 [B, n_classes] */
+  JEPA_B200_POOL_ATTENTIVE = 3, /* attentive-pool classifier logits, f32 [B, n_classes] */
+  JEPA_B200_POOL_LEWM = 4       /* the LeWM projector on the final-normed CLS row: world-model states,
+                                   f32 [B, D] (a model loaded with wm_depth > 0) */
 } jepa_b200_pool;
 
 typedef enum {
@@ -111,6 +113,16 @@ typedef struct {
                        * the attention output, the MLP's hidden values, the weights' 16-bit form)
                        * is bf16 instead of f16; the residual stream, LayerNorm statistics,
                        * softmax and every accumulation stay f32. */
+  /* LeWM world model (wm_depth 0: none), run by jepa_b200_lewm_predict / _rollout and
+   * POOL_LEWM ("LeWorldModel Push-T" card, intro: the CLS row projected to a state,
+   * six AdaLN-zero causal blocks conditioned on a 10-d action; benchmarks page, "LeWM
+   * world model": a 3-frame window of 192-d states).  The state width is dim (at most
+   * 256, heads of 64: dim = 64 * wm_heads); wm_mlp and wm_pred_hidden (the hidden width
+   * of pred.proj) at most 1024, multiples of 64; wm_proj_hidden (enc.proj's hidden
+   * width) a multiple of 64; wm_action_dim at most 64; wm_window (frames a predictor
+   * call reads, the rows of pred.pos_embed) at most 32.  Needs has_cls; excludes
+   * pred_depth > 0 (both name their tensors pred.*). */
+  int wm_depth, wm_heads, wm_mlp, wm_action_dim, wm_window, wm_proj_hidden, wm_pred_hidden;
 } jepa_b200_config;
 
 /* One entry of the tensor table.  Host memory, owned by the caller; it is
@@ -138,7 +150,14 @@ typedef struct jepa_b200_model jepa_b200_model;
  * with a predictor pred.embed.{weight [Dp, D], bias}, pred.mask_tokens
  * [1, Dp], pred.pos_embed [N, Dp], pred.blk.<i>.* (the encoder block's
  * tensors at width Dp = pred_dim), pred.norm.*, pred.proj.{weight [D, Dp],
- * bias [D]}.
+ * bias [D]}; with a world model enc.proj.{0,2}.{weight [Hp, D] / [D, Hp], bias},
+ * pred.action_embed.{0,2}.{weight [D, A] / [D, D], bias [D]}, pred.pos_embed
+ * [wm_window, D], pred.blk.<i>.{adaln.weight [6D, D], adaln.bias [6D], attn_qkv,
+ * attn_out, ffn_up, ffn_down}.{weight,bias} (no LayerNorm tensors: the blocks'
+ * LayerNorms have no affine parameters), pred.norm.*, pred.proj.{0,2}.{weight
+ * [Hq, D] / [D, Hq], bias}.  The world model's matrices are unpacked once to
+ * 16-bit arenas that its kernel streams (q8_0 / q4_0 sources keep their blocks
+ * as well); pred.action_embed.0.weight stays f32.
  * q8_0 / q4_0 are accepted only for the matrices that page re-types and only
  * when the input dimension is a multiple of 64.  f32 matrices are rounded to
  * f16 once here; 1-D tensors and pos_embed are kept in f32.  A q8_0 / q4_0
@@ -186,6 +205,34 @@ JEPA_B200_API int jepa_b200_encode(jepa_b200_model *m, const float *pixels, int 
  * B * (n_ctx + n_tgt) above 524288 rows), ERR_CUDA. */
 JEPA_B200_API int jepa_b200_predict(jepa_b200_model *m, const float *tokens, int B, const int *ctx_idx, int n_ctx,
                                     const int *tgt_idx, int n_tgt, float *out, size_t out_bytes, void *stream);
+
+/* The LeWM predictor ("LeWorldModel Push-T" card, intro; benchmarks page,
+ * "LeWM world model"), one predictor call over T <= wm_window frames of C
+ * independent candidates.  For frame t: x = state + pred.pos_embed[t];
+ * c = action_embed.2(SiLU(action_embed.0(action))); six AdaLN-zero blocks
+ * ([shift1 scale1 gate1 shift2 scale2 gate2] = adaln(SiLU(c)); x += gate1 *
+ * attn_out(attention(LN(x)(1 + scale1) + shift1)) with frame t reading frames
+ * <= t; x += gate2 * ffn_down(GELU(ffn_up(LN(x)(1 + scale2) + shift2)))),
+ * then pred.proj.2(GELU(pred.proj.0(pred.norm(x)))): row t is the predicted
+ * state of frame t + 1.  Row t depends on frames <= t only, bit for bit.
+ * states:  device, f32 [C, T, D];  actions: device, f32 [C, T, wm_action_dim];
+ * out:     device, f32 [C, T, D]; out_bytes its size.
+ * One kernel launch on `stream`.  Errors: ERR_ARG (null, C or T
+ * < 1, no world model), ERR_SHAPE (T > wm_window, out_bytes too small),
+ * ERR_CUDA. */
+JEPA_B200_API int jepa_b200_lewm_predict(jepa_b200_model *m, const float *states, const float *actions, int C, int T,
+                                         float *out, size_t out_bytes, void *stream);
+
+/* Rollout of the LeWM predictor: from T0 observed states per candidate, `steps`
+ * predictor calls, each over the last min(wm_window, frames so far) frames,
+ * each appending the prediction of its last row as the next frame.
+ * states:  device, f32 [C, T0, D];
+ * actions: device, f32 [C, T0 + steps - 1, wm_action_dim] (action f of frame f);
+ * out:     device, f32 [C, steps, D]: the states of frames T0 .. T0 + steps - 1.
+ * The whole rollout is one kernel launch on `stream`.  Errors: ERR_ARG (null,
+ * C, T0 or steps < 1, no world model), ERR_SHAPE (out_bytes too small), ERR_CUDA. */
+JEPA_B200_API int jepa_b200_lewm_rollout(jepa_b200_model *m, const float *states, int T0, const float *actions, int C,
+                                         int steps, float *out, size_t out_bytes, void *stream);
 
 /* End-to-end variant with HOST buffers: copies pixels (host, f32 [B, frames,
  * 3, H, W]; pinned memory makes the copy asynchronous) to model-owned device

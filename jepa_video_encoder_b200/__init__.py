@@ -67,8 +67,9 @@ def check_out(out, on_cuda: bool, device: Optional[int] = None) -> None:
 
 
 def make_config(cfg: "synth.EncoderConfig", quant_f16_copy: bool = False,
-                predictor: Optional["synth.PredictorConfig"] = None) -> _abi.Config:
-    pr = predictor
+                predictor: Optional["synth.PredictorConfig"] = None,
+                world_model: Optional["synth.WorldModelConfig"] = None) -> _abi.Config:
+    pr, wm = predictor, world_model
     return _abi.Config(dim=cfg.dim, depth=cfg.depth, heads=cfg.heads, mlp=cfg.mlp, patch=cfg.patch,
                        tubelet=cfg.tubelet, img_h=cfg.img_h, img_w=cfg.img_w, frames=cfg.frames,
                        has_cls=1 if cfg.has_cls else 0, mask=synth.MASK_IDS[cfg.mask],
@@ -76,17 +77,23 @@ def make_config(cfg: "synth.EncoderConfig", quant_f16_copy: bool = False,
                        rope=1 if cfg.rope else 0, quant_f16_copy=1 if quant_f16_copy else 0,
                        pred_depth=pr.depth if pr else 0, pred_dim=pr.dim if pr else 0,
                        pred_heads=pr.heads if pr else 0, pred_mlp=pr.mlp if pr else 0,
-                       act_bf16=1 if cfg.act_bf16 else 0)
+                       act_bf16=1 if cfg.act_bf16 else 0,
+                       wm_depth=wm.depth if wm else 0, wm_heads=wm.heads if wm else 0, wm_mlp=wm.mlp if wm else 0,
+                       wm_action_dim=wm.action_dim if wm else 0, wm_window=wm.window if wm else 0,
+                       wm_proj_hidden=wm.proj_hidden if wm else 0, wm_pred_hidden=wm.pred_hidden if wm else 0)
 
 
 class Model:
     """A loaded encoder on one CUDA device.  quant_f16_copy: also keep an f16
     copy of the q8_0 / q4_0 matrices for the large GEMMs (default: blocks
     only, unpacked in every GEMM's loader).  predictor: the shape of a masked
-    predictor whose pred.* tensors are in the table (see predict)."""
+    predictor whose pred.* tensors are in the table (see predict);
+    world_model: the shape of a LeWM world model whose tensors are in the
+    table (see lewm_predict, lewm_rollout and the "lewm" pool)."""
 
     def __init__(self, cfg: "synth.EncoderConfig", table: List["synth.Tensor"], device: int = 0,
-                 quant_f16_copy: bool = False, predictor: Optional["synth.PredictorConfig"] = None):
+                 quant_f16_copy: bool = False, predictor: Optional["synth.PredictorConfig"] = None,
+                 world_model: Optional["synth.WorldModelConfig"] = None):
         lib = load_library()
         self.cfg = cfg
         self.device = device
@@ -103,7 +110,7 @@ class Model:
                 e.shape[j] = s
             e.data = t.data.ctypes.data
             e.nbytes = t.nbytes
-        self._cfg = make_config(cfg, quant_f16_copy, predictor)
+        self._cfg = make_config(cfg, quant_f16_copy, predictor, world_model)
         h = ctypes.c_void_p()
         check(lib.jepa_b200_load_weights(ctypes.byref(self._cfg), entries, len(table), device, ctypes.byref(h)),
               "load_weights")
@@ -181,6 +188,44 @@ class Model:
         check(load_library().jepa_b200_predict(self._h, tokens.data_ptr(), B, ci.ctypes.data, len(ci), ti.ctypes.data,
                                                len(ti), out.data_ptr(), out.numel() * 4, _stream_ptr(stream)),
               "predict")
+        return out
+
+    def _wm_in(self, t, name, ndim):
+        import torch
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous() \
+                or t.dim() != ndim or t.device.index != self.device:
+            raise ValueError(f"{name} must be a contiguous float32 tensor of {ndim} dims on cuda:{self.device}")
+
+    def lewm_predict(self, states, actions, out=None, stream=None):
+        """LeWM predictor call: states CUDA float32 [C, T, dim], actions
+        [C, T, action_dim] -> float32 [C, T, dim], row t the predicted state
+        of frame t + 1.  Asynchronous."""
+        import torch
+        self._wm_in(states, "states", 3)
+        self._wm_in(actions, "actions", 3)
+        C, T = int(states.shape[0]), int(states.shape[1])
+        if out is None:
+            out = torch.empty((C, T, int(states.shape[2])), dtype=torch.float32, device=states.device)
+        check_out(out, True, self.device)
+        check(load_library().jepa_b200_lewm_predict(self._h, states.data_ptr(), actions.data_ptr(), C, T,
+                                                    out.data_ptr(), out.numel() * 4, _stream_ptr(stream)),
+              "lewm_predict")
+        return out
+
+    def lewm_rollout(self, states, actions, steps: int, out=None, stream=None):
+        """LeWM rollout: states CUDA float32 [C, T0, dim] (observed frames),
+        actions [C, T0 + steps - 1, action_dim] -> float32 [C, steps, dim],
+        the predicted states of frames T0 .. T0 + steps - 1.  Asynchronous."""
+        import torch
+        self._wm_in(states, "states", 3)
+        self._wm_in(actions, "actions", 3)
+        C, T0 = int(states.shape[0]), int(states.shape[1])
+        if out is None:
+            out = torch.empty((C, steps, int(states.shape[2])), dtype=torch.float32, device=states.device)
+        check_out(out, True, self.device)
+        check(load_library().jepa_b200_lewm_rollout(self._h, states.data_ptr(), T0, actions.data_ptr(), C, steps,
+                                                    out.data_ptr(), out.numel() * 4, _stream_ptr(stream)),
+              "lewm_rollout")
         return out
 
     def encode_host(self, pixels, pool: Optional[str] = None, out=None, stream=None):

@@ -21,7 +21,9 @@ class Config(ctypes.Structure):
                 ("frames", c_int), ("has_cls", c_int), ("mask", c_int),
                 ("head_sa_blocks", c_int), ("n_classes", c_int), ("ln_eps", c_float), ("rope", c_int),
                 ("quant_f16_copy", c_int), ("pred_depth", c_int), ("pred_dim", c_int), ("pred_heads", c_int),
-                ("pred_mlp", c_int), ("act_bf16", c_int)]
+                ("pred_mlp", c_int), ("act_bf16", c_int), ("wm_depth", c_int), ("wm_heads", c_int),
+                ("wm_mlp", c_int), ("wm_action_dim", c_int), ("wm_window", c_int), ("wm_proj_hidden", c_int),
+                ("wm_pred_hidden", c_int)]
 
 
 class TensorEntry(ctypes.Structure):
@@ -36,6 +38,9 @@ SIGNATURES = {
     "jepa_b200_encode_host": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_size_t, c_void_p]),
     "jepa_b200_predict": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_int, c_void_p, c_int, c_void_p, c_size_t,
                                   c_void_p]),
+    "jepa_b200_lewm_predict": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_size_t, c_void_p]),
+    "jepa_b200_lewm_rollout": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_int, c_int, c_void_p, c_size_t,
+                                       c_void_p]),
     "jepa_b200_out_shape": (c_int, [c_void_p, c_int, c_int, POINTER(c_int64)]),
     "jepa_b200_debug_stage": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_size_t, c_void_p]),
     "jepa_b200_sync_status": (c_int, [c_void_p, c_void_p]),

@@ -20,6 +20,7 @@
 #include <vector>
 
 #include "internal.h"
+#include "world_model.h"
 
 using namespace jb;
 
@@ -80,6 +81,14 @@ struct jepa_b200_model {
   float *b_pembed = nullptr, *pmask = nullptr, *ppos = nullptr, *pnorm_g = nullptr, *pnorm_b = nullptr,
         *b_pproj = nullptr;
   std::vector<LayerW> pred;
+  // LeWM world model (cfg.wm_depth > 0): the projector for POOL_LEWM and the
+  // fused predictor's weight arenas and f32 vectors
+  DevMatrix wproj0, wproj2;
+  float *b_wproj0 = nullptr, *b_wproj2 = nullptr;
+  WmArena wm;
+  float *wm_w_act0 = nullptr, *wm_b_act0 = nullptr, *wm_b_act2 = nullptr, *wm_pos = nullptr;
+  float *wm_b_ada = nullptr, *wm_b_qkv = nullptr, *wm_b_out = nullptr, *wm_b_up = nullptr, *wm_b_down = nullptr;
+  float *wm_norm_g = nullptr, *wm_norm_b = nullptr, *wm_b_p0 = nullptr, *wm_b_p2 = nullptr;
   std::vector<void*> allocs;
   size_t weight_bytes = 0;
 
@@ -90,6 +99,7 @@ struct jepa_b200_model {
   __half *Y = nullptr, *Q = nullptr, *Kb = nullptr, *Vt = nullptr, *O = nullptr, *H = nullptr;
   float *Yf = nullptr, *partial = nullptr;
   float *hq = nullptr, *hattn = nullptr, *hz = nullptr, *hzn = nullptr, *hu = nullptr;
+  float* hp = nullptr;  // the LeWM projector's hidden rows [B, wm_proj_hidden]
   std::vector<void*> ws_allocs;
   std::vector<BlockOps> enc_ops, head_ops;
   GemmOp pe_op, kv_op;
@@ -149,7 +159,8 @@ bool is_retyped(const std::string& n) {
   static const char* suffixes[] = {"attn_qkv.weight",     "attn_out.weight",     "ffn_up.weight",
                                    "ffn_down.weight",     "head.xattn.q.weight", "head.xattn.k.weight",
                                    "head.xattn.v.weight", "head.xattn.out.weight", "head.cls.weight",
-                                   "pred.embed.weight",   "pred.proj.weight"};
+                                   "pred.embed.weight",   "pred.proj.weight",    "enc.proj.0.weight",
+                                   "enc.proj.2.weight",   "pred.proj.0.weight",  "pred.proj.2.weight"};
   for (const char* s : suffixes) {
     const size_t L = strlen(s);
     if (n.size() >= L && n.compare(n.size() - L, L, s) == 0) return true;
@@ -369,6 +380,47 @@ struct Loader {
     }
     return M;
   }
+  // One matrix [N, K] into rows row0 .. row0 + N - 1 of a 16-bit arena of
+  // row length K: f32 / f16 values rounded once to f16 (bf16 in a bf16
+  // model); q8_0 / q4_0 blocks uploaded and unpacked on the device to the
+  // same values the GEMM loaders produce.
+  void arena_put(void* arena, int64_t row0, const std::string& name, int64_t N, int64_t K) {
+    const jepa_b200_tensor* t = get(name, {N, K});
+    if (!t || dry || status != JEPA_B200_OK) return;
+    uint8_t* dst = static_cast<uint8_t*>(arena) + static_cast<size_t>(row0 * K) * 2;
+    const bool bf = m->cfg.act_bf16 != 0;
+    if (t->dtype == JEPA_B200_F32 || t->dtype == JEPA_B200_F16) {
+      std::vector<float> v = host_floats(t);
+      std::vector<uint16_t> h(v.size());
+      for (size_t i = 0; i < v.size(); ++i)
+        h[i] = bf ? __bfloat16_as_ushort(__float2bfloat16_rn(v[i])) : __half_as_ushort(__float2half_rn(v[i]));
+      upload(dst, h.data(), h.size() * 2);
+      return;
+    }
+    DevMatrix Q = matrix({t}, K, K);
+    if (status == JEPA_B200_OK &&
+        launch_dequant_f16(Q.bmode, Q.data, Q.scales, static_cast<int>(N), static_cast<int>(K),
+                           reinterpret_cast<__half*>(dst), nullptr, bf) != JEPA_B200_OK)
+      status = JEPA_B200_ERR_CUDA;
+  }
+  // The per-block f32 vectors prefix<i>.suffix [len] of blocks 0..n-1, stacked.
+  float* vec_stack(const std::string& prefix, const std::string& suffix, int n, int64_t len) {
+    std::vector<float> all;
+    for (int i = 0; i < n && status == JEPA_B200_OK; ++i) {
+      const jepa_b200_tensor* t = get(prefix + std::to_string(i) + "." + suffix, {len});
+      if (!t) return nullptr;
+      if (t->dtype != JEPA_B200_F32 && t->dtype != JEPA_B200_F16) {
+        status = JEPA_B200_ERR_DTYPE;
+        return nullptr;
+      }
+      std::vector<float> v = host_floats(t);
+      all.insert(all.end(), v.begin(), v.end());
+    }
+    if (status != JEPA_B200_OK) return nullptr;
+    float* d = static_cast<float*>(dalloc(all.size() * 4));
+    if (d) upload(d, all.data(), all.size() * 4);
+    return d;
+  }
   DevMatrix mat(const std::string& name, int64_t N, int64_t K) {
     const jepa_b200_tensor* t = get(name, {N, K});
     if (!t) return DevMatrix();
@@ -423,6 +475,17 @@ int validate_config(const jepa_b200_config* c) {
       return JEPA_B200_ERR_SHAPE;
     const int hd = c->pred_dim / c->pred_heads;
     if (hd != 32 && hd != 64) return JEPA_B200_ERR_SHAPE;
+  }
+  if (c->wm_depth < 0) return JEPA_B200_ERR_ARG;
+  if (c->wm_depth > 0 && c->pred_depth > 0) return JEPA_B200_ERR_ARG;  // both name their tensors pred.*
+  if (c->wm_depth > 0) {
+    // the fused world-model kernel: state width at most 256 in heads of 64,
+    // MLP and output widths at most 1024, at most 32 frames a window
+    if (c->dim > 256 || c->wm_heads < 1 || c->dim != 64 * c->wm_heads || c->wm_mlp < 64 || c->wm_mlp % 64 ||
+        c->wm_mlp > 1024 || c->wm_pred_hidden < 64 || c->wm_pred_hidden % 64 || c->wm_pred_hidden > 1024 ||
+        c->wm_proj_hidden < 64 || c->wm_proj_hidden % 64 || c->wm_proj_hidden > 16384 || c->wm_action_dim < 1 ||
+        c->wm_action_dim > 64 || c->wm_window < 1 || c->wm_window > 32 || !c->has_cls)
+      return JEPA_B200_ERR_SHAPE;
   }
   if (c->rope && (c->has_cls || c->frames / c->tubelet > kRopeMaxPos || c->img_h / c->patch > kRopeMaxPos ||
                   c->img_w / c->patch > kRopeMaxPos))
@@ -511,6 +574,8 @@ int alloc_workspace(jepa_b200_model* m, int B) {
   s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->hz), B * D * 4);
   s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->hzn), B * D * 4);
   s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->hu), static_cast<size_t>(B) * c.mlp * 4);
+  if (c.wm_depth > 0)
+    s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->hp), static_cast<size_t>(B) * c.wm_proj_hidden * 4);
   if (s) {
     free_list(m->ws_allocs);
     return s;
@@ -723,7 +788,8 @@ size_t out_elems(const jepa_b200_model* m, int B, int pool) {
   switch (pool) {
     case JEPA_B200_POOL_NONE: return static_cast<size_t>(B) * m->N * m->cfg.dim;
     case JEPA_B200_POOL_MEAN:
-    case JEPA_B200_POOL_CLS: return static_cast<size_t>(B) * m->cfg.dim;
+    case JEPA_B200_POOL_CLS:
+    case JEPA_B200_POOL_LEWM: return static_cast<size_t>(B) * m->cfg.dim;
     case JEPA_B200_POOL_ATTENTIVE: return static_cast<size_t>(B) * m->cfg.n_classes;
     default: return 0;
   }
@@ -731,7 +797,8 @@ size_t out_elems(const jepa_b200_model* m, int B, int pool) {
 
 int check_encode_args(jepa_b200_model* m, const void* pixels, int B, int pool, const void* out, size_t out_bytes) {
   if (!m || !pixels || !out || B < 1) return JEPA_B200_ERR_ARG;
-  if (pool < JEPA_B200_POOL_NONE || pool > JEPA_B200_POOL_ATTENTIVE) return JEPA_B200_ERR_ARG;
+  if (pool < JEPA_B200_POOL_NONE || pool > JEPA_B200_POOL_LEWM) return JEPA_B200_ERR_ARG;
+  if (pool == JEPA_B200_POOL_LEWM && m->cfg.wm_depth < 1) return JEPA_B200_ERR_MISSING_TENSOR;
   if (pool == JEPA_B200_POOL_ATTENTIVE && !m->has_head) return JEPA_B200_ERR_MISSING_TENSOR;
   if (pool == JEPA_B200_POOL_CLS && !m->cfg.has_cls) return JEPA_B200_ERR_ARG;
   if (static_cast<long long>(B) * m->N > (1ll << 31) / 4096) return JEPA_B200_ERR_SHAPE;
@@ -751,6 +818,8 @@ int enqueue_forward(jepa_b200_model* m, const float* pixels, int B, int pool, fl
       s = launch_layernorm(m->X, R, D, 1, m->norm_g, m->norm_b, c.ln_eps, out, false, st);
     else if (pool == JEPA_B200_POOL_CLS)
       s = launch_layernorm(m->X, B, D, m->N, m->norm_g, m->norm_b, c.ln_eps, out, false, st);
+    else if (pool == JEPA_B200_POOL_LEWM)
+      s = launch_layernorm(m->X, B, D, m->N, m->norm_g, m->norm_b, c.ln_eps, m->hz, false, st);
     else
       s = launch_layernorm(m->X, R, D, 1, m->norm_g, m->norm_b, c.ln_eps, m->Yf, false, st);
     m->launches += 1;
@@ -761,6 +830,12 @@ int enqueue_forward(jepa_b200_model* m, const float* pixels, int B, int pool, fl
     m->launches += 2;
   }
   if (!s && pool == JEPA_B200_POOL_ATTENTIVE) s = run_head(m, B, out, st);
+  if (!s && pool == JEPA_B200_POOL_LEWM) {  // the LeWM projector on the final-normed CLS rows
+    ProfScope ps(m, JEPA_B200_KC_POOL_HEAD, st);
+    s = launch_gemv(m->hz, B, D, m->wproj0, m->b_wproj0, 1, nullptr, 0, m->hp, st);
+    if (!s) s = launch_gemv(m->hp, B, c.wm_proj_hidden, m->wproj2, m->b_wproj2, 0, nullptr, 0, out, st);
+    m->launches += 2;
+  }
   return s;
 }
 
@@ -881,6 +956,7 @@ int enqueue_predict(jepa_b200_model* m, const float* tokens, int B, int nc, int 
 }  // namespace
 
 static void load_sequence(Loader& L);
+static void load_world_model(Loader& L);
 
 extern "C" {
 
@@ -1048,6 +1124,59 @@ static void load_sequence(Loader& L) {
     m->pproj = L.mat("pred.proj.weight", D, Dp);
     m->b_pproj = L.vec("pred.proj.bias", D);
   }
+  if (c.wm_depth > 0) load_world_model(L);
+}
+
+// The LeWM world model: the projector as two matrices for the few-row
+// kernels, the predictor's matrices in three 16-bit arenas (row layout in
+// WmArena), its vectors in f32.
+static void load_world_model(Loader& L) {
+  jepa_b200_model* m = L.m;
+  const jepa_b200_config& c = m->cfg;
+  const int64_t D = c.dim, Mh = c.wm_mlp, Hq = c.wm_pred_hidden, Hp = c.wm_proj_hidden, A = c.wm_action_dim;
+  const int depth = c.wm_depth;
+  m->wproj0 = L.mat("enc.proj.0.weight", Hp, D);
+  m->b_wproj0 = L.vec("enc.proj.0.bias", Hp);
+  m->wproj2 = L.mat("enc.proj.2.weight", D, Hp);
+  m->b_wproj2 = L.vec("enc.proj.2.bias", D);
+  WmArena& a = m->wm;
+  a.D = static_cast<int>(D);
+  a.mlp = static_cast<int>(Mh);
+  a.hq = static_cast<int>(Hq);
+  a.bf16 = c.act_bf16 ? 1 : 0;
+  const int64_t blk = 10 * D + Mh;
+  a.rows_d = static_cast<int>(D + depth * blk + Hq);
+  a.rows_m = static_cast<int>(depth * D);
+  a.rows_h = static_cast<int>(D);
+  a.d = L.dalloc(static_cast<size_t>(a.rows_d) * D * 2);
+  a.m = L.dalloc(static_cast<size_t>(a.rows_m) * Mh * 2);
+  a.h = L.dalloc(static_cast<size_t>(a.rows_h) * Hq * 2);
+  L.arena_put(a.d, 0, "pred.action_embed.2.weight", D, D);
+  for (int b = 0; b < depth; ++b) {
+    const std::string p = "pred.blk." + std::to_string(b) + ".";
+    const int64_t base = D + b * blk;
+    L.arena_put(a.d, base, p + "adaln.weight", 6 * D, D);
+    L.arena_put(a.d, base + 6 * D, p + "attn_qkv.weight", 3 * D, D);
+    L.arena_put(a.d, base + 9 * D, p + "attn_out.weight", D, D);
+    L.arena_put(a.d, base + 10 * D, p + "ffn_up.weight", Mh, D);
+    L.arena_put(a.m, b * D, p + "ffn_down.weight", D, Mh);
+  }
+  L.arena_put(a.d, D + depth * blk, "pred.proj.0.weight", Hq, D);
+  L.arena_put(a.h, 0, "pred.proj.2.weight", D, Hq);
+  m->wm_w_act0 = L.table2d("pred.action_embed.0.weight", D, A);
+  m->wm_b_act0 = L.vec("pred.action_embed.0.bias", D);
+  m->wm_b_act2 = L.vec("pred.action_embed.2.bias", D);
+  m->wm_pos = L.table2d("pred.pos_embed", c.wm_window, D);
+  m->wm_b_ada = L.vec_stack("pred.blk.", "adaln.bias", depth, 6 * D);
+  m->wm_b_qkv = L.vec_stack("pred.blk.", "attn_qkv.bias", depth, 3 * D);
+  m->wm_b_out = L.vec_stack("pred.blk.", "attn_out.bias", depth, D);
+  m->wm_b_up = L.vec_stack("pred.blk.", "ffn_up.bias", depth, Mh);
+  m->wm_b_down = L.vec_stack("pred.blk.", "ffn_down.bias", depth, D);
+  m->wm_norm_g = L.vec("pred.norm.weight", D);
+  m->wm_norm_b = L.vec("pred.norm.bias", D);
+  m->wm_b_p0 = L.vec("pred.proj.0.bias", Hq);
+  m->wm_b_p2 = L.vec("pred.proj.2.bias", D);
+  if (!L.dry && L.status == JEPA_B200_OK && wm_arena_maps(&a) != JEPA_B200_OK) L.status = JEPA_B200_ERR_CUDA;
 }
 
 extern "C" {
@@ -1071,6 +1200,10 @@ int jepa_b200_out_shape(const jepa_b200_model* m, int B, int pool, int64_t shape
     case JEPA_B200_POOL_ATTENTIVE:
       if (!m->has_head) return JEPA_B200_ERR_MISSING_TENSOR;
       shape[1] = m->cfg.n_classes;
+      return 2;
+    case JEPA_B200_POOL_LEWM:
+      if (m->cfg.wm_depth < 1) return JEPA_B200_ERR_MISSING_TENSOR;
+      shape[1] = m->cfg.dim;
       return 2;
     default:
       return JEPA_B200_ERR_ARG;
@@ -1160,6 +1293,72 @@ int jepa_b200_predict(jepa_b200_model* m, const float* tokens, int B, const int*
   if (cudaEventRecord(m->ev1, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
   m->have_timing = true;
   return JEPA_B200_OK;
+}
+
+// One launch of the fused world-model kernel (steps 0: a predictor call).
+static int wm_call(jepa_b200_model* m, const float* states, const float* actions, int C, int T0, int steps,
+                   float* out, void* stream) {
+  const jepa_b200_config& c = m->cfg;
+  WmParams p{};
+  p.D = c.dim;
+  p.heads = c.wm_heads;
+  p.mlp = c.wm_mlp;
+  p.hq = c.wm_pred_hidden;
+  p.A = c.wm_action_dim;
+  p.window = c.wm_window;
+  p.depth = c.wm_depth;
+  p.T0 = T0;
+  p.steps = steps;
+  p.n_cand = C;
+  p.n_act = steps > 0 ? T0 + steps - 1 : T0;
+  p.eps = c.ln_eps;
+  p.states = states;
+  p.actions = actions;
+  p.out = out;
+  p.w_act0 = m->wm_w_act0;
+  p.b_act0 = m->wm_b_act0;
+  p.b_act2 = m->wm_b_act2;
+  p.pos = m->wm_pos;
+  p.b_ada = m->wm_b_ada;
+  p.b_qkv = m->wm_b_qkv;
+  p.b_out = m->wm_b_out;
+  p.b_up = m->wm_b_up;
+  p.b_down = m->wm_b_down;
+  p.norm_g = m->wm_norm_g;
+  p.norm_b = m->wm_norm_b;
+  p.b_p0 = m->wm_b_p0;
+  p.b_p2 = m->wm_b_p2;
+  p.err = m->err;
+  p.timeout_ns = m->timeout_ns;
+  DeviceGuard guard(m->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  m->launches = 0;
+  m->have_timing = false;
+  if (cudaEventRecord(m->ev0, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+  int s = wm_launch(m->wm, p, st);
+  if (s) return s;
+  m->launches = 1;
+  if (cudaEventRecord(m->ev1, st) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+  m->have_timing = true;
+  return JEPA_B200_OK;
+}
+
+int jepa_b200_lewm_predict(jepa_b200_model* m, const float* states, const float* actions, int C, int T, float* out,
+                           size_t out_bytes, void* stream) {
+  if (!m || !states || !actions || !out || C < 1 || T < 1) return JEPA_B200_ERR_ARG;
+  if (m->cfg.wm_depth < 1) return JEPA_B200_ERR_ARG;
+  if (T > m->cfg.wm_window) return JEPA_B200_ERR_SHAPE;
+  if (out_bytes < static_cast<size_t>(C) * T * m->cfg.dim * 4) return JEPA_B200_ERR_SHAPE;
+  return wm_call(m, states, actions, C, T, 0, out, stream);
+}
+
+int jepa_b200_lewm_rollout(jepa_b200_model* m, const float* states, int T0, const float* actions, int C, int steps,
+                           float* out, size_t out_bytes, void* stream) {
+  if (!m || !states || !actions || !out || C < 1 || T0 < 1 || steps < 1) return JEPA_B200_ERR_ARG;
+  if (m->cfg.wm_depth < 1) return JEPA_B200_ERR_ARG;
+  if (out_bytes < static_cast<size_t>(C) * steps * m->cfg.dim * 4) return JEPA_B200_ERR_SHAPE;
+  if (static_cast<long long>(C) * (T0 + steps) * m->cfg.dim >= (1ll << 40)) return JEPA_B200_ERR_SHAPE;
+  return wm_call(m, states, actions, C, T0, steps, out, stream);
 }
 
 int jepa_b200_encode_host(jepa_b200_model* m, const float* pixels, int B, int pool, float* out, size_t out_bytes,

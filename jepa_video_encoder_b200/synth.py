@@ -38,7 +38,8 @@ Q8_0_BLOCK_BYTES = 34   # fp16 scale + 32 x int8
 Q4_0_BLOCK_BYTES = 18   # fp16 scale + 16 bytes of nibbles
 
 POOL_NONE, POOL_MEAN, POOL_CLS, POOL_ATTENTIVE = 0, 1, 2, 3
-POOL_IDS = {"none": POOL_NONE, "mean": POOL_MEAN, "cls": POOL_CLS, "attentive": POOL_ATTENTIVE}
+POOL_LEWM = 4
+POOL_IDS = {"none": POOL_NONE, "mean": POOL_MEAN, "cls": POOL_CLS, "attentive": POOL_ATTENTIVE, "lewm": POOL_LEWM}
 MASK_BIDIR, MASK_BLOCK_CAUSAL = 0, 1
 MASK_IDS = {"bidir": MASK_BIDIR, "block_causal": MASK_BLOCK_CAUSAL}
 

@@ -57,7 +57,7 @@ def _tiny_cfg(**kw):
     return base.with_(**kw)
 
 
-def _load(lib, cfg, table, predictor=None):
+def _load(lib, cfg, table, predictor=None, world_model=None):
     entries = (_abi.TensorEntry * len(table))()
     keep = []
     for i, t in enumerate(table):
@@ -70,7 +70,7 @@ def _load(lib, cfg, table, predictor=None):
             entries[i].shape[j] = s
         entries[i].data = t.data.ctypes.data
         entries[i].nbytes = t.nbytes
-    c = make_config(cfg, predictor=predictor)
+    c = make_config(cfg, predictor=predictor, world_model=world_model)
     h = ctypes.c_void_p()
     st = lib.jepa_b200_load_weights(ctypes.byref(c), entries, len(table), 0, ctypes.byref(h))
     if st == 0:
@@ -228,3 +228,39 @@ def test_predictor_config_and_table_validation(lib):
     bad[i] = synth.Tensor("pred.pos_embed", synth.DT_Q8_0, bad[i].shape,
                           synth.quantize_q8_0(np.zeros(bad[i].shape, np.float32)))
     assert _load(lib, cfg, bad, pc) == _abi.ERR_DTYPE
+
+
+def test_world_model_config_and_table_validation(lib):
+    """The world model's shape limits (state width at most 256 in heads of 64,
+    MLP / output widths multiples of 64 up to 1024, window at most 32, a CLS
+    row to project) and its tensors, checked on the host."""
+    cfg = _tiny_cfg(dim=128, heads=2, mlp=256, mask="bidir")
+    ok = 0 if _has_gpu() else _abi.ERR_CUDA
+    wc = synth.WorldModelConfig(name="w", enc=cfg, dim=128, depth=2, heads=2, mlp=256, window=3, proj_hidden=256,
+                                pred_hidden=256)
+    table = synth.make_tensor_table(cfg) + synth.make_world_model_table(wc)
+    assert _load(lib, cfg, table, world_model=wc) == ok
+    assert _load(lib, cfg, table, world_model=wc.with_(heads=4)) == _abi.ERR_SHAPE        # head dim 32
+    assert _load(lib, cfg, table, world_model=wc.with_(mlp=200)) == _abi.ERR_SHAPE
+    assert _load(lib, cfg, table, world_model=wc.with_(mlp=2048)) == _abi.ERR_SHAPE       # above 1024
+    assert _load(lib, cfg, table, world_model=wc.with_(pred_hidden=96)) == _abi.ERR_SHAPE
+    assert _load(lib, cfg, table, world_model=wc.with_(window=33)) == _abi.ERR_SHAPE
+    assert _load(lib, cfg, table, world_model=wc.with_(action_dim=65)) == _abi.ERR_SHAPE
+    assert _load(lib, cfg, table, world_model=wc.with_(depth=-1)) == _abi.ERR_ARG
+    no_cls = cfg.with_(has_cls=False)
+    assert _load(lib, no_cls, synth.make_tensor_table(no_cls) + synth.make_world_model_table(wc),
+                 world_model=wc) == _abi.ERR_SHAPE
+    pc = synth.PredictorConfig(name="p", enc=cfg, dim=128, depth=1, heads=2, mlp=256)
+    assert _load(lib, cfg, table + synth.make_predictor_table(pc), predictor=pc, world_model=wc) == _abi.ERR_ARG
+    for gone in ("pred.blk.1.adaln.bias", "pred.action_embed.0.weight", "enc.proj.2.weight", "pred.proj.0.bias"):
+        assert _load(lib, cfg, [t for t in table if t.name != gone], world_model=wc) == _abi.ERR_MISSING_TENSOR
+    # the re-typed matrices may be quantised; adaLN and the action embedder stay f32 / f16
+    q = synth.make_tensor_table(cfg) + synth.make_world_model_table(wc.with_(weights="q4_0"))
+    dt = {t.name: t.dtype for t in q}
+    assert dt["pred.proj.0.weight"] == synth.DT_Q4_0 and dt["pred.blk.0.adaln.weight"] == synth.DT_F32
+    assert _load(lib, cfg, q, world_model=wc) == ok
+    bad = list(table)
+    i = [t.name for t in bad].index("pred.blk.0.adaln.weight")
+    bad[i] = synth.Tensor(bad[i].name, synth.DT_Q8_0, bad[i].shape,
+                          synth.quantize_q8_0(np.zeros(bad[i].shape, np.float32)))
+    assert _load(lib, cfg, bad, world_model=wc) == _abi.ERR_DTYPE
