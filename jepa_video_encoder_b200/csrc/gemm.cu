@@ -871,15 +871,28 @@ struct Gemm2Cfg {
   static constexpr int RAW_W = BMODE == B_Q8 ? 64 : 32;
   static constexpr int RAW_BYTES = CONV ? (BN / 2) * RAW_W : 0;
   static constexpr int SC_BYTES = CONV ? (BN / 2) * 16 : 0;
-  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + RAW_BYTES + SC_BYTES + 1023) / 1024 * 1024;
+  // a stage of the MMA ring: the A tile and this CTA's half of the B tile
+  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + 1023) / 1024 * 1024;
   static constexpr int STAGING = 8 * 4096;  // epilogue staging
-  static constexpr int MAX_STAGES = (227 * 1024 - STAGING - 1024) / STAGE_BYTES;
-  // quantised: four stages, converter warp w always converting stage w (its
-  // barrier phases then follow one another, never two apart)
-  static constexpr int STAGES = CONV ? 4 : (BN == 256 ? 6 : (BN == 192 ? 6 : 8));
-  static_assert(!CONV || MAX_STAGES >= 4, "four quantised stages must fit in shared memory");
+  // quantised: four MMA stages, converter warp w always filling the B tile of
+  // stage w; the codes and scales come through a ring of their own, as deep
+  // as the rest of shared memory allows, freed by the converter warps as soon
+  // as a K block is unpacked, so their loads run ahead of the MMA ring
+  // (q4_0's smaller code tiles leave room for a fifth MMA stage beside five
+  // code stages; q8_0 keeps four MMA stages and six code stages).
+  static constexpr int STAGES = CONV ? (BMODE == B_Q4 ? 5 : 4) : (BN == 256 ? 6 : (BN == 192 ? 6 : 8));
+  static constexpr int RAW_STAGE_BYTES = CONV ? (RAW_BYTES + SC_BYTES + 1023) / 1024 * 1024 : 0;
+  static constexpr int RSTAGES_FIT =
+      CONV ? (227 * 1024 - STAGES * STAGE_BYTES - STAGING - 1024) / (RAW_STAGE_BYTES > 0 ? RAW_STAGE_BYTES : 1) : 0;
+  static constexpr int RSTAGES = CONV ? (RSTAGES_FIT > 8 ? 8 : RSTAGES_FIT) : 0;
+  // At least as many code slots as converter warps: the converter warp of K
+  // block i last waited for block i - 4, so with RSTAGES >= 4 the previous fill
+  // of slot i % RSTAGES (block i - RSTAGES) has landed and the slot's barrier is
+  // never two phases behind the parity the warp waits for.  A shallower ring
+  // lets a warp see an old phase as complete.
+  static_assert(!CONV || RSTAGES >= 4, "the code ring needs at least as many slots as converter warps");
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + STAGING + 1024;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + RSTAGES * RAW_STAGE_BYTES + STAGING + 1024;
   static constexpr int THREADS = CONV ? 448 : 320;
 };
 
@@ -951,7 +964,9 @@ __global__ void __launch_bounds__(Gemm2Cfg<BN, BMODE>::THREADS, 1)
   constexpr int S = C::STAGES;
   constexpr bool CONV = C::CONV;
   extern __shared__ uint8_t dsmem[];
-  __shared__ uint64_t full_bar[S], empty_bar[S], conv_bar[S], raw_bar[S], tfull_bar[2], tempty_bar[2], drain_bar;
+  constexpr int RS = C::RSTAGES > 0 ? C::RSTAGES : 1;
+  __shared__ uint64_t full_bar[S], empty_bar[S], conv_bar[S], raw_full[RS], raw_empty[RS], tfull_bar[2], tempty_bar[2],
+      drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -965,7 +980,10 @@ __global__ void __launch_bounds__(Gemm2Cfg<BN, BMODE>::THREADS, 1)
       mbar_init(&full_bar[s], 1);     // leader: one expect-tx arrival + the bytes of both CTAs
       mbar_init(&empty_bar[s], 1);    // both: the leader's multicast commit
       mbar_init(&conv_bar[s], 2);     // leader: the stage's converter warp in each CTA
-      mbar_init(&raw_bar[s], 1);      // both: this CTA's codes and scales (expect-tx + bytes)
+    }
+    for (int r = 0; r < RS; ++r) {
+      mbar_init(&raw_full[r], 1);     // both: this CTA's codes and scales (expect-tx + bytes)
+      mbar_init(&raw_empty[r], 1);    // both: the converter warp that unpacked the slot
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);    // both: the leader's multicast commit
@@ -1018,16 +1036,8 @@ __global__ void __launch_bounds__(Gemm2Cfg<BN, BMODE>::THREADS, 1)
           uint8_t* sB = sA + C::A_BYTES;
           if (rank == 0) mbar_expect_tx(&full_bar[stage], CONV ? 2u * C::A_BYTES : 2u * (C::A_BYTES + C::B_BYTES));
           const uint32_t fb = leader_full0 + static_cast<uint32_t>(stage * sizeof(uint64_t));
-          const int n0 = nb * BN + static_cast<int>(rank) * (BN / 2);
           tma_load_2d_pair(sA, &tmA, fb, kb * 64, mb * 256 + static_cast<int>(rank) * 128);
-          if (!CONV) {
-            tma_load_2d_pair(sB, &tmB, fb, kb * 64, n0);
-          } else {  // this CTA's codes and scales, counted on its own barrier
-            uint8_t* sRaw = sB + C::B_BYTES;
-            mbar_expect_tx(&raw_bar[stage], static_cast<uint32_t>(C::RAW_BYTES + C::SC_BYTES));
-            tma_load_2d(sRaw, &tmB, &raw_bar[stage], kb * C::RAW_W, n0);
-            tma_load_2d(sRaw + C::RAW_BYTES, &tmS, &raw_bar[stage], (2 * kb) & ~7, n0);
-          }
+          if (!CONV) tma_load_2d_pair(sB, &tmB, fb, kb * 64, nb * BN + static_cast<int>(rank) * (BN / 2));
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           if (++stage == S) {
@@ -1036,12 +1046,39 @@ __global__ void __launch_bounds__(Gemm2Cfg<BN, BMODE>::THREADS, 1)
           }
         }
       }
-      if (!ok) {  // let the copies already counted on the barriers land
+      if (!ok && rank == 0) {  // let the copies already counted on the barriers land
         for (int s = 0; s < S; ++s)
-          if ((armed >> s) & 1u) {
-            if (rank == 0) mbar_wait_drain(&full_bar[s], (armed_par >> s) & 1u);
-            if (CONV) mbar_wait_drain(&raw_bar[s], (armed_par >> s) & 1u);
+          if ((armed >> s) & 1u) mbar_wait_drain(&full_bar[s], (armed_par >> s) & 1u);
+      }
+    } else if (CONV && lane == 1) {
+      // this CTA's codes and scales of every K block, through their own ring
+      uint8_t* raw_ring = smem + S * C::STAGE_BYTES;
+      int r = 0;
+      uint32_t rphase = 0, armed = 0, armed_par = 0;
+      bool ok = true;
+      for (int t = cid; t < num_tiles && ok; t += n_clusters) {
+        const int nb = t % p.n_tiles;
+        const int n0 = nb * BN + static_cast<int>(rank) * (BN / 2);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&raw_empty[r], rphase ^ 1, w)) {
+            ok = false;
+            break;
           }
+          uint8_t* sRaw = raw_ring + r * C::RAW_STAGE_BYTES;
+          mbar_expect_tx(&raw_full[r], static_cast<uint32_t>(C::RAW_BYTES + C::SC_BYTES));
+          tma_load_2d(sRaw, &tmB, &raw_full[r], kb * C::RAW_W, n0);
+          tma_load_2d(sRaw + C::RAW_BYTES, &tmS, &raw_full[r], (2 * kb) & ~7, n0);
+          armed |= 1u << r;
+          armed_par = (armed_par & ~(1u << r)) | (rphase << r);
+          if (++r == RS) {
+            r = 0;
+            rphase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < RS; ++s)
+          if ((armed >> s) & 1u) mbar_wait_drain(&raw_full[s], (armed_par >> s) & 1u);
       }
     }
   } else if (warp == 1) {
@@ -1094,7 +1131,7 @@ __global__ void __launch_bounds__(Gemm2Cfg<BN, BMODE>::THREADS, 1)
     const int quad = warp & 3;
     const int chalf = (warp - 2) >> 2;
     const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
-    uint8_t* stage_buf = smem + S * C::STAGE_BYTES + (warp - 2) * 4096;
+    uint8_t* stage_buf = smem + S * C::STAGE_BYTES + C::RSTAGES * C::RAW_STAGE_BYTES + (warp - 2) * 4096;
     bool pending = false;
     int acc = 0;
     uint32_t aphase = 0;
@@ -1131,16 +1168,23 @@ __global__ void __launch_bounds__(Gemm2Cfg<BN, BMODE>::THREADS, 1)
     const int cw = warp - 10;
     const uint32_t leader_conv0 = mapa_shared(smem_u32(&conv_bar[0]), 0);
     const int total = ((num_tiles - cid + n_clusters - 1) / n_clusters) * kblocks;  // K blocks this pair runs
+    uint8_t* raw_ring = smem + S * C::STAGE_BYTES;
     for (int i = cw; i < total; i += 4) {
-      const int stage = i % S;
+      const int stage = i % S, r = i % RS;
       const uint32_t phase = static_cast<uint32_t>(i / S) & 1u;
-      bool okw = mbar_wait(&raw_bar[stage], phase, w);
+      const uint32_t rphase = static_cast<uint32_t>(i / RS) & 1u;
+      // the codes have landed, and the MMA that read this stage's B tile before is done
+      bool okw = mbar_wait(&raw_full[r], rphase, w) && mbar_wait(&empty_bar[stage], phase ^ 1, w);
       if (!__all_sync(0xffffffffu, okw)) break;
       uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
-      quant_stage_convert<BMODE, BN / 2, BF>(sB + C::B_BYTES, sB + C::B_BYTES + C::RAW_BYTES, sB, i % kblocks, lane);
+      uint8_t* sRaw = raw_ring + r * C::RAW_STAGE_BYTES;
+      quant_stage_convert<BMODE, BN / 2, BF>(sRaw, sRaw + C::RAW_BYTES, sB, i % kblocks, lane);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_conv0 + static_cast<uint32_t>(stage * sizeof(uint64_t)));
+      if (lane == 0) {
+        mbar_arrive(&raw_empty[r]);
+        mbar_arrive_cluster(leader_conv0 + static_cast<uint32_t>(stage * sizeof(uint64_t)));
+      }
     }
   }
   tc_fence_before();
