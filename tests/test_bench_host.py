@@ -4,6 +4,7 @@ import json
 import os
 import sys
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -130,3 +131,24 @@ def test_clock_log_keeps_the_timed_region(tmp_path):
     log.write_text("garbled, 0, 1800, 1965, 1, 0x0, Not Active, Not Active, Not Active, Not Active\n")
     c = bench.parse_clock_log(str(log), 0, t0, t1)
     assert c["samples"] == 1 and c["sm_mhz"] == 1800.0 and c["in_region"] is False
+
+
+def test_world_model_flops_and_tile_stream():
+    """The world-model line's FLOP count against a count of the oracle's
+    matrix products, and its weight-stream size against the matrices it
+    covers (every tile 128 x 64 f16; the adaLN chunks start on tiles)."""
+    import bench
+    from jepa_video_encoder_b200 import synth
+    wc = synth.LEWM_WM_STEP
+    D, M, H, A, d = wc.dim, wc.mlp, wc.pred_hidden, wc.action_dim, wc.depth
+    for T in (1, 2, 3):
+        mats = d * (6 * D * D + 3 * D * D + D * D + 2 * D * M) + D * D + A * D + 2 * D * H
+        attn = d * 4 * D * T * (T + 1) // 2
+        assert bench._wm_flops_per_call(wc, T) == 2 * T * mats + attn
+    tiles = bench._wm_tile_bytes(wc) // 16384
+    # D = 192: two 128-row tiles per 192-row chunk, three 64-wide K chunks
+    per_block = 6 * 2 * 3 + 5 * 3 + 2 * 3 + 6 * 3 + 2 * 12
+    assert tiles == 2 * 3 + d * per_block + 6 * 3 + 2 * 12
+    weights = sum(int(np.prod(s)) for n, s, k in synth.world_model_specs(wc)
+                  if n.startswith("pred.") and n.endswith("weight") and len(s) == 2 and "action_embed.0" not in n)
+    assert weights * 2 <= bench._wm_tile_bytes(wc) <= weights * 2 * 1.3
