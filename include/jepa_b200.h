@@ -285,7 +285,7 @@ JEPA_B200_API int jepa_b200_last_launch_count(const jepa_b200_model *m);
 
 /* Kernel classes of the per-kernel timing below. */
 typedef enum {
-  JEPA_B200_KC_PATCH_EMBED = 0, /* implicit-GEMM patch-embed + CLS rows */
+  JEPA_B200_KC_PATCH_EMBED = 0, /* patch matrix + patch-embed GEMM + CLS rows */
   JEPA_B200_KC_LAYERNORM = 1,   /* LN1, LN2 and the final norm */
   JEPA_B200_KC_GEMM_QKV = 2,
   JEPA_B200_KC_ATTENTION = 3,
@@ -373,7 +373,10 @@ JEPA_B200_API int jepa_b200_op_linear_qkv(const void *A, int M, int K, const voi
 JEPA_B200_API int jepa_b200_op_attention(const void *q, const void *k, const void *vt, int B, int heads, int ntok, int npad,
                            int mask, int has_cls, int patches_per_slot, void *out, void *stream);
 
-/* Tubelet patch-embed as an implicit GEMM, plus pos_embed and the CLS row.
+/* Tubelet patch-embed, plus pos_embed and the CLS row: the pixels unfolded
+ * into the patch matrix (f16, in a per-device scratch buffer of the library
+ * that grows on demand: calls on several streams must not overlap), then the
+ * tensor-core GEMM whose epilogue adds the bias and the positional rows.
  * pixels f32 [B, T, 3, H, W]; w_pe f16 [D, kpad] (kpad = 3*kt*p*p rounded up
  * to 64, zero padded); bias f32 [D]; pos f32 [ntok, D]; cls f32 [D] (has_cls);
  * x out f32 [B, ntok, D] with ntok = has_cls + (T/kt)(H/p)(W/p).  The shape

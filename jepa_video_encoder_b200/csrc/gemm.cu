@@ -4,8 +4,9 @@
 // rule": attn_qkv, attn_out, ffn_up, ffn_down per block) spends its time in
 // four GEMMs whose A operand is the token matrix [B*N, D] (or [B*N, 4D]) and
 // whose B operand is a weight matrix [N_out, K] in PyTorch [out, in] order.
-// The same kernel, with a gathering A loader, is the tubelet patch-embed (a
-// conv with stride = kernel, i.e. an implicit GEMM over unfolded pixels).
+// The tubelet patch-embed (a conv with stride = kernel) is the same GEMM over
+// the unfolded patch matrix (built by launch_patchify), with an epilogue that
+// adds the positional row and writes the token rows.
 //
 // Design (one CTA per SM, persistent over output tiles):
 //   warp 0      TMA producer: A tile [128 x 64] and, for f16 weights, the
@@ -18,11 +19,10 @@
 //               TMEM lane quadrant, each half of the columns), bias, then
 //               f16 store / GELU / f32 residual add / QKV head scatter /
 //               patch-embed + pos_embed;
-//   warps 10-13 (quantised weights or patch-embed only) converters: unpack
-//               q8_0 (q*d) or q4_0 ((q-8)*d) blocks, or gather pixels, into
-//               the swizzled operand tile in shared memory.
-// That single-CTA kernel serves the patch-embed and GEMMs of fewer than 256
-// rows.  The encoder's GEMMs (256 rows or more, f16 weights or the f16 copy
+//   warps 10-13 (quantised weights only) converters: unpack q8_0 (q*d) or
+//               q4_0 ((q-8)*d) blocks into the swizzled B tile in shared
+//               memory.
+// That single-CTA kernel serves the GEMMs of fewer than 256 rows.  The encoder's GEMMs (256 rows or more, f16 weights or the f16 copy
 // of dequantised ones) run the CTA-pair variant further down: two SMs share
 // a 256 x BN tile through tcgen05.mma.cta_group::2.
 #include <cudaTypedefs.h>
@@ -271,108 +271,6 @@ __device__ __forceinline__ void fill_b_quant(uint8_t* sB, const GemmParams& p, i
     else
       unpack8<BMODE>(q, nsh, __half2half2(d), w);
     st_shared_v4(sbase + sw128_offset(r, u * 8), w[0], w[1], w[2], w[3]);
-  }
-}
-
-// The patch-embed's A operand is gathered straight from the pixels: a
-// [128 x 64] slice of the unfolded patch matrix per K block, row m = patch
-// (clip b, slot t', patch row, patch col), column k = (c, dt, kh, kw) in the
-// row-major order of a conv weight [D, 3, kt, p, p].  Columns >= 3*kt*p*p
-// and rows >= M are zero.  Pixel offset = rowbase(m) + koff(k), with
-//   rowbase = ((b*T + t'*kt) * 3) * H*W + (patch row * p) * W + patch col * p
-//   koff    = (dt*3 + c) * H*W + kh * W + kw.
-
-// Fast gather for patches whose rows are multiples of 8 pixels on 16-byte
-// aligned image rows: a converter thread always fills the same 8-column unit
-// (u = ct % 8) of the same 8 tile rows, so the pixel offset of each of its
-// rows is computed once per tile (rowbase) and the offset of its unit once
-// per K block; each unit is two 16-byte loads.
-__device__ __forceinline__ bool patch_vec8(const PatchSrc& s) {
-  return (s.patch % 8 == 0) && (s.W % 4 == 0) && ((s.H * s.W) % 4 == 0) &&
-         ((reinterpret_cast<uintptr_t>(s.pixels) & 15) == 0);
-}
-
-__device__ __forceinline__ void patch_rowbases(const GemmParams& p, int m0, int ct, long long (&rowbase)[8]) {
-  const PatchSrc& s = p.patch;
-  const int wp = s.W / s.patch;
-  const int ppf = (s.H / s.patch) * wp;
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int m = m0 + (ct >> 3) + 16 * it;
-    if (m < p.M) {
-      const int b = m / s.n_patches, i = m % s.n_patches;
-      const int tp = i / ppf, rem = i % ppf;
-      const int hp = rem / wp, wq = rem % wp;
-      rowbase[it] = ((static_cast<long long>(b) * s.T + tp * s.tubelet) * 3) * s.H * s.W +
-                    static_cast<long long>(hp * s.patch) * s.W + wq * s.patch;
-    } else {
-      rowbase[it] = -1;
-    }
-  }
-}
-
-template <bool BF>
-__device__ __forceinline__ void fill_a_patch_vec8(uint8_t* sA, const GemmParams& p, int kb, int ct,
-                                                  const long long (&rowbase)[8]) {
-  const PatchSrc& s = p.patch;
-  const int u = ct & 7;
-  const int k = kb * 64 + u * 8;
-  long long koff = -1;
-  if (k < s.k_real) {
-    const int pp = s.patch * s.patch, ktpp = s.tubelet * pp;
-    const int c = k / ktpp, rk = k % ktpp;
-    const int dt = rk / pp, rk2 = rk % pp;
-    const int kh = rk2 / s.patch, kw = rk2 % s.patch;
-    koff = static_cast<long long>(dt * 3 + c) * s.H * s.W + static_cast<long long>(kh) * s.W + kw;
-  }
-  const uint32_t sbase = smem_u32(sA);
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int r = (ct >> 3) + 16 * it;
-    uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;
-    if (rowbase[it] >= 0 && koff >= 0) {
-      const float4* src = reinterpret_cast<const float4*>(s.pixels + rowbase[it] + koff);
-      const float4 a = __ldg(src), b = __ldg(src + 1);
-      w0 = pack2<BF>(a.x, a.y);
-      w1 = pack2<BF>(a.z, a.w);
-      w2 = pack2<BF>(b.x, b.y);
-      w3 = pack2<BF>(b.z, b.w);
-    }
-    st_shared_v4(sbase + sw128_offset(r, u * 8), w0, w1, w2, w3);
-  }
-}
-
-// General gather (any patch size, pixels 4-byte aligned): the ownership of
-// the fast path above, with the 8 column offsets of the thread's unit taken
-// once per K block and 4-byte loads, all 64 of a K block independent.
-template <bool BF>
-__device__ __forceinline__ void fill_a_patch_rows(uint8_t* sA, const GemmParams& p, int kb, int ct,
-                                                  const long long (&rowbase)[8]) {
-  const PatchSrc& s = p.patch;
-  const int u = ct & 7;
-  const int pp = s.patch * s.patch, ktpp = s.tubelet * pp;
-  long long koff[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int k = kb * 64 + u * 8 + e;
-    koff[e] = -1;
-    if (k < s.k_real) {
-      const int c = k / ktpp, rk = k % ktpp;
-      const int dt = rk / pp, rk2 = rk % pp;
-      const int kh = rk2 / s.patch, kw = rk2 % s.patch;
-      koff[e] = static_cast<long long>(dt * 3 + c) * s.H * s.W + static_cast<long long>(kh) * s.W + kw;
-    }
-  }
-  const uint32_t sbase = smem_u32(sA);
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int r = (ct >> 3) + 16 * it;
-    float f[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-      f[e] = (rowbase[it] >= 0 && koff[e] >= 0) ? __ldg(s.pixels + rowbase[it] + koff[e]) : 0.0f;
-    st_shared_v4(sbase + sw128_offset(r, u * 8), pack2<BF>(f[0], f[1]), pack2<BF>(f[2], f[3]),
-                 pack2<BF>(f[4], f[5]), pack2<BF>(f[6], f[7]));
   }
 }
 
@@ -627,13 +525,13 @@ __device__ __forceinline__ void epilogue_tile_qkv(const GemmParams& p, const CUt
   }
 }
 
-template <int BN, int BMODE, bool GATHER, bool ROPE, bool BF>
-__global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
+template <int BN, int BMODE, bool ROPE, bool BF>
+__global__ void __launch_bounds__(BMODE != B_F16 ? 448 : 320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
                    const GemmParams p) {
   using C = GemmCfg<BN>;
-  constexpr bool CONV = (BMODE != B_F16) || GATHER;
+  constexpr bool CONV = BMODE != B_F16;
   constexpr int S = C::STAGES;
   extern __shared__ uint8_t dsmem[];
   __shared__ uint64_t full_bar[S], conv_bar[S], empty_bar[S], tfull_bar[2], tempty_bar[2], drain_bar;
@@ -663,7 +561,7 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    if (!GATHER) tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmA);
     if (BMODE == B_F16) tma_prefetch_desc(&tmB);
   }
   tc_fence_before();
@@ -695,9 +593,9 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
           }
           uint8_t* sA = smem + stage * C::STAGE_BYTES;
           uint8_t* sB = sA + C::A_BYTES;
-          constexpr uint32_t tx = (GATHER ? 0u : (uint32_t)C::A_BYTES) + (BMODE == B_F16 ? (uint32_t)C::B_BYTES : 0u);
+          constexpr uint32_t tx = (uint32_t)C::A_BYTES + (BMODE == B_F16 ? (uint32_t)C::B_BYTES : 0u);
           mbar_expect_tx(&full_bar[stage], tx);
-          if (!GATHER) tma_load_2d(sA, &tmA, &full_bar[stage], kb * 64, mb * 128);
+          tma_load_2d(sA, &tmA, &full_bar[stage], kb * 64, mb * 128);
           if (BMODE == B_F16) tma_load_2d(sB, &tmB, &full_bar[stage], kb * 64, nb * BN);
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
@@ -776,7 +674,7 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
       const int nb = t % p.n_tiles, mb = t / p.n_tiles;
       const int row = mb * 128 + quad * 32 + lane;
       const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
-      constexpr bool kLowReg = BMODE != B_F16 || GATHER;
+      constexpr bool kLowReg = BMODE != B_F16;
       bool done = false;
       if constexpr (!kLowReg) {  // the 128-register kernels keep the row-by-row QKV stores
         if (p.tma_epi && p.epi == EPI_QKV) {
@@ -800,14 +698,11 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
     if (pending && lane == 0) bulk_wait0();
   } else if (CONV) {
     const int ct = threadIdx.x - 320;
-    const bool vec8 = GATHER && patch_vec8(p.patch);
-    long long rowbase[8];
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      const int nb = t % p.n_tiles, mb = t / p.n_tiles;
-      if (GATHER) patch_rowbases(p, mb * 128, ct, rowbase);
+      const int nb = t % p.n_tiles;
       for (int kb = 0; kb < kblocks; ++kb) {
         bool okw = mbar_wait(&empty_bar[stage], phase ^ 1, w);
         okw = __all_sync(0xffffffffu, okw);
@@ -815,14 +710,8 @@ __global__ void __launch_bounds__((BMODE != B_F16 || GATHER) ? 448 : 320, 1)
           ok = false;
           break;
         }
-        uint8_t* sA = smem + stage * C::STAGE_BYTES;
-        uint8_t* sB = sA + C::A_BYTES;
-        if (GATHER && vec8)
-          fill_a_patch_vec8<BF>(sA, p, kb, ct, rowbase);
-        else if (GATHER)
-          fill_a_patch_rows<BF>(sA, p, kb, ct, rowbase);
-        else
-          fill_b_quant<BMODE, BN, BF>(sB, p, nb * BN, kb, ct);
+        uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
+        fill_b_quant<BMODE, BN, BF>(sB, p, nb * BN, kb, ct);
         fence_proxy_async_smem();
         mbar_arrive(&conv_bar[stage]);
         if (++stage == S) {
@@ -1270,13 +1159,15 @@ int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& Win
   // 256 x 64 weight tile of a 256 x 256 x 64 product) and smaller ones in
   // the single-CTA kernel's.
   DevMatrix W = Win;
+  // a patch source (EPI_PATCH) comes with A, the unfolded patch matrix; the
+  // epilogue places the rows and adds the positional table
   if (W.bmode != B_F16 && W.f16 && !patch && M >= 256) {
     W.bmode = B_F16;
     W.data = W.f16;
     W.scales = nullptr;
   }
   if (!op || !out || M < 1 || K < 64 || K % 64 != 0 || W.K != K || W.N < 1 || !W.data) return JEPA_B200_ERR_SHAPE;
-  if (!patch && !A) return JEPA_B200_ERR_ARG;
+  if (!A) return JEPA_B200_ERR_ARG;
   const int N = W.N;
   const int bn = N % 256 == 0 ? 256 : (N % 192 == 0 ? 192 : (N % 128 == 0 ? 128 : 0));
   if (!bn) return JEPA_B200_ERR_SHAPE;
@@ -1288,7 +1179,7 @@ int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& Win
   op->bn = bn;
   op->bmode = W.bmode;
   op->bf16 = W.bf16;  // the model's 16-bit type: A, the unpacked weights and 16-bit outputs
-  op->gather = patch ? 1 : 0;
+  op->gather = 0;
   GemmParams& p = op->p;
   p.M = M;
   p.N = N;
@@ -1303,7 +1194,7 @@ int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& Win
   if (patch) p.patch = *patch;
   p.bq = W.bmode != B_F16 ? W.data : nullptr;
   p.bscale = W.scales;
-  if (!patch) {
+  {
     const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
     const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
     const uint32_t box[2] = {64, 128};
@@ -1341,7 +1232,7 @@ int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& Win
   }
   // at least two 128-row blocks: the CTA-pair kernel (quantised weights need
   // a scale table whose rows TMA can address: 8-scale groups, 16-byte rows)
-  op->pair = (!patch && M >= 256 && (W.bmode == B_F16 || (W.scales_pad && W.sc_ld % 8 == 0))) ? 1 : 0;
+  op->pair = (M >= 256 && (W.bmode == B_F16 || (W.scales_pad && W.sc_ld % 8 == 0))) ? 1 : 0;
   if (W.bmode == B_F16) {
     const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
     const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
@@ -1370,12 +1261,12 @@ int gemm_prepare(GemmOp* op, const __half* A, int M, int K, const DevMatrix& Win
   return JEPA_B200_OK;
 }
 
-template <int BN, int BMODE, bool GATHER, bool ROPE, bool BF>
+template <int BN, int BMODE, bool ROPE, bool BF>
 static int launch_impl(const GemmOp& op, cudaStream_t st) {
-  auto kern = gemm_tc_kernel<BN, BMODE, GATHER, ROPE, BF>;
+  auto kern = gemm_tc_kernel<BN, BMODE, ROPE, BF>;
   static std::atomic<unsigned long long> attr_done{0};
   if (!smem_attr_once(attr_done, kern, GemmCfg<BN>::SMEM)) return JEPA_B200_ERR_CUDA;
-  constexpr int threads = (BMODE != B_F16 || GATHER) ? 448 : 320;
+  constexpr int threads = BMODE != B_F16 ? 448 : 320;
   if (launch_pdl(kern, dim3(op.grid), dim3(threads), GemmCfg<BN>::SMEM, st, 1, op.tmA, op.tmB, op.tmC, op.tmC2, op.p) !=
       cudaSuccess)
     return JEPA_B200_ERR_CUDA;
@@ -1395,7 +1286,7 @@ static int launch_pair(const GemmOp& op, cudaStream_t st) {
 }
 
 // Every instance is selected here from the op: tile width, weight format,
-// patch gather, rotary q / k, 16-bit activation type.
+// rotary q / k, 16-bit activation type.
 template <bool BF>
 static int launch_typed(const GemmOp& op, cudaStream_t st) {
   // rotary q / k only in the QKV GEMMs of a rotary model: their own instances,
@@ -1409,22 +1300,15 @@ static int launch_typed(const GemmOp& op, cudaStream_t st) {
   }
 #define JB_SINGLE(BNV)                                                                                              \
   switch (op.bmode) {                                                                                               \
-    case B_Q8: return rope ? launch_impl<BNV, B_Q8, false, true, BF>(op, st) : launch_impl<BNV, B_Q8, false, false, BF>(op, st); \
-    case B_Q4: return rope ? launch_impl<BNV, B_Q4, false, true, BF>(op, st) : launch_impl<BNV, B_Q4, false, false, BF>(op, st); \
-    default: return rope ? launch_impl<BNV, B_F16, false, true, BF>(op, st) : launch_impl<BNV, B_F16, false, false, BF>(op, st); \
+    case B_Q8: return rope ? launch_impl<BNV, B_Q8, true, BF>(op, st) : launch_impl<BNV, B_Q8, false, BF>(op, st); \
+    case B_Q4: return rope ? launch_impl<BNV, B_Q4, true, BF>(op, st) : launch_impl<BNV, B_Q4, false, BF>(op, st); \
+    default: return rope ? launch_impl<BNV, B_F16, true, BF>(op, st) : launch_impl<BNV, B_F16, false, BF>(op, st); \
   }
   if (op.pair) {
     switch (op.bn) {
       case 256: JB_PAIR(256)
       case 192: JB_PAIR(192)
       default: JB_PAIR(128)
-    }
-  }
-  if (op.gather) {
-    switch (op.bn) {
-      case 256: return launch_impl<256, B_F16, true, false, BF>(op, st);
-      case 192: return launch_impl<192, B_F16, true, false, BF>(op, st);
-      default: return launch_impl<128, B_F16, true, false, BF>(op, st);
     }
   }
   switch (op.bn) {

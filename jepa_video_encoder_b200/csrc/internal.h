@@ -55,7 +55,7 @@ struct QkvDst {
 // Positions per axis the rotary table holds (slots, patch rows, patch columns).
 constexpr int kRopeMaxPos = 64;
 
-// Source geometry of the implicit-GEMM patch-embed.
+// Source geometry of the patch-embed (the patch matrix and the GEMM epilogue).
 struct PatchSrc {
   const float* pixels = nullptr;
   int T = 0, H = 0, W = 0, patch = 0, tubelet = 0;

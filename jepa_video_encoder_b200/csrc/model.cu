@@ -3,7 +3,7 @@
 // pass (the C ABI calls of include/jepa_b200.h).
 //
 // Sequence of jepa_b200_encode (B clips, R = B * N token rows):
-//   patch-embed (implicit GEMM + pos_embed) and the CLS rows       -> X f32 [R, D]
+//   patch matrix, patch-embed GEMM (+ pos_embed) and the CLS rows   -> X f32 [R, D]
 //   per block:  LN1 -> Y f16; QKV GEMM -> Q, K, V^T (head-major)
 //               attention -> O f16 [R, D]; out GEMM: X += O Wo^T + bo
 //               LN2 -> Y; up GEMM + GELU -> H f16 [R, 4D]; down GEMM: X += H Wd^T + bd
@@ -20,6 +20,7 @@
 #include <vector>
 
 #include "internal.h"
+#include "patchify.h"
 #include "world_model.h"
 
 using namespace jb;
@@ -100,6 +101,7 @@ struct jepa_b200_model {
   float *Yf = nullptr, *partial = nullptr;
   float *hq = nullptr, *hattn = nullptr, *hz = nullptr, *hzn = nullptr, *hu = nullptr;
   float* hp = nullptr;  // the LeWM projector's hidden rows [B, wm_proj_hidden]
+  __half* Ape = nullptr;  // the unfolded patch matrix [B * Np, Kpe_pad] (patch-embed A operand)
   std::vector<void*> ws_allocs;
   std::vector<BlockOps> enc_ops, head_ops;
   GemmOp pe_op, kv_op;
@@ -574,6 +576,7 @@ int alloc_workspace(jepa_b200_model* m, int B) {
   s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->hz), B * D * 4);
   s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->hzn), B * D * 4);
   s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->hu), static_cast<size_t>(B) * c.mlp * 4);
+  s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->Ape), static_cast<size_t>(B) * m->Np * m->Kpe_pad * 2);
   if (c.wm_depth > 0)
     s = s ? s : alloc_ws(m, reinterpret_cast<void**>(&m->hp), static_cast<size_t>(B) * c.wm_proj_hidden * 4);
   if (s) {
@@ -608,7 +611,9 @@ int prepare_ops(jepa_b200_model* m, int B) {
   ps.pos = m->pos;
   ps.ntok = m->N;
   ps.has_cls = c.has_cls ? 1 : 0;
-  if ((s = gemm_prepare(&m->pe_op, nullptr, B * m->Np, m->Kpe_pad, m->pe, m->b_pe, EPI_PATCH, m->X, c.dim, nullptr,
+  // patch-embed: the unfolded patch matrix (launch_patchify) through the
+  // TMA-fed GEMM, whose epilogue adds the bias and positional row in place
+  if ((s = gemm_prepare(&m->pe_op, m->Ape, B * m->Np, m->Kpe_pad, m->pe, m->b_pe, EPI_PATCH, m->X, c.dim, nullptr,
                         &ps)))
     return s;
   if ((s = attn_prepare(&m->attn_enc, m->Q, m->Kb, m->Vt, B, c.heads, m->N, m->npad, c.mask, c.has_cls, m->ppf,
@@ -747,12 +752,12 @@ int run_block(jepa_b200_model* m, const LayerW& L, const BlockOps& ops, const At
 int run_embed_and_blocks(jepa_b200_model* m, const float* pixels, int B, int n_layers, cudaStream_t st) {
   const jepa_b200_config& c = m->cfg;
   const int R = B * m->N;
-  GemmOp pe = m->pe_op;
-  pe.p.patch.pixels = pixels;
   {
     ProfScope ps(m, JEPA_B200_KC_PATCH_EMBED, st);
-    JB_TRY(gemm_launch(pe, st, m->err, m->timeout_ns));
-    m->launches += 1;
+    PatchSrc src = m->pe_op.p.patch;
+    JB_TRY(launch_patchify(pixels, src, B, m->Kpe_pad, m->Ape, st, c.act_bf16 != 0));
+    JB_TRY(gemm_launch(m->pe_op, st, m->err, m->timeout_ns));
+    m->launches += 2;
     if (c.has_cls) {
       JB_TRY(launch_cls_rows(m->X, B, m->N, c.dim, m->cls, m->pos, st));
       m->launches += 1;

@@ -9,6 +9,7 @@
 #include <algorithm>
 
 #include "internal.h"
+#include "patchify.h"
 
 namespace jb {
 
@@ -135,6 +136,78 @@ __global__ void cls_rows_kernel(float* x, int B, int ntok, int D, const float* c
 int launch_cls_rows(float* x, int B, int ntok, int D, const float* cls, const float* pos, cudaStream_t st) {
   if (!x || !cls || !pos) return JEPA_B200_ERR_ARG;
   launch_pdl(cls_rows_kernel, dim3((D + 255) / 256, B), dim3(256), 0, st, 1, x, B, ntok, D, cls, pos);
+  return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
+}
+
+// Patch-embed, input side: the unfolded patch matrix of the tubelet
+// convolution, rounded to the 16-bit type, as the A operand of a TMA-fed
+// GEMM.  Row m = patch (clip b, slot t', patch row py, patch column px),
+// column k = (c, dt, kh, kw) in the row-major order of a conv weight
+// [D, 3, kt, p, p]; columns k >= 3 kt p^2 (up to the padded K) are zero.
+// One thread writes 8 consecutive columns of one row (16 bytes); with
+// p % 8 == 0 those are 8 consecutive pixels of one image row, read as two
+// 16-byte loads when the image rows allow it.
+template <bool BF>
+__global__ void __launch_bounds__(256) patchify_kernel(const float* __restrict__ px, int T, int H, int W, int p,
+                                                        int kt, int n_patches, long long rows, int K, int Kpad,
+                                                        int vec, uint16_t* __restrict__ a) {
+  pdl_wait();
+  pdl_trigger();
+  const int groups = Kpad / 8;
+  const long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (g >= rows * groups) return;
+  const long long m = g / groups;
+  const int k0 = static_cast<int>(g - m * groups) * 8;
+  const long long b = m / n_patches;
+  const int i = static_cast<int>(m - b * n_patches);
+  const int wp = W / p, ppf = (H / p) * wp;
+  const int ts = i / ppf, py = (i % ppf) / wp, pxi = i % wp;
+  const size_t hw = static_cast<size_t>(H) * W;
+  float v[8];
+  if (vec && k0 + 8 <= K) {
+    // 8 pixels of one image row (p % 8 == 0): kw = k0 % p .. + 7, 16-byte aligned
+    const int kw = k0 % p, kh = (k0 / p) % p, dt = (k0 / (p * p)) % kt, c = k0 / (p * p * kt);
+    const size_t f = static_cast<size_t>(b) * T + static_cast<size_t>(ts) * kt + dt;
+    const float* src = px + (f * 3 + c) * hw + static_cast<size_t>(py * p + kh) * W + pxi * p + kw;
+    const float4 u = __ldg(reinterpret_cast<const float4*>(src)), w = __ldg(reinterpret_cast<const float4*>(src + 4));
+    v[0] = u.x;
+    v[1] = u.y;
+    v[2] = u.z;
+    v[3] = u.w;
+    v[4] = w.x;
+    v[5] = w.y;
+    v[6] = w.z;
+    v[7] = w.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int k = k0 + e;
+      v[e] = 0.0f;
+      if (k < K) {
+        const int kw = k % p, kh = (k / p) % p, dt = (k / (p * p)) % kt, c = k / (p * p * kt);
+        const size_t f = static_cast<size_t>(b) * T + static_cast<size_t>(ts) * kt + dt;
+        v[e] = __ldg(px + (f * 3 + c) * hw + static_cast<size_t>(py * p + kh) * W + pxi * p + kw);
+      }
+    }
+  }
+  *reinterpret_cast<uint4*>(a + m * Kpad + k0) =
+      make_uint4(pack2<BF>(v[0], v[1]), pack2<BF>(v[2], v[3]), pack2<BF>(v[4], v[5]), pack2<BF>(v[6], v[7]));
+}
+
+int launch_patchify(const float* pixels, const PatchSrc& s, int B, int Kpad, void* a, cudaStream_t st, bool bf16) {
+  if (!pixels || !a || B < 1) return JEPA_B200_ERR_ARG;
+  if (Kpad % 8 != 0 || Kpad < s.k_real || s.patch < 1 || s.tubelet < 1 || (reinterpret_cast<uintptr_t>(a) & 15))
+    return JEPA_B200_ERR_SHAPE;
+  // 16-byte pixel loads need 8-pixel patch rows on 16-byte-aligned image rows
+  const int vec = (s.patch % 8 == 0) && (s.W % 4 == 0) && ((static_cast<size_t>(s.H) * s.W) % 4 == 0) &&
+                          ((reinterpret_cast<uintptr_t>(pixels) & 15) == 0)
+                      ? 1
+                      : 0;
+  const long long rows = static_cast<long long>(B) * s.n_patches;
+  const long long threads = rows * (Kpad / 8);
+  launch_pdl(bf16 ? patchify_kernel<true> : patchify_kernel<false>, dim3(static_cast<unsigned>((threads + 255) / 256)),
+             dim3(256), 0, st, 1, pixels, s.T, s.H, s.W, s.patch, s.tubelet, s.n_patches, rows, s.k_real, Kpad, vec,
+             static_cast<uint16_t*>(a));
   return cudaGetLastError() == cudaSuccess ? JEPA_B200_OK : JEPA_B200_ERR_CUDA;
 }
 

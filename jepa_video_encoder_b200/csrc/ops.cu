@@ -5,6 +5,7 @@
 #include <mutex>
 
 #include "internal.h"
+#include "patchify.h"
 
 using namespace jb;
 
@@ -198,9 +199,34 @@ int jepa_b200_op_patch_embed(const float* pixels, int B, int T, int H, int W, in
   ps.pos = pos;
   ps.ntok = ntok;
   ps.has_cls = has_cls ? 1 : 0;
+  // the unfolded patch matrix goes to a per-device scratch buffer that grows
+  // on demand (growing waits for the device to be idle)
+  static std::mutex mu;
+  static void* scratch[64] = {nullptr};
+  static size_t scratch_bytes[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return JEPA_B200_ERR_CUDA;
+  const size_t need = static_cast<size_t>(B) * n_patches * kpad * 2;
+  void* a = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (scratch_bytes[dev] < need) {
+      cudaDeviceSynchronize();
+      if (scratch[dev]) cudaFree(scratch[dev]);
+      scratch[dev] = nullptr;
+      scratch_bytes[dev] = 0;
+      if (cudaMalloc(&scratch[dev], need) != cudaSuccess) return JEPA_B200_ERR_CUDA;
+      scratch_bytes[dev] = need;
+    }
+    a = scratch[dev];
+  }
   GemmOp op;
-  if ((s = gemm_prepare(&op, nullptr, B * n_patches, kpad, Wm, bias, EPI_PATCH, x, D, nullptr, &ps))) return s;
+  if ((s = gemm_prepare(&op, static_cast<const __half*>(a), B * n_patches, kpad, Wm, bias, EPI_PATCH, x, D, nullptr,
+                        &ps)))
+    return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = launch_patchify(pixels, ps, B, kpad, a, st, false))) return s;
   if ((s = gemm_launch(op, st, e, g_timeout_ns))) return s;
   if (has_cls) return launch_cls_rows(x, B, ntok, D, cls, pos, st);
   return JEPA_B200_OK;
