@@ -181,3 +181,24 @@ def test_lewm_errors():
         m2.encode(dev(synth.make_pixels(wc.enc, batch=1)), pool="lewm")
     assert e.value.status == jb._abi.ERR_MISSING_TENSOR
     m2.close()
+
+
+def test_lewm_timeout_path():
+    """A zero wait bound makes the world-model kernel give up at its first
+    wait and unwind (every role drains what it issued); the model reports
+    ERR_TIMEOUT, and the next call with the normal bound gives the same bits
+    as before."""
+    need_cuda()
+    wc = _wc(frames=1, steps=3)
+    m, _ = _model(wc)
+    st, ac = synth.make_world_model_inputs(wc, candidates=5)
+    good = host(m.lewm_rollout(dev(st), dev(ac), wc.steps))
+    assert m.sync_status() == 0
+    m.set_timeout_ns(0)
+    m.lewm_rollout(dev(st), dev(ac), wc.steps)
+    assert m.sync_status() == jb._abi.ERR_TIMEOUT
+    m.set_timeout_ns(4_000_000_000)
+    again = host(m.lewm_rollout(dev(st), dev(ac), wc.steps))
+    assert m.sync_status() == 0
+    assert np.array_equal(good, again)
+    m.close()
