@@ -788,29 +788,48 @@ struct Gemm2Cfg {
 // One converter warp unpacks a whole stage: this CTA's BN/2 weight rows of
 // one K block, read from the staged codes and scales, to f16 in the
 // swizzled B tile.  Lane l takes the K offset 8 (l % 8) of rows l / 8 + 4 j.
+// The rows go in batches of eight whose shared-memory loads are all issued
+// before the batch is converted, the next batch's loads before this batch's
+// stores: the loads and stores are ordered asm statements, so without the
+// batching each row's load would wait for the previous row's store and the
+// unpack of a stage would run at shared-memory latency.
 template <int BMODE, int ROWS, bool BF>
 __device__ __forceinline__ void quant_stage_convert(const uint8_t* sRaw, const uint8_t* sSc, uint8_t* sB, int kb,
                                                     int lane) {
   constexpr int RAW_W = BMODE == B_Q8 ? 64 : 32;
+  constexpr int kBatch = 8, kBatches = ROWS / (4 * kBatch);
+  static_assert(ROWS % (4 * kBatch) == 0, "rows of a stage in whole batches");
   const uint32_t raw = smem_u32(sRaw), sc = smem_u32(sSc), sbase = smem_u32(sB);
-  const int u = lane & 7;
+  const int u = lane & 7, r0 = lane >> 3;
   // q8_0: bytes 8u..8u+7 of the row's 64; q4_0: the K offset's block (u / 4)
   // holds 16 bytes, its elements j and j + 16 in byte j (low, high nibble)
   const int off = BMODE == B_Q8 ? 8 * u : 16 * (u >> 2) + 8 * (u & 1);
   const int nsh = (BMODE == B_Q4 && (u & 2)) ? 4 : 0;
   const int sidx = ((2 * kb) & 7) + (u >> 2);  // the unit's scale in the row's group of 8
-#pragma unroll 8
-  for (int r = lane >> 3; r < ROWS; r += 4) {
-    uint2 q;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(q.x), "=r"(q.y) : "r"(raw + r * RAW_W + off));
-    unsigned short dbits;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(dbits) : "r"(sc + r * 16 + sidx * 2));
-    uint32_t w[4];
-    if constexpr (BF)
-      unpack8_bf16<BMODE>(q, nsh, __half2float(__ushort_as_half(dbits)), w);
-    else
-      unpack8<BMODE>(q, nsh, __half2half2(__ushort_as_half(dbits)), w);
-    st_shared_v4(sbase + sw128_offset(r, u * 8), w[0], w[1], w[2], w[3]);
+  uint2 q[2][kBatch];
+  unsigned short dbits[2][kBatch];
+  auto load = [&](int b, uint2 (&qb)[kBatch], unsigned short (&db)[kBatch]) {
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int r = r0 + 4 * (kBatch * b + j);
+      asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(qb[j].x), "=r"(qb[j].y) : "r"(raw + r * RAW_W + off));
+      asm volatile("ld.shared.u16 %0, [%1];" : "=h"(db[j]) : "r"(sc + r * 16 + sidx * 2));
+    }
+  };
+  load(0, q[0], dbits[0]);
+#pragma unroll
+  for (int b = 0; b < kBatches; ++b) {
+    if (b + 1 < kBatches) load(b + 1, q[(b + 1) & 1], dbits[(b + 1) & 1]);
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int r = r0 + 4 * (kBatch * b + j);
+      uint32_t w[4];
+      if constexpr (BF)
+        unpack8_bf16<BMODE>(q[b & 1][j], nsh, __half2float(__ushort_as_half(dbits[b & 1][j])), w);
+      else
+        unpack8<BMODE>(q[b & 1][j], nsh, __half2half2(__ushort_as_half(dbits[b & 1][j])), w);
+      st_shared_v4(sbase + sw128_offset(r, u * 8), w[0], w[1], w[2], w[3]);
+    }
   }
 }
 
