@@ -743,12 +743,12 @@ __global__ void __launch_bounds__(BMODE != B_F16 ? 448 : 320, 1)
 //
 // B operand: f16 weights come by TMA (BMODE B_F16, 320 threads).  q8_0 /
 // q4_0 weights (BMODE B_Q8 / B_Q4, 448 threads) are unpacked in the loader:
-// four converter warps per CTA read the codes and scales of their CTA's
-// BN/2 weight rows straight from global memory, one K block ahead of the
-// one they convert (the loads need no shared-memory stage), and write the
-// f16 values into the swizzled B tile; each converter warp then arrives on
-// the leader's conversion barrier (cluster scope), which the MMA issuer
-// waits for beside the TMA barrier of the A tiles.
+// a second producer lane stages the codes and scale groups of the CTA's
+// BN/2 weight rows by TMA into a ring of their own, four converter warps
+// per CTA unpack them (shared memory to shared memory) into the swizzled
+// f16 B tile of the MMA ring, and each converter warp then arrives on the
+// leader's conversion barrier (cluster scope), which the MMA issuer waits
+// for beside the TMA barrier of the A tiles.
 template <int BN, int BMODE>
 struct Gemm2Cfg {
   static constexpr bool CONV = BMODE != B_F16;
