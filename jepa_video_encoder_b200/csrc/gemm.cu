@@ -45,17 +45,45 @@ struct GemmCfg {
   static constexpr int SMEM = STAGES * STAGE_BYTES + 8 * 4096 + 1024;  // + epilogue staging
 };
 
-// Two GELUs: packed polynomial, or (LOWREG, kernels launched with 448
-// threads and so at most 128 registers a thread) the scalar one whose
-// coefficients are instruction immediates rather than register pairs.
+// gelu_q's coefficients, each twice, as the operand pairs of the packed
+// polynomial in constant memory: the 128-register kernels read them from the
+// constant bank instead of holding twelve register pairs (the same
+// coefficients as gelu_q, which a host test compares).
+__constant__ float2 kGeluPairs[12] = {
+    {-1.000000000e+00f, -1.000000000e+00f}, {-1.151105762e+00f, -1.151105762e+00f},
+    {-4.592085183e-01f, -4.592085183e-01f}, {-5.247146264e-02f, -5.247146264e-02f},
+    {6.975546945e-03f, 6.975546945e-03f}, {-5.228150712e-06f, -5.228150712e-06f},
+    {-2.895472280e-04f, -2.895472280e-04f}, {8.469620661e-05f, 8.469620661e-05f},
+    {-1.389817317e-05f, -1.389817317e-05f}, {1.411672088e-06f, 1.411672088e-06f},
+    {-8.283102204e-08f, -8.283102204e-08f}, {2.152039880e-09f, 2.152039880e-09f},
+};
+
+// Two GELUs in packed f32x2 arithmetic with the coefficient pairs from
+// constant memory: the same f32 operations as gelu2 (and gelu1), so the
+// same results.
+__device__ __forceinline__ void gelu2_cbank(float& x0, float& x1) {
+  const float u0 = fabsf(x0), u1 = fabsf(x1);
+  const uint64_t c = f2_pack(fminf(u0, 6.0f), fminf(u1, 6.0f));
+  uint64_t q = *reinterpret_cast<const uint64_t*>(&kGeluPairs[11]);
+#pragma unroll
+  for (int k = 10; k >= 0; --k) q = f2_fma(q, c, *reinterpret_cast<const uint64_t*>(&kGeluPairs[k]));
+  float q0, q1;
+  f2_unpack(q, q0, q1);
+  x0 = fmaf(-u0, ex2_approx(q0), fmaxf(x0, 0.0f));
+  x1 = fmaf(-u1, ex2_approx(q1), fmaxf(x1, 0.0f));
+}
+
+// Two GELUs: coefficient pairs in registers, or (LOWREG, kernels launched
+// with 448 threads and so at most 128 registers a thread) in constant
+// memory.  The scalar form with immediate coefficients (gelu1) issues twice
+// the polynomial's instructions, which in the quantised-weight kernels the
+// converter warps on the same SM sub-partitions pay for.
 template <bool LOWREG>
 __device__ __forceinline__ void gelu_pair(float& a, float& b) {
-  if (LOWREG) {
-    a = gelu1(a);
-    b = gelu1(b);
-  } else {
+  if (LOWREG)
+    gelu2_cbank(a, b);
+  else
     gelu2(a, b);
-  }
 }
 
 // Rotary positions: turn the pair (x0, x1) at head dims (d, d + 1), d even,

@@ -62,3 +62,17 @@ def test_gelu_fit_reproduces_kernel_table():
     fitted = mod.fit()
     c = kernel_coefficients()
     np.testing.assert_allclose(fitted, c, rtol=1e-5, atol=1e-12)
+
+
+def test_gemm_constant_pairs_match_kernel_table():
+    """The quantised-weight GEMMs evaluate the same polynomial from a table of
+    coefficient pairs in constant memory (gemm.cu, kGeluPairs): both entries
+    of every pair equal gelu_q's coefficient of the same degree."""
+    src = (CSRC / "gemm.cu").read_text()
+    body = re.search(r"__constant__ float2 kGeluPairs\[12\]\s*=\s*\{(.*?)\};", src, re.S)
+    assert body, "kGeluPairs not found in gemm.cu"
+    pairs = re.findall(r"\{\s*([^,{}]+?)f?\s*,\s*([^,{}]+?)f?\s*\}", body.group(1))
+    assert len(pairs) == 12
+    got = np.array([[float(a.rstrip("f")), float(b.rstrip("f"))] for a, b in pairs], dtype=np.float32)
+    c = kernel_coefficients()
+    assert np.array_equal(got[:, 0], c) and np.array_equal(got[:, 1], c)
