@@ -202,3 +202,28 @@ def test_lewm_timeout_path():
     assert m.sync_status() == 0
     assert np.array_equal(good, again)
     m.close()
+
+
+def test_lewm_largest_shape():
+    """The largest shape the kernel accepts (state width 256 in four 64-dim
+    heads, MLP and output hidden widths 1024, a 32-frame window: the shared
+    memory the launch reserves): one predictor call over 32 frames, and a
+    34-step rollout whose window fills up and then slides."""
+    need_cuda()
+    enc = synth.small_config(synth.LEWM_VIT_TI, dim=256, heads=4, mlp=256, depth=1)
+    wc = _wc(enc=enc, dim=256, heads=4, mlp=1024, pred_hidden=1024, window=32, frames=32)
+    m, table = _model(wc)
+    W = _W(table)
+    st, ac = synth.make_world_model_inputs(wc, candidates=3)
+    got = host(m.lewm_predict(dev(st), dev(ac)))
+    assert m.sync_status() == 0
+    ref = orc.lewm_predict(wc, W, st, ac)
+    assert_tokens_close(got, ref, COS_F16, REL_MAX_F16, what="largest shape, predict")
+    wr = wc.with_(frames=1, steps=34)
+    st, ac = synth.make_world_model_inputs(wr, candidates=2)
+    got = host(m.lewm_rollout(dev(st), dev(ac), wr.steps))
+    assert m.sync_status() == 0
+    m.close()
+    ref = orc.lewm_rollout(wr, W, st, ac, wr.steps)
+    assert_tokens_close(got, ref, COS_ROLLOUT, None, what="largest shape, rollout")
+    assert_tokens_close(got[:, :1], ref[:, :1], COS_F16, REL_MAX_F16, what="largest shape, rollout step 0")
