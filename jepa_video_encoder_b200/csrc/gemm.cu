@@ -791,12 +791,13 @@ struct Gemm2Cfg {
   // a stage of the MMA ring: the A tile and this CTA's half of the B tile
   static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + 1023) / 1024 * 1024;
   static constexpr int STAGING = 8 * 4096;  // epilogue staging
-  // quantised: four MMA stages, converter warp w always filling the B tile of
-  // stage w; the codes and scales come through a ring of their own, as deep
-  // as the rest of shared memory allows, freed by the converter warps as soon
-  // as a K block is unpacked, so their loads run ahead of the MMA ring
-  // (q4_0's smaller code tiles leave room for a fifth MMA stage beside five
-  // code stages; q8_0 keeps four MMA stages and six code stages).
+  // quantised: four or five MMA stages, converter warp w filling the B tiles
+  // of K blocks w, w + 4, ...; the codes and scales come through a ring of
+  // their own, as deep as the rest of shared memory allows, freed by the
+  // converter warps as soon as a K block is unpacked, so their loads run
+  // ahead of the MMA ring (q4_0's smaller code tiles leave room for a fifth
+  // MMA stage beside five code stages; q8_0 keeps four MMA stages and six
+  // code stages).
   static constexpr int STAGES = CONV ? (BMODE == B_Q4 ? 5 : 4) : (BN == 256 ? 6 : (BN == 192 ? 6 : 8));
   static constexpr int RAW_STAGE_BYTES = CONV ? (RAW_BYTES + SC_BYTES + 1023) / 1024 * 1024 : 0;
   static constexpr int RSTAGES_FIT =
