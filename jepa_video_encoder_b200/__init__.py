@@ -9,7 +9,7 @@ path: without the built library (or a CUDA device) the calls raise.
 from __future__ import annotations
 
 import ctypes
-from typing import List, Optional
+from typing import List, Optional, Tuple
 
 from . import _abi, synth
 from ._abi import JepaError, check, load_library
@@ -56,6 +56,47 @@ def check_pixels(cfg: "synth.EncoderConfig", pixels, on_cuda: bool, device: Opti
     return int(pixels.shape[0])
 
 
+def check_tokens(cfg: "synth.EncoderConfig", tokens, device: Optional[int] = None, on_cuda: bool = True) -> int:
+    """Validate the predictor's input, the encoder's last_hidden_state: a
+    contiguous float32 tensor [B, N, dim] on a CUDA device (``device``; the
+    host with on_cuda False) with B >= 1, N the encoder's tokens per clip and
+    dim its width (the library reads B * N * dim values from the pointer and
+    cannot see the tensor's size).  Returns B."""
+    import torch
+    if not isinstance(tokens, torch.Tensor) or tokens.is_cuda != on_cuda or tokens.dtype != torch.float32 \
+            or not tokens.is_contiguous() or (on_cuda and device is not None and tokens.device.index != device):
+        raise ValueError("tokens must be a contiguous float32 tensor on " + (f"cuda:{device}" if on_cuda else "the host"))
+    want = (cfg.n_tokens, cfg.dim)
+    if tokens.dim() != 3 or tuple(tokens.shape[1:]) != want or tokens.shape[0] < 1:
+        raise ValueError(f"tokens must be [B, {want[0]}, {want[1]}], got {list(tokens.shape)}")
+    return int(tokens.shape[0])
+
+
+def check_world_model_inputs(wc: "synth.WorldModelConfig", states, actions, steps: int = 0,
+                             device: Optional[int] = None, on_cuda: bool = True) -> Tuple[int, int]:
+    """Validate a world-model call's inputs: contiguous float32 tensors of
+    three dims on a CUDA device (``device``; the host with on_cuda False),
+    states [C, T, dim] with C, T >= 1, and actions [C, A_rows, action_dim]
+    with A_rows = T for a predictor call (steps 0) or T + steps - 1 for a
+    rollout of steps >= 1 (the library reads exactly those rows and cannot
+    see the tensors' sizes).  Returns (C, T)."""
+    import torch
+    for t, name in ((states, "states"), (actions, "actions")):
+        if not isinstance(t, torch.Tensor) or t.is_cuda != on_cuda or t.dtype != torch.float32 \
+                or not t.is_contiguous() or t.dim() != 3 or (on_cuda and device is not None and t.device.index != device):
+            raise ValueError(f"{name} must be a contiguous float32 tensor of 3 dims on "
+                             + (f"cuda:{device}" if on_cuda else "the host"))
+    C, T = int(states.shape[0]), int(states.shape[1])
+    if C < 1 or T < 1 or int(states.shape[2]) != wc.dim:
+        raise ValueError(f"states must be [C, T, {wc.dim}] with C, T >= 1, got {list(states.shape)}")
+    if steps < 0:
+        raise ValueError(f"steps must be >= 1 for a rollout, got {steps}")
+    rows = T if steps == 0 else T + steps - 1
+    if tuple(actions.shape) != (C, rows, wc.action_dim):
+        raise ValueError(f"actions must be [{C}, {rows}, {wc.action_dim}], got {list(actions.shape)}")
+    return C, T
+
+
 def check_out(out, on_cuda: bool, device: Optional[int] = None) -> None:
     """A caller-supplied output: float32, contiguous, on the same side as the
     pixels (its size is checked by the library against the pool mode)."""
@@ -97,6 +138,7 @@ class Model:
         lib = load_library()
         self.cfg = cfg
         self.device = device
+        self.world_model = world_model
         entries = (_abi.TensorEntry * len(table))()
         self._keep = []
         for i, t in enumerate(table):
@@ -176,12 +218,9 @@ class Model:
         float32 [B, len(tgt_idx), dim].  Asynchronous."""
         import numpy as np
         import torch
-        if not isinstance(tokens, torch.Tensor) or not tokens.is_cuda or tokens.dtype != torch.float32 \
-                or not tokens.is_contiguous() or tokens.dim() != 3 or tokens.device.index != self.device:
-            raise ValueError(f"tokens must be a contiguous float32 tensor [B, N, D] on cuda:{self.device}")
+        B = check_tokens(self.cfg, tokens, self.device)
         ci = np.ascontiguousarray(np.asarray(ctx_idx, dtype=np.int32))
         ti = np.ascontiguousarray(np.asarray(tgt_idx, dtype=np.int32))
-        B = int(tokens.shape[0])
         if out is None:
             out = torch.empty((B, len(ti), int(tokens.shape[2])), dtype=torch.float32, device=tokens.device)
         check_out(out, True, self.device)
@@ -190,20 +229,17 @@ class Model:
               "predict")
         return out
 
-    def _wm_in(self, t, name, ndim):
-        import torch
-        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous() \
-                or t.dim() != ndim or t.device.index != self.device:
-            raise ValueError(f"{name} must be a contiguous float32 tensor of {ndim} dims on cuda:{self.device}")
+    def _wm_cfg(self):
+        if self.world_model is None:
+            raise JepaError(_abi.ERR_ARG, "the model was loaded without a world model")
+        return self.world_model
 
     def lewm_predict(self, states, actions, out=None, stream=None):
         """LeWM predictor call: states CUDA float32 [C, T, dim], actions
         [C, T, action_dim] -> float32 [C, T, dim], row t the predicted state
         of frame t + 1.  Asynchronous."""
         import torch
-        self._wm_in(states, "states", 3)
-        self._wm_in(actions, "actions", 3)
-        C, T = int(states.shape[0]), int(states.shape[1])
+        C, T = check_world_model_inputs(self._wm_cfg(), states, actions, 0, self.device)
         if out is None:
             out = torch.empty((C, T, int(states.shape[2])), dtype=torch.float32, device=states.device)
         check_out(out, True, self.device)
@@ -217,9 +253,9 @@ class Model:
         actions [C, T0 + steps - 1, action_dim] -> float32 [C, steps, dim],
         the predicted states of frames T0 .. T0 + steps - 1.  Asynchronous."""
         import torch
-        self._wm_in(states, "states", 3)
-        self._wm_in(actions, "actions", 3)
-        C, T0 = int(states.shape[0]), int(states.shape[1])
+        if steps < 1:
+            raise ValueError(f"steps must be >= 1, got {steps}")
+        C, T0 = check_world_model_inputs(self._wm_cfg(), states, actions, steps, self.device)
         if out is None:
             out = torch.empty((C, steps, int(states.shape[2])), dtype=torch.float32, device=states.device)
         check_out(out, True, self.device)

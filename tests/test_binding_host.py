@@ -78,3 +78,45 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_abi, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         _abi.load_library(str(tmp_path / "libjepa_b200.so"))
+
+
+def test_check_tokens():
+    """The predictor's input must be [B, N, dim] of the loaded encoder: the
+    library reads B * N * dim values through the pointer."""
+    cfg = CFG
+    good = torch.zeros((2, cfg.n_tokens, cfg.dim))
+    assert jb.check_tokens(cfg, good, on_cuda=False) == 2
+    for bad in (torch.zeros((2, cfg.n_tokens - 1, cfg.dim)),     # fewer tokens than the encoder's
+                torch.zeros((2, cfg.n_tokens, cfg.dim + 64)),     # another width
+                torch.zeros((0, cfg.n_tokens, cfg.dim)),          # empty batch
+                torch.zeros((cfg.n_tokens, cfg.dim)),             # no batch axis
+                torch.zeros((2, cfg.n_tokens, cfg.dim), dtype=torch.float16),
+                torch.zeros((2, cfg.dim, cfg.n_tokens)).transpose(1, 2)):   # strided view
+        with pytest.raises(ValueError):
+            jb.check_tokens(cfg, bad, on_cuda=False)
+    with pytest.raises(ValueError):
+        jb.check_tokens(cfg, good, on_cuda=True, device=0)        # a host tensor where a device one is due
+
+
+def test_check_world_model_inputs():
+    """States [C, T, dim] and actions [C, T, A] for a predictor call, or
+    [C, T + steps - 1, A] for a rollout: the library reads exactly those
+    rows through the pointers."""
+    wc = synth.LEWM_WM_STEP
+    D, A = wc.dim, wc.action_dim
+    st, ac = torch.zeros((5, 3, D)), torch.zeros((5, 3, A))
+    assert jb.check_world_model_inputs(wc, st, ac, 0, on_cuda=False) == (5, 3)
+    assert jb.check_world_model_inputs(wc, st[:, :1].contiguous(), torch.zeros((5, 20, A)), 20,
+                                       on_cuda=False) == (5, 1)
+    bad = [(st, torch.zeros((5, 2, A)), 0),            # fewer action rows than frames
+           (st, torch.zeros((4, 3, A)), 0),            # candidates differ
+           (st, torch.zeros((5, 3, A + 1)), 0),        # another action width
+           (torch.zeros((5, 3, D + 64)), ac, 0),       # another state width
+           (torch.zeros((0, 3, D)), torch.zeros((0, 3, A)), 0),   # no candidates
+           (torch.zeros((5, 0, D)), torch.zeros((5, 0, A)), 0),   # no frames
+           (st, ac, 2),                                # a 2-step rollout from 3 frames reads 4 action rows
+           (st, ac, -1),
+           (st, ac.to(torch.float16), 0)]
+    for s_, a_, steps in bad:
+        with pytest.raises(ValueError):
+            jb.check_world_model_inputs(wc, s_, a_, steps, on_cuda=False)
