@@ -303,6 +303,42 @@ class Model:
 # ---------------------------------------------------------------------------
 # Single-kernel entry points (torch CUDA tensors in, asynchronous)
 # ---------------------------------------------------------------------------
+def _buf(t, nbytes: int, name: str) -> int:
+    """Device address of an operand of a single-op call, after checking that
+    it is a contiguous tensor of at least nbytes bytes: the library reads and
+    writes through the plain pointer the sizes that the call's dimensions
+    give, and cannot see the tensor's own."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    have = t.numel() * t.element_size()
+    if have < nbytes:
+        raise ValueError(f"{name} holds {have} bytes; the call's dimensions address {nbytes}")
+    return _dptr(t)
+
+
+def _opt(t, nbytes: int, name: str) -> Optional[int]:
+    return None if t is None else _buf(t, nbytes, name)
+
+
+def _weight_bytes(w_dtype: int, N: int, K: int) -> int:
+    """Bytes of a weight operand of op_linear / op_gemv: f16 [N, K], or the
+    repacked q8_0 codes [N, K] / q4_0 nibble bytes [N, K/2]."""
+    if w_dtype == synth.DT_Q8_0:
+        return N * K
+    if w_dtype == synth.DT_Q4_0:
+        return N * (K // 2)
+    if w_dtype == synth.DT_F32:
+        return N * K * 4
+    return N * K * 2
+
+
+def _scale_bytes(w_dtype: int, N: int, K: int) -> int:
+    return N * (K // 32) * 2 if w_dtype in (synth.DT_Q8_0, synth.DT_Q4_0) else 0
+
+
 def op_sync_status(stream=None) -> int:
     return int(load_library().jepa_b200_op_sync_status(_stream_ptr(stream)))
 
@@ -316,71 +352,96 @@ def layernorm(x, gamma, beta, eps: float, out, in_row_stride: int = 1, rows: Opt
     D = x.shape[-1]
     rows = out.numel() // D if rows is None else rows
     dt = synth.DT_F16 if out.dtype == torch.float16 else synth.DT_F32
-    check(load_library().jepa_b200_op_layernorm(_dptr(x), rows, D, in_row_stride, _dptr(gamma), _dptr(beta), eps,
-                                                _dptr(out), dt, _stream_ptr(stream)), "layernorm")
+    x_rows = (rows - 1) * in_row_stride + 1 if rows > 0 else 0
+    check(load_library().jepa_b200_op_layernorm(_buf(x, x_rows * D * 4, "x"), rows, D, in_row_stride,
+                                                _buf(gamma, D * 4, "gamma"), _buf(beta, D * 4, "beta"), eps,
+                                                _buf(out, rows * D * out.element_size(), "out"), dt,
+                                                _stream_ptr(stream)), "layernorm")
     return out
 
 
 def repack(dtype: int, blocks, N: int, K: int, qs, scales, stream=None):
-    check(load_library().jepa_b200_op_repack(dtype, _dptr(blocks), N, K, _dptr(qs), _dptr(scales),
+    block_bytes = 34 if dtype == synth.DT_Q8_0 else 18
+    check(load_library().jepa_b200_op_repack(dtype, _buf(blocks, N * (K // 32) * block_bytes, "blocks"), N, K,
+                                             _buf(qs, _weight_bytes(dtype, N, K), "qs"),
+                                             _buf(scales, _scale_bytes(dtype, N, K), "scales"),
                                              _stream_ptr(stream)), "repack")
 
 
 def dequant_f16(dtype: int, qs, scales, N: int, K: int, out, stream=None):
-    check(load_library().jepa_b200_op_dequant_f16(dtype, _dptr(qs), _dptr(scales), N, K, _dptr(out),
-                                                  _stream_ptr(stream)), "dequant_f16")
+    check(load_library().jepa_b200_op_dequant_f16(dtype, _buf(qs, _weight_bytes(dtype, N, K), "qs"),
+                                                  _buf(scales, _scale_bytes(dtype, N, K), "scales"), N, K,
+                                                  _buf(out, N * K * 2, "out"), _stream_ptr(stream)), "dequant_f16")
     return out
 
 
 def linear(A, w, w_dtype: int, N: int, bias, epilogue: int, out, w_scales=None, stream=None):
     M, K = A.shape
-    check(load_library().jepa_b200_op_linear(_dptr(A), M, K, _dptr(w), _dptr(w_scales) if w_scales is not None else None,
-                                             w_dtype, N, _dptr(bias) if bias is not None else None, epilogue,
-                                             _dptr(out), out.shape[-1], _stream_ptr(stream)), "linear")
+    ldo = out.shape[-1]
+    out_es = 2 if epilogue in (0, 1) else 4
+    check(load_library().jepa_b200_op_linear(_buf(A, M * K * 2, "A"), M, K, _buf(w, _weight_bytes(w_dtype, N, K), "w"),
+                                             _opt(w_scales, _scale_bytes(w_dtype, N, K), "w_scales"), w_dtype, N,
+                                             _opt(bias, N * 4, "bias"), epilogue, _buf(out, M * ldo * out_es, "out"),
+                                             ldo, _stream_ptr(stream)), "linear")
     return out
 
 
 def linear_qkv(A, w, w_dtype: int, N: int, bias, ntok: int, heads: int, npad: int, first_part: int, q, k, vt,
                w_scales=None, stream=None):
     M, K = A.shape
-    f = lambda t: _dptr(t) if t is not None else None
-    check(load_library().jepa_b200_op_linear_qkv(_dptr(A), M, K, _dptr(w), f(w_scales), w_dtype, N, f(bias), ntok,
-                                                 heads, npad, first_part, f(q), f(k), f(vt), _stream_ptr(stream)),
+    clips = M // ntok if ntok > 0 else 0
+    qk_bytes = clips * heads * ntok * 64 * 2
+    check(load_library().jepa_b200_op_linear_qkv(_buf(A, M * K * 2, "A"), M, K, _buf(w, _weight_bytes(w_dtype, N, K), "w"),
+                                                 _opt(w_scales, _scale_bytes(w_dtype, N, K), "w_scales"), w_dtype, N,
+                                                 _opt(bias, N * 4, "bias"), ntok, heads, npad, first_part,
+                                                 _opt(q, qk_bytes, "q"), _opt(k, qk_bytes, "k"),
+                                                 _opt(vt, clips * heads * 64 * npad * 2, "vt"), _stream_ptr(stream)),
           "linear_qkv")
 
 
 def attention(q, k, vt, B: int, heads: int, ntok: int, npad: int, mask: int, has_cls: int, ppf: int, out,
               stream=None):
-    check(load_library().jepa_b200_op_attention(_dptr(q), _dptr(k), _dptr(vt), B, heads, ntok, npad, mask, has_cls,
-                                                ppf, _dptr(out), _stream_ptr(stream)), "attention")
+    qk_bytes = B * heads * ntok * 64 * 2
+    check(load_library().jepa_b200_op_attention(_buf(q, qk_bytes, "q"), _buf(k, qk_bytes, "k"),
+                                                _buf(vt, B * heads * 64 * npad * 2, "vt"), B, heads, ntok, npad, mask,
+                                                has_cls, ppf, _buf(out, B * ntok * heads * 64 * 2, "out"),
+                                                _stream_ptr(stream)), "attention")
     return out
 
 
 def patch_embed(pixels, patch: int, tubelet: int, w_pe, D: int, bias, pos, cls, has_cls: int, x, stream=None):
     B, T, _, H, W = pixels.shape
-    check(load_library().jepa_b200_op_patch_embed(_dptr(pixels), B, T, H, W, patch, tubelet, _dptr(w_pe), D,
-                                                  _dptr(bias) if bias is not None else None, _dptr(pos),
-                                                  _dptr(cls) if cls is not None else None, has_cls, _dptr(x),
-                                                  _stream_ptr(stream)), "patch_embed")
+    if patch < 1 or tubelet < 1:
+        raise ValueError("patch and tubelet must be positive")
+    kpad = (3 * tubelet * patch * patch + 63) // 64 * 64
+    ntok = (1 if has_cls else 0) + (T // tubelet) * (H // patch) * (W // patch)
+    check(load_library().jepa_b200_op_patch_embed(_buf(pixels, pixels.numel() * 4, "pixels"), B, T, H, W, patch,
+                                                  tubelet, _buf(w_pe, D * kpad * 2, "w_pe"), D,
+                                                  _opt(bias, D * 4, "bias"), _buf(pos, ntok * D * 4, "pos"),
+                                                  _opt(cls, D * 4 if has_cls else 0, "cls"), has_cls,
+                                                  _buf(x, B * ntok * D * 4, "x"), _stream_ptr(stream)), "patch_embed")
     return x
 
 
 def gemv(x, w, w_dtype: int, N: int, bias, epi: int, y, resid=None, resid_row_stride: int = 0, w_scales=None,
          stream=None):
     M, K = x.shape
-    f = lambda t: _dptr(t) if t is not None else None
-    check(load_library().jepa_b200_op_gemv(_dptr(x), M, K, _dptr(w), f(w_scales), w_dtype, N, f(bias), epi, f(resid),
-                                           resid_row_stride, _dptr(y), _stream_ptr(stream)), "gemv")
+    resid_bytes = ((M - 1) * resid_row_stride + N) * 4 if M > 0 else 0
+    check(load_library().jepa_b200_op_gemv(_buf(x, M * K * 4, "x"), M, K, _buf(w, _weight_bytes(w_dtype, N, K), "w"),
+                                           _opt(w_scales, _scale_bytes(w_dtype, N, K), "w_scales"), w_dtype, N,
+                                           _opt(bias, N * 4, "bias"), epi, _opt(resid, resid_bytes, "resid"),
+                                           resid_row_stride, _buf(y, M * N * 4, "y"), _stream_ptr(stream)), "gemv")
     return y
 
 
 def xattn_1q(q, k, vt, B: int, heads: int, ntok: int, npad: int, out, stream=None):
-    check(load_library().jepa_b200_op_xattn_1q(_dptr(q), _dptr(k), _dptr(vt), B, heads, ntok, npad, _dptr(out),
-                                               _stream_ptr(stream)), "xattn_1q")
+    check(load_library().jepa_b200_op_xattn_1q(_buf(q, heads * 64 * 4, "q"), _buf(k, B * heads * ntok * 64 * 2, "k"),
+                                               _buf(vt, B * heads * 64 * npad * 2, "vt"), B, heads, ntok, npad,
+                                               _buf(out, B * heads * 64 * 4, "out"), _stream_ptr(stream)), "xattn_1q")
     return out
 
 
 def mean_pool(y, B: int, ntok: int, D: int, first: int, out, stream=None):
-    check(load_library().jepa_b200_op_mean_pool(_dptr(y), B, ntok, D, first, _dptr(out), _stream_ptr(stream)),
-          "mean_pool")
+    check(load_library().jepa_b200_op_mean_pool(_buf(y, B * ntok * D * 4, "y"), B, ntok, D, first,
+                                                _buf(out, B * D * 4, "out"), _stream_ptr(stream)), "mean_pool")
     return out

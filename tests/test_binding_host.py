@@ -120,3 +120,24 @@ def test_check_world_model_inputs():
     for s_, a_, steps in bad:
         with pytest.raises(ValueError):
             jb.check_world_model_inputs(wc, s_, a_, steps, on_cuda=False)
+
+
+def test_single_op_operand_sizes():
+    """The single-op wrappers check each operand's bytes against what the
+    call's dimensions address before handing the pointer over: a short
+    tensor is refused on the host (here before the device check)."""
+    with pytest.raises(ValueError, match="holds 40 bytes"):
+        jb._buf(torch.zeros(10), 41, "x")
+    with pytest.raises(ValueError, match="contiguous"):
+        jb._buf(torch.zeros((4, 4)).t(), 4, "x")
+    with pytest.raises(ValueError, match="CUDA"):
+        jb._buf(torch.zeros(10), 40, "x")                     # big enough, but on the host
+    # weight operands: f16 [N, K], q8_0 codes [N, K], q4_0 nibbles [N, K/2], f16 scales [N, K/32]
+    assert jb._weight_bytes(synth.DT_F16, 128, 256) == 128 * 256 * 2
+    assert jb._weight_bytes(synth.DT_Q8_0, 128, 256) == 128 * 256
+    assert jb._weight_bytes(synth.DT_Q4_0, 128, 256) == 128 * 128
+    assert jb._scale_bytes(synth.DT_Q4_0, 128, 256) == 128 * 8 * 2
+    assert jb._scale_bytes(synth.DT_F16, 128, 256) == 0
+    # mean pool of 2 clips x 10 tokens x 64 from a 9-token buffer
+    with pytest.raises(ValueError, match="y holds"):
+        jb.mean_pool(torch.zeros((2, 9, 64)), 2, 10, 64, 1, torch.zeros((2, 64)))
