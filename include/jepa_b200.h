@@ -413,8 +413,8 @@ JEPA_B200_API int jepa_b200_op_mean_pool(const float *y, int B, int ntok, int D,
  * y f32 [B, ntok, D] -> out f32 [B, D] (mean over rows first..ntok-1), device
  * pointers.  Limit: B * D <= 32768; larger sizes return ERR_SHAPE before any
  * device work.  The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress) with that device current; make that first
- * call before any stream capture.  Every call shares the array and overwrites
+ * address (cudaGetSymbolAddress) with that device current and keeps it for
+ * the later calls on that device.  Every call shares the array and overwrites
  * the partial sums it reads, so its previous contents never matter, but calls
  * that overlap on the GPU (two streams, two host threads) race on it.
  * Returns OK, ERR_ARG, ERR_SHAPE or ERR_CUDA. */
