@@ -55,7 +55,7 @@ typedef enum {
   JEPA_B200_ERR_DTYPE = -4,          /* dtype not allowed for that tensor */
   JEPA_B200_ERR_CUDA = -5,           /* a CUDA runtime/driver call failed */
   JEPA_B200_ERR_TIMEOUT = -6,        /* a bounded device-side wait ran out; the kernel unwound */
-  JEPA_B200_ERR_UNSUPPORTED = -7     /* valid request this build does not implement */
+  JEPA_B200_ERR_UNSUPPORTED = -7     /* valid request the library does not implement */
 } jepa_b200_status;
 
 /* Tensor dtypes use ggml's type ids (0 f32, 1 f16, 2 q4_0, 8 q8_0), the
